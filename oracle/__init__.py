@@ -1,0 +1,156 @@
+"""Q4 oracle: ctypes wrapper around the scalar C reference in ``q4_oracle.c``.
+
+TEST INFRASTRUCTURE. Only the tests, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline / reference leg may import this package.  The product
+library never links or calls it, and it imports nothing from the product.
+
+Format and products follow the QORA-4B thread (zingnex.cn, section
+"量化与内存管理") and the QORA-LLM-0.8B model card (section "Weight Format"):
+4-bit symmetric quantisation, group size 32, one scale per group, products
+against the dequantised weights.  The exact encoding is written out in the
+header comment of ``q4_oracle.c``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "q4_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+FLAG_NONFINITE = 1
+FLAG_SCALE_OVERFLOW = 2
+
+_CFLAGS = ["-O2", "-fno-fast-math", "-ffp-contract=off", "-fopenmp", "-fPIC", "-shared", "-std=c11"]
+
+
+def build(force: bool = False) -> str:
+    """Compile ``q4_oracle.c`` into ``liboracle.so`` next to it (gcc, no SIMD flags)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", *_CFLAGS, _SRC, "-o", tmp, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        lib = ctypes.CDLL(build())
+        i64, vp, i32 = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int
+        lib.oracle_f32_to_f16.argtypes = [ctypes.c_float]
+        lib.oracle_f32_to_f16.restype = ctypes.c_uint16
+        lib.oracle_f16_to_f32.argtypes = [ctypes.c_uint16]
+        lib.oracle_f16_to_f32.restype = ctypes.c_float
+        lib.oracle_bf16_to_f32.argtypes = [ctypes.c_uint16]
+        lib.oracle_bf16_to_f32.restype = ctypes.c_float
+        lib.oracle_f32_to_f16_array.argtypes = [vp, vp, i64]
+        lib.oracle_f32_to_f16_array.restype = None
+        lib.oracle_f16_to_f32_array.argtypes = [vp, vp, i64]
+        lib.oracle_f16_to_f32_array.restype = None
+        lib.oracle_q4_quantize.argtypes = [vp, i64, i64, vp, vp, vp]
+        lib.oracle_q4_quantize.restype = i32
+        lib.oracle_q4_dequant.argtypes = [vp, vp, i64, i64, vp]
+        lib.oracle_q4_dequant.restype = None
+        lib.oracle_q4_matmul_rows.argtypes = [vp, i32, i64, i64, vp, vp, vp, i64, vp, i32]
+        lib.oracle_q4_matmul_rows.restype = i32
+        lib.oracle_q4_matmul.argtypes = [vp, i32, i64, i64, vp, vp, i64, vp, i32]
+        lib.oracle_q4_matmul.restype = i32
+        lib.oracle_max_threads.argtypes = []
+        lib.oracle_max_threads.restype = i32
+        _lib = lib
+        return lib
+
+
+def _ptr(a: np.ndarray) -> int:
+    return a.ctypes.data
+
+
+def f32_to_f16_bits(x) -> np.ndarray:
+    """IEEE binary16 round-to-nearest-even of each f32 value, as uint16 bits."""
+    a = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.empty(a.shape, dtype=np.uint16)
+    _load().oracle_f32_to_f16_array(_ptr(a), _ptr(out), a.size)
+    return out
+
+
+def f16_bits_to_f32(h) -> np.ndarray:
+    a = np.ascontiguousarray(h, dtype=np.uint16)
+    out = np.empty(a.shape, dtype=np.float32)
+    _load().oracle_f16_to_f32_array(_ptr(a), _ptr(out), a.size)
+    return out
+
+
+def quantize(W: np.ndarray):
+    """W f32 [N,K] -> (packed uint8 [N,K/2], scales uint16 binary16 bits [N,K/32], flags)."""
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    N, K = W.shape
+    if K % 32:
+        raise ValueError("K must be a multiple of 32")
+    packed = np.empty((N, K // 2), dtype=np.uint8)
+    scales = np.empty((N, K // 32), dtype=np.uint16)
+    flags = np.zeros(1, dtype=np.uint32)
+    rc = _load().oracle_q4_quantize(_ptr(W), N, K, _ptr(packed), _ptr(scales), _ptr(flags))
+    if rc != 0:
+        raise RuntimeError("oracle quantize failed")
+    return packed, scales, int(flags[0])
+
+
+def dequantize(packed: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """Exact binary64 dequantised weights [N,K]."""
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint16)
+    N, K = packed.shape[0], packed.shape[1] * 2
+    out = np.empty((N, K), dtype=np.float64)
+    _load().oracle_q4_dequant(_ptr(packed), _ptr(scales), N, K, _ptr(out))
+    return out
+
+
+def matmul(x: np.ndarray, packed: np.ndarray, scales: np.ndarray, rows=None, threads: int = 1) -> np.ndarray:
+    """y = x . dequant(W)^T in binary64.
+
+    x: [M,K] float32, or uint16 holding bfloat16 bits.  rows: optional subset of
+    output rows (int64 indices); the result then has shape [M, len(rows)].
+    """
+    if x.dtype == np.uint16:
+        is_bf16 = 1
+    elif x.dtype == np.float32:
+        is_bf16 = 0
+    else:
+        raise TypeError("x must be float32 or uint16 (bfloat16 bits)")
+    x = np.ascontiguousarray(x)
+    if x.ndim == 1:
+        x = x[None, :]
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint16)
+    M, K = x.shape
+    N = packed.shape[0]
+    if packed.shape[1] * 2 != K or scales.shape != (N, K // 32):
+        raise ValueError("shape mismatch between x, packed and scales")
+    lib = _load()
+    if rows is None:
+        y = np.empty((M, N), dtype=np.float64)
+        rc = lib.oracle_q4_matmul(_ptr(x), is_bf16, M, K, _ptr(packed), _ptr(scales), N, _ptr(y), threads)
+    else:
+        r = np.ascontiguousarray(rows, dtype=np.int64)
+        if r.size and (r.min() < 0 or r.max() >= N):
+            raise IndexError("row index out of range")
+        y = np.empty((M, r.size), dtype=np.float64)
+        rc = lib.oracle_q4_matmul_rows(_ptr(x), is_bf16, M, K, _ptr(packed), _ptr(scales),
+                                       _ptr(r), r.size, _ptr(y), threads)
+    if rc != 0:
+        raise MemoryError("oracle matmul: allocation failed")
+    return y
+
+
+def max_threads() -> int:
+    return int(_load().oracle_max_threads())
