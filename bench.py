@@ -1,0 +1,527 @@
+#!/usr/bin/env python3
+"""Benchmark of the Q4 (4-bit symmetric, group-32) decode GEMV on B200.
+
+Headline workload: the QORA-4B-shaped decode projections -- M=1, K=2560,
+N in {2048, 4096, 1024}, weights N(0, 0.02^2) with 1% outlier groups, bf16 x.
+One step = one GEMV per projection (3 launches) against resident Q4 weights.
+Metric: effective GB/s = algorithmic bytes (packed codes + binary16 scales + x +
+f32 y) / device time.  L2 stays cold: every step reads a different copy of the
+weights, and the copies together exceed 3x the L2 size.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--rows all|main]
+
+Prints one JSON line (rank 0).  Under torchrun each rank runs its own
+independent problem (weak scaling, no collective on the data path); the time is
+the max over ranks.  --impl reference times the CPU oracle instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth_inputs  # noqa: E402
+
+METRIC = "Q4 GEMV effective GB/s"
+UNIT = "GB/s"
+MAIN = synth_inputs.DECODE_PROJ
+WORKLOAD = ("decode projections M=1 K=2560 N={2048,4096,1024} (QORA-4B shaped), "
+            "Q4 group-32 weights N(0,0.02^2) with 1% outlier groups, bf16 x, f32 y")
+
+
+def gemv_bytes(M, N, K, x_bytes=2):
+    return N * K // 2 + N * (K // 32) * 2 + M * K * x_bytes + M * N * 4
+
+
+STEP_BYTES = sum(gemv_bytes(w.M, w.N, w.K) for w in MAIN)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(path))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def kernel_source_hash(name):
+    p = os.path.join(ROOT, "bit_weight_only_quantize_b200", "csrc", name)
+    return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
+
+
+def recorded_traffic(kernel, workload, src_file):
+    """DRAM bytes per launch from the committed ncu summary, if taken on this source."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    want = kernel_source_hash(src_file)
+    for line in open(path):
+        f = dict(kv.split("=", 1) for kv in line.split() if "=" in kv)
+        if f.get("kernel") == kernel and f.get("workload") == workload and f.get("src") == want:
+            return float(f["bytes_per_launch"])
+    return None
+
+
+# ---------------------------------------------------------------- clocks (NVML)
+REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+           0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+           0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    def __init__(self, torch_device):
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self.ok = False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            bus = torch.cuda.get_device_properties(torch_device).pci_bus_id
+            self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report no clocks rather than guessing
+            self.err = str(e)
+
+    def sample(self):
+        if not self.ok:
+            return
+        try:
+            self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+            self.reasons |= int(self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+        except Exception:
+            pass
+
+    def _run(self):
+        while not self._stop.is_set():
+            self.sample()
+            time.sleep(0.001)
+
+    def start(self):
+        self.samples, self.reasons = [], 0
+        self._stop.clear()
+        self.t = threading.Thread(target=self._run, daemon=True)
+        self.t.start()
+
+    def stop(self):
+        self._stop.set()
+        self.t.join()
+
+    def report(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "error": getattr(self, "err", "")}
+        names = [n for b, n in REASONS.items() if self.reasons & b and b != 0x1]
+        med = statistics.median(self.samples) if self.samples else None
+        return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------- device side
+def setup_dist(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def make_quantized(torch, q4, w, seed, device):
+    W = synth_inputs.weights(w.weights, w.N, w.K, seed)
+    Wd = torch.from_numpy(W).to(device)
+    packed, scales = q4.quantize(Wd)
+    del Wd
+    return W, packed, scales
+
+
+class DecodeStep:
+    """The three projections, with C rotating copies of their Q4 weights."""
+
+    def __init__(self, torch, q4, lib, rank, device, l2_bytes):
+        self.torch, self.lib = torch, lib
+        self.device = device
+        self.mats = []
+        set_bytes = 0
+        for w in MAIN:
+            W, packed, scales = make_quantized(torch, q4, w, rank, device)
+            self.mats.append((w, W, packed, scales))
+            set_bytes += packed.numel() + scales.numel() * 2
+        self.copies = max(2, -(-3 * l2_bytes // set_bytes) + 1)
+        self.pk = [[p] + [p.clone() for _ in range(self.copies - 1)] for (_, _, p, _) in self.mats]
+        self.sc = [[s] + [s.clone() for _ in range(self.copies - 1)] for (_, _, _, s) in self.mats]
+        self.rotated_bytes = set_bytes * self.copies
+        x = synth_inputs.activations(1, 2560, "bf16", rank)
+        self.x_np = x
+        self.x = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(device)
+        self.y = [torch.empty((1, w.N), dtype=torch.float32, device=device) for (w, *_) in self.mats]
+        need = max(q4.gemv_workspace_size(1, w.N, w.K) for w in MAIN)
+        self.ws = torch.zeros(max(need, 16), dtype=torch.uint8, device=device)
+
+    def launch(self, step, stream_handle):
+        c = step % self.copies
+        for j, (w, *_rest) in enumerate(self.mats):
+            st = self.lib.q4_gemv(self.x.data_ptr(), 1, 1, w.K, self.pk[j][c].data_ptr(), self.sc[j][c].data_ptr(),
+                                  w.N, self.y[j].data_ptr(), self.ws.data_ptr(), self.ws.numel(), stream_handle)
+            if st != 0:
+                raise RuntimeError(f"q4_gemv failed with status {st}")
+
+    def check(self):
+        """Max relative error of the last outputs on sampled rows, against the oracle."""
+        import oracle
+        worst = 0.0
+        for j, (w, W, packed, scales) in enumerate(self.mats):
+            rows = np.linspace(0, w.N - 1, 64).astype(np.int64)
+            pk = packed.cpu().numpy().view(np.uint8)
+            sc = scales.cpu().numpy().view(np.uint16)
+            ref = oracle.matmul(self.x_np, pk, sc, rows=rows)
+            got = self.y[j].cpu().numpy()[:, rows]
+            worst = max(worst, float(np.max(np.abs(got - ref)) / max(np.max(np.abs(ref)), 1e-30)))
+        return worst
+
+
+def timed_graph(torch, launch, steps, period, stream):
+    """Capture `period` steps in one CUDA graph (and the remainder in another) and
+    return a function that replays exactly `steps` steps."""
+    graphs = []
+    full, rem = divmod(steps, period)
+    with torch.cuda.stream(stream):
+        def capture(n, base):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for i in range(n):
+                    launch(base + i, stream.cuda_stream)
+            return g
+        g_full = capture(period, 0) if full else None
+        g_rem = capture(rem, 0) if rem else None
+
+    def run():
+        for _ in range(full):
+            g_full.replay()
+        if g_rem is not None:
+            g_rem.replay()
+    graphs.extend([g_full, g_rem])
+    return run, graphs
+
+
+def measure_main(torch, q4, lib, args, world, rank, device, peaks, dist):
+    props = torch.cuda.get_device_properties(device)
+    l2 = int(getattr(props, "L2_cache_size", 126 * 2 ** 20))
+    step = DecodeStep(torch, q4, lib, rank, device, l2)
+    stream = torch.cuda.Stream(device=device)
+    # warm-up (eager, through the same C ABI), then capture
+    for i in range(args.warmup):
+        step.launch(i, stream.cuda_stream)
+    torch.cuda.synchronize(device)
+    period = step.copies * max(1, 64 // step.copies)
+    run, graphs = timed_graph(torch, step.launch, args.steps, period, stream)
+    run()                                  # one untimed pass of the graphs
+    torch.cuda.synchronize(device)
+
+    clocks = ClockSampler(device)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize(device)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    clocks.start()
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        run()
+    e1.record(stream)
+    clocks.sample()
+    torch.cuda.synchronize(device)
+    clocks.stop()
+    if dist is not None:
+        dist.barrier()
+    ms = e0.elapsed_time(e1)
+    ms_max = ms
+    if dist is not None:
+        t = torch.tensor([ms], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_max = float(t.item())
+    err = step.check()
+    del graphs
+    return step, ms_max, clocks.report(), err
+
+
+def measure_e2e(torch, q4, step, steps, device, dist=None, world=1):
+    """Same metric through the public Python API, per step: pinned x -> device,
+    the three GEMVs, outputs -> pinned host, host waits for the result."""
+    n = max(1, min(steps, 2000))
+    x_host = torch.from_numpy(step.x_np.view(np.int16)).view(torch.bfloat16).pin_memory()
+    y_host = [torch.empty(y.shape, dtype=y.dtype).pin_memory() for y in step.y]
+    x_dev = torch.empty_like(step.x)
+    stream = torch.cuda.current_stream(device)
+
+    def one(i):
+        c = i % step.copies
+        x_dev.copy_(x_host, non_blocking=True)
+        for j, (w, *_r) in enumerate(step.mats):
+            q4.gemv(x_dev, step.pk[j][c], step.sc[j][c], out=step.y[j], workspace=step.ws)
+        for j in range(len(step.mats)):
+            y_host[j].copy_(step.y[j], non_blocking=True)
+        stream.synchronize()
+
+    for i in range(3):
+        one(i)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(n):
+        one(i)
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    ms = e0.elapsed_time(e1) / n
+    if dist is not None:
+        t = torch.tensor([ms], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    return {"value": world * STEP_BYTES / (ms * 1e-3) / 1e9, "unit": UNIT,
+            "h2d_bytes_per_step": x_host.numel() * 2,
+            "d2h_bytes_per_step": sum(y.numel() * 4 for y in y_host),
+            "steps": n, "ms_per_step": ms, "api": "bit_weight_only_quantize_b200.gemv (pinned host buffers)"}
+
+
+def time_launches(torch, fn, n, device, stream):
+    """Average device time of fn() over n launches captured in one graph."""
+    with torch.cuda.stream(stream):
+        fn(0)
+    torch.cuda.synchronize(device)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(n):
+                fn(i)
+    g.replay()
+    torch.cuda.synchronize(device)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    return e0.elapsed_time(e1) / n
+
+
+def measure_rows(torch, q4, lib, device, peaks, l2):
+    """Every other hot-path row of the library at its configuration, one GPU."""
+    out = {}
+    stream = torch.cuda.Stream(device=device)
+    hbm = peaks["hbm_gbs"]
+
+    # LM head: 358.6 MB per launch, already larger than L2.
+    w = synth_inputs.LM_HEAD
+    W, packed, scales = make_quantized(torch, q4, w, 0, device)
+    x = torch.from_numpy(synth_inputs.activations(1, w.K, "bf16", 0).view(np.int16)).view(torch.bfloat16).to(device)
+    y = torch.empty((1, w.N), dtype=torch.float32, device=device)
+    ws_n = q4.gemv_workspace_size(1, w.N, w.K)
+    ws = torch.zeros(max(ws_n, 16), dtype=torch.uint8, device=device)
+
+    def lm(i):
+        st = lib.q4_gemv(x.data_ptr(), 1, 1, w.K, packed.data_ptr(), scales.data_ptr(), w.N, y.data_ptr(),
+                         ws.data_ptr(), ws.numel(), stream.cuda_stream)
+        assert st == 0
+    ms = time_launches(torch, lm, 20, device, stream)
+    b = gemv_bytes(1, w.N, w.K)
+    out["lm_head_gemv"] = {"workload": "M=1 K=2560 N=248320 bf16 x", "ms": ms, "GB/s": b / ms / 1e6,
+                           "frac_hbm": b / ms / 1e6 / hbm, "bytes": b, "launches": 20}
+
+    # Quantise the LM-head weights: reads 4 B and writes 0.5625 B per weight.
+    Wd = torch.from_numpy(W).to(device)
+    del W
+    pk2 = torch.empty_like(packed)
+    sc2 = torch.empty_like(scales)
+
+    def qz(i):
+        st = lib.q4_quantize(Wd.data_ptr(), w.N, w.K, pk2.data_ptr(), sc2.data_ptr(), None, stream.cuda_stream)
+        assert st == 0
+    ms = time_launches(torch, qz, 5, device, stream)
+    b = w.N * w.K * 4 + w.N * w.K // 2 + w.N * (w.K // 32) * 2
+    out["quantize"] = {"workload": "W f32 248320x2560 -> Q4", "ms": ms, "GB/s": b / ms / 1e6,
+                       "frac_hbm": b / ms / 1e6 / hbm, "bytes": b, "launches": 5,
+                       "bit_exact_vs_first_encode": bool(torch.equal(pk2, packed) and torch.equal(sc2, scales))}
+    del Wd, pk2, sc2, packed, scales
+
+    # Small-batch decode M in {2,4,8,16}, N=4096, rotating copies for a cold L2.
+    for sw in synth_inputs.SMALL_BATCH:
+        _, packed, scales = make_quantized(torch, q4, sw, 0, device)
+        setb = packed.numel() + scales.numel() * 2
+        copies = max(2, -(-3 * l2 // setb) + 1)
+        pks = [packed] + [packed.clone() for _ in range(copies - 1)]
+        scs = [scales] + [scales.clone() for _ in range(copies - 1)]
+        xs = torch.from_numpy(synth_inputs.activations(sw.M, sw.K, "bf16", 0).view(np.int16)).view(
+            torch.bfloat16).to(device)
+        ys = torch.empty((sw.M, sw.N), dtype=torch.float32, device=device)
+        need = q4.gemv_workspace_size(sw.M, sw.N, sw.K)
+        wss = torch.zeros(max(need, 16), dtype=torch.uint8, device=device)
+
+        def sb(i, pks=pks, scs=scs, xs=xs, ys=ys, wss=wss, sw=sw, copies=copies):
+            c = i % copies
+            st = lib.q4_gemv(xs.data_ptr(), 1, sw.M, sw.K, pks[c].data_ptr(), scs[c].data_ptr(), sw.N,
+                             ys.data_ptr(), wss.data_ptr(), wss.numel(), stream.cuda_stream)
+            assert st == 0
+        ms = time_launches(torch, sb, copies * 4, device, stream)
+        b = gemv_bytes(sw.M, sw.N, sw.K)
+        out[f"gemv_m{sw.M}"] = {"workload": f"M={sw.M} K=2560 N=4096 bf16 x", "ms": ms, "GB/s": b / ms / 1e6,
+                                "frac_hbm": b / ms / 1e6 / hbm, "bytes": b, "launches": copies * 4}
+        del pks, scs
+    torch.cuda.synchronize(device)
+    return out
+
+
+def cpu_baseline(seconds=10.0):
+    """The oracle as it stands, on all host cores, over the headline workload."""
+    import oracle
+    threads = os.cpu_count() or 1
+    mats = []
+    for w in MAIN:
+        W = synth_inputs.weights(w.weights, w.N, w.K, 0)
+        packed, scales, _ = oracle.quantize(W)
+        mats.append((w, packed, scales))
+    x = synth_inputs.activations(1, 2560, "bf16", 0)
+    t0 = time.perf_counter()
+    passes = 0
+    while True:
+        for w, packed, scales in mats:
+            oracle.matmul(x, packed, scales, threads=threads)
+        passes += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": STEP_BYTES * passes / dt / 1e9, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{passes} full passes of the three decode projections (binary64 oracle, "
+                      f"OpenMP over rows), {dt:.1f} s"}
+
+
+def run_reference(args, world, rank):
+    """The oracle timed on the host as the reference arm (rank 0 only)."""
+    if rank != 0:
+        return
+    import oracle
+    threads = os.cpu_count() or 1
+    mats = []
+    for w in MAIN:
+        W = synth_inputs.weights(w.weights, w.N, w.K, 0)
+        packed, scales, _ = oracle.quantize(W)
+        mats.append((w, packed, scales))
+    x = synth_inputs.activations(1, 2560, "bf16", 0)
+
+    def step(frac):
+        b = 0
+        for w, packed, scales in mats:
+            n = max(1, int(round(w.N * frac)))
+            rows = np.arange(n, dtype=np.int64)
+            oracle.matmul(x, packed, scales, rows=rows, threads=threads)
+            b += gemv_bytes(1, n, w.K)
+        return b
+
+    t0 = time.perf_counter()
+    step(1.0)
+    t_full = time.perf_counter() - t0
+    budget = 120.0
+    frac = min(1.0, budget / max(1e-9, t_full * (args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        step(frac)
+    t0 = time.perf_counter()
+    total = 0
+    for _ in range(args.steps):
+        total += step(frac)
+    dt = time.perf_counter() - t0
+    value = total / dt / 1e9
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "reference": "CPU oracle (scalar C, binary64), no GPU"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": f"{frac:.4f} of the rows of each projection per step"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--rows", choices=["all", "main"], default="all")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world, rank, local = setup_dist(args)
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+
+    import torch
+    import bit_weight_only_quantize_b200 as q4
+    from bit_weight_only_quantize_b200 import _lib
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist_mod
+        dist_mod.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+        dist = dist_mod
+    lib = _lib.load()
+    peaks = load_peaks()
+
+    step, ms, clocks, err = measure_main(torch, q4, lib, args, world, rank, device, peaks, dist)
+    ms_step = ms / args.steps
+    value = world * STEP_BYTES * args.steps / (ms * 1e-3) / 1e9
+    per_gpu = STEP_BYTES / (ms_step * 1e-3) / 1e9
+    launches = 3 * args.steps
+    traffic = recorded_traffic("gemv_ffma_kernel", "decode_proj", "gemv.cu")
+    roofline = {"bound": "hbm", "achieved": per_gpu, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": per_gpu / peaks["hbm_gbs"], "traffic": traffic,
+                "peak_source": f"{peaks['source']} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
+                "kernel": "gemv_ffma_kernel", "algorithmic_bytes_per_launch": STEP_BYTES / 3,
+                "avg_launch_us": ms * 1e3 / launches}
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "bytes_per_step": STEP_BYTES,
+                       "l2": f"rotating {step.copies} weight copies = {step.rotated_bytes / 1e6:.0f} MB "
+                             f"(> 3x L2) so every step reads cold weights",
+                       "timing": "CUDA graph of the steps, CUDA events on the launching stream, max over ranks",
+                       "parallelism": f"replicas x{world} (independent problems, no collective)",
+                       "check_max_rel_err_sampled_rows": err},
+            "roofline": roofline, "gpu_launches": launches, "clocks": clocks}
+    if dist is not None:
+        dist.barrier()
+    line["e2e"] = measure_e2e(torch, q4, step, args.steps, device, dist, world)
+    if world == 1:
+        del step
+        torch.cuda.empty_cache()
+        if args.rows == "all":
+            props = torch.cuda.get_device_properties(device)
+            l2 = int(getattr(props, "L2_cache_size", 126 * 2 ** 20))
+            line["rows"] = measure_rows(torch, q4, lib, device, peaks, l2)
+        line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

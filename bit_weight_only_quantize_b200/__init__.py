@@ -1,0 +1,99 @@
+"""B200 (sm_100a) Q4 weight-only quantisation: quantise, decode GEMV, prefill GEMM.
+
+Thin torch-facing wrappers over the C ABI in ``include/q4.h``.  torch supplies
+device memory and the current stream; every step of the computation runs in the
+library's CUDA kernels.  The weight format is 4-bit symmetric with one binary16
+scale per group of 32 weights along K (QORA-4B thread, section "量化与内存管理";
+QORA-LLM-0.8B model card, section "Weight Format").
+"""
+from __future__ import annotations
+
+import torch
+
+from . import _lib
+from ._lib import Q4Error, FLAG_NONFINITE, FLAG_SCALE_OVERFLOW, GEMV_MAX_M  # noqa: F401
+
+__all__ = [
+    "quantize", "gemv", "gemv_workspace_size", "Q4Error", "FLAG_NONFINITE", "FLAG_SCALE_OVERFLOW",
+    "GEMV_MAX_M",
+]
+
+
+def _stream() -> int:
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _need(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must have dtype {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dimensions")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def quantize(W: torch.Tensor, flags: torch.Tensor | None = None):
+    """f32 W[N,K] -> (packed uint8 [N,K/2], scales binary16 as int16 bits [N,K/32]).
+
+    ``flags`` (optional int32 tensor of one element) receives the OR of the
+    Q4 flag bits; it is not cleared first.
+    """
+    _need(W, "W", torch.float32, 2)
+    N, K = W.shape
+    packed = torch.empty((N, K // 2), dtype=torch.uint8, device=W.device)
+    scales = torch.empty((N, max(K // 32, 0)), dtype=torch.int16, device=W.device)
+    fptr = None
+    if flags is not None:
+        _need(flags, "flags", torch.int32, 1)
+        fptr = flags.data_ptr()
+    with torch.cuda.device(W.device):
+        st = _lib.load().q4_quantize(W.data_ptr(), N, K, packed.data_ptr(), scales.data_ptr(), fptr, _stream())
+    _lib.check(st, "q4_quantize")
+    return packed, scales
+
+
+def gemv_workspace_size(M: int, N: int, K: int) -> int:
+    return int(_lib.load().q4_gemv_workspace_size(M, N, K))
+
+
+def gemv(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, out: torch.Tensor | None = None,
+         workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """y[M,N] (f32) = x[M,K] . dequant(W)^T for M <= 16; x is float32 or bfloat16.
+
+    ``workspace`` (uint8, zero-filled before first use) is allocated here when
+    the shape needs one and none is given.
+    """
+    if x.dtype == torch.float32:
+        xt = _lib.Q4_F32
+    elif x.dtype == torch.bfloat16:
+        xt = _lib.Q4_BF16
+    else:
+        raise TypeError("x must be float32 or bfloat16")
+    _need(x, "x", x.dtype, 2)
+    _need(packed, "packed", torch.uint8, 2)
+    _need(scales, "scales", torch.int16, 2)
+    M, K = x.shape
+    N = packed.shape[0]
+    if packed.shape[1] * 2 != K or tuple(scales.shape) != (N, K // 32):
+        raise ValueError("shape mismatch between x, packed and scales")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float32, device=x.device)
+    else:
+        _need(out, "out", torch.float32, 2)
+        if tuple(out.shape) != (M, N):
+            raise ValueError("out has the wrong shape")
+    lib = _lib.load()
+    with torch.cuda.device(x.device):
+        need = int(lib.q4_gemv_workspace_size(M, N, K))
+        if need and workspace is None:
+            workspace = torch.zeros(need, dtype=torch.uint8, device=x.device)
+        ws_ptr = workspace.data_ptr() if workspace is not None else None
+        ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+        st = lib.q4_gemv(x.data_ptr(), xt, M, K, packed.data_ptr(), scales.data_ptr(), N,
+                         out.data_ptr(), ws_ptr, ws_bytes, _stream())
+    _lib.check(st, "q4_gemv")
+    return out

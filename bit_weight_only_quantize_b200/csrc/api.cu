@@ -1,0 +1,137 @@
+// C ABI of the library (declared in include/q4.h): argument validation, device
+// checks and dispatch to the kernels.  Every argument check happens before the
+// first CUDA call, so a bad call returns its status without touching the device.
+#include <stdint.h>
+
+#include <mutex>
+
+#include "q4_common.cuh"
+
+namespace q4 {
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::once_flag g_once[kMaxDevices];
+DeviceInfo g_info[kMaxDevices];
+q4_status g_info_status[kMaxDevices];
+
+void query(int dev)
+{
+    DeviceInfo d = {};
+    d.device = dev;
+    q4_status st = Q4_OK;
+    if (cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.cc_minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.l2_bytes, cudaDevAttrL2CacheSize, dev) != cudaSuccess) {
+        cudaGetLastError();
+        st = Q4_ERR_CUDA;
+    } else if (d.cc_major != 10 || d.cc_minor != 0) {
+        st = Q4_ERR_UNSUPPORTED_DEVICE;    // the kernels are built for sm_100a only
+    }
+    g_info[dev] = d;
+    g_info_status[dev] = st;
+}
+}  // namespace
+
+q4_status current_device(DeviceInfo* out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return Q4_ERR_CUDA;
+    }
+    if (dev < 0 || dev >= kMaxDevices) return Q4_ERR_UNSUPPORTED_DEVICE;
+    std::call_once(g_once[dev], query, dev);
+    *out = g_info[dev];
+    return g_info_status[dev];
+}
+
+}  // namespace q4
+
+namespace {
+
+bool misaligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) != 0; }
+
+// K: positive multiple of 32; N >= 0; both small enough for 32-bit row/group indices.
+q4_status check_nk(int64_t N, int64_t K)
+{
+    if (N < 0 || K < 32 || (K % 32) != 0) return Q4_ERR_SHAPE;
+    if (N > INT32_MAX || K > INT32_MAX || N > (INT64_C(1) << 62) / K) return Q4_ERR_SHAPE;
+    return Q4_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int q4_abi_version(void) { return 1; }
+
+const char* q4_status_string(q4_status status)
+{
+    switch (status) {
+    case Q4_OK: return "Q4_OK";
+    case Q4_ERR_INVALID_ARG: return "Q4_ERR_INVALID_ARG: a required pointer is NULL or an enum is out of range";
+    case Q4_ERR_SHAPE: return "Q4_ERR_SHAPE: K must be a positive multiple of 32, N >= 0, M in range";
+    case Q4_ERR_ALIGN: return "Q4_ERR_ALIGN: a pointer violates its documented alignment";
+    case Q4_ERR_DTYPE: return "Q4_ERR_DTYPE: unsupported data type";
+    case Q4_ERR_WORKSPACE: return "Q4_ERR_WORKSPACE: workspace missing or too small";
+    case Q4_ERR_CUDA: return "Q4_ERR_CUDA: a CUDA call or kernel launch failed";
+    case Q4_ERR_UNSUPPORTED_DEVICE: return "Q4_ERR_UNSUPPORTED_DEVICE: the current device is not sm_100";
+    }
+    return "Q4_ERR_UNKNOWN";
+}
+
+q4_status q4_quantize(const float* W, int64_t N, int64_t K, uint8_t* packed, uint16_t* scales,
+                      uint32_t* flags, void* stream)
+{
+    q4_status st = check_nk(N, K);
+    if (st != Q4_OK) return st;
+    if (N == 0) return Q4_OK;
+    if (!W || !packed || !scales) return Q4_ERR_INVALID_ARG;
+    if (misaligned(W, 16) || misaligned(packed, 16) || misaligned(scales, 2) || (flags && misaligned(flags, 4)))
+        return Q4_ERR_ALIGN;
+    q4::DeviceInfo dev;
+    if ((st = q4::current_device(&dev)) != Q4_OK) return st;
+    return q4::launch_quantize(W, N, K, packed, scales, flags, static_cast<cudaStream_t>(stream), dev);
+}
+
+size_t q4_gemv_workspace_size(int64_t M, int64_t N, int64_t K)
+{
+    if (M < 1 || M > Q4_GEMV_MAX_M || N < 1 || check_nk(N, K) != Q4_OK) return 0;
+    q4::DeviceInfo dev;
+    if (q4::current_device(&dev) != Q4_OK) return 0;
+    q4::GemvPlan plan;
+    if (!q4::plan_gemv(M, N, K, Q4_BF16, dev, &plan)) return 0;
+    q4::GemvPlan plan32;
+    if (!q4::plan_gemv(M, N, K, Q4_F32, dev, &plan32)) return 0;
+    return plan.workspace_bytes > plan32.workspace_bytes ? plan.workspace_bytes : plan32.workspace_bytes;
+}
+
+q4_status q4_gemv(const void* x, q4_dtype x_dtype, int64_t M, int64_t K, const uint8_t* packed,
+                  const uint16_t* scales, int64_t N, float* y, void* workspace, size_t workspace_bytes,
+                  void* stream)
+{
+    if (x_dtype != Q4_F32 && x_dtype != Q4_BF16) return Q4_ERR_DTYPE;
+    if (M < 0 || M > Q4_GEMV_MAX_M) return Q4_ERR_SHAPE;
+    q4_status st = check_nk(N, K);
+    if (st != Q4_OK) return st;
+    if (M == 0 || N == 0) return Q4_OK;
+    if (!x || !packed || !scales || !y) return Q4_ERR_INVALID_ARG;
+    if (misaligned(x, 16) || misaligned(packed, 16) || misaligned(scales, 2) || misaligned(y, 4) ||
+        (workspace && misaligned(workspace, 16)))
+        return Q4_ERR_ALIGN;
+    q4::DeviceInfo dev;
+    if ((st = q4::current_device(&dev)) != Q4_OK) return st;
+    q4::GemvPlan plan;
+    if (!q4::plan_gemv(M, N, K, x_dtype, dev, &plan)) {
+        cudaGetLastError();
+        return Q4_ERR_CUDA;
+    }
+    if (plan.workspace_bytes > 0 && (!workspace || workspace_bytes < plan.workspace_bytes)) return Q4_ERR_WORKSPACE;
+    return q4::launch_gemv(x, x_dtype, M, K, packed, scales, N, y, workspace, plan,
+                           static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

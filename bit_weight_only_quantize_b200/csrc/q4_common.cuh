@@ -1,0 +1,53 @@
+// Shared declarations of the CUDA library (internal; not part of the ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "q4.h"
+
+namespace q4 {
+
+struct DeviceInfo {
+    int device;
+    int sm_count;
+    int cc_major;
+    int cc_minor;
+    int max_smem_optin;     // bytes of dynamic shared memory one block may opt into
+    int l2_bytes;
+};
+
+// Attributes of the current device, cached per device id.  Returns Q4_ERR_CUDA on
+// failure and Q4_ERR_UNSUPPORTED_DEVICE when the device is not sm_100.
+q4_status current_device(DeviceInfo* out);
+
+// Launch wrappers (defined next to their kernels).  Arguments are already
+// validated by the ABI layer.
+q4_status launch_quantize(const float* W, int64_t N, int64_t K, uint8_t* packed, uint16_t* scales,
+                          uint32_t* flags, cudaStream_t stream, const DeviceInfo& dev);
+
+struct GemvPlan {
+    int kernel;             // which GEMV kernel family serves the shape
+    int splits;             // K splits across thread blocks (1 = none)
+    int groups_per_split;   // 32-wide groups of K each split covers
+    int row_blocks;         // blocks of rows
+    int grid_x;             // thread blocks per split
+    int smem_bytes;         // dynamic shared memory per block
+    size_t workspace_bytes; // partial sums + counters (0 when splits == 1)
+};
+
+bool plan_gemv(int64_t M, int64_t N, int64_t K, q4_dtype xt, const DeviceInfo& dev, GemvPlan* plan);
+q4_status launch_gemv(const void* x, q4_dtype xt, int64_t M, int64_t K, const uint8_t* packed,
+                      const uint16_t* scales, int64_t N, float* y, void* workspace,
+                      const GemvPlan& plan, cudaStream_t stream);
+
+// Programmatic dependent launch: a kernel launched with the programmatic
+// stream-serialisation attribute may start before its predecessor finishes;
+// pdl_wait() blocks until the predecessor has completed and its writes are
+// visible, and must precede every global read or write of the kernel.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+}  // namespace q4

@@ -1,0 +1,131 @@
+/*
+ * q4.h - C ABI of the B200 (sm_100a) Q4 weight-only quantisation library.
+ *
+ * Weight format.  The QORA-4B thread (zingnex.cn, section "量化与内存管理") and
+ * the QORA-LLM-0.8B model card (section "Weight Format") quantise weights to
+ * 4 bits, symmetrically, in groups of 32 along the reduction axis K, with one
+ * scale per group.  They leave the encoding details open; this library fixes
+ * them as follows, for a weight matrix W[N,K] (row n = one output feature):
+ *
+ *   for every row n and group g (the 32 values W[n, 32g .. 32g+31]):
+ *     amax = max |w|                               exact
+ *     s    = binary16_rne( f32(amax) / 7 )         IEEE f32 division, then round to
+ *                                                  nearest even into binary16
+ *     if s == +0: every code is 8 (each byte 0x88) and the stored scale is 0x0000
+ *     else:      code_k = clamp(rint_even(w_k / f32(s)), -8, 7) + 8   (f32 division)
+ *   packed[n, k/2] = code_{2i} | code_{2i+1} << 4   (low nibble = even k)
+ *   scales[n, g]   = s (binary16 bit pattern)
+ *   dequantised weight w'[n,k] = (code - 8) * f32(s)
+ *
+ * A group holding a NaN or an infinity, or whose scale would round to binary16
+ * infinity (amax/7 >= 65520), is stored as a zero group and reported through the
+ * flag word (Q4_FLAG_NONFINITE, Q4_FLAG_SCALE_OVERFLOW).
+ *
+ * Products.  The pages run "multi-threaded GEMV/GEMM" against these weights
+ * (model card, "Weight Format"; "File Structure": GEMV/GEMM kernels for Q4,
+ * prefill).  Here:
+ *   y[m, n] = sum_k x[m, k] * w'[n, k]        (x row-major [M,K], y row-major [M,N])
+ * q4_gemv serves decode (M = 1..16: one token, or a few tokens verified together).
+ *
+ * Conventions for every entry point:
+ *  - Pointers named d_* / documented as device pointers must point to device
+ *    memory of the current CUDA device.  The caller allocates and owns every
+ *    buffer; the library allocates nothing and keeps no state between calls
+ *    except cached device attributes.
+ *  - All matrices are dense, contiguous and row-major.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Work is
+ *    enqueued asynchronously; argument errors are returned synchronously before
+ *    anything is enqueued; a launch failure returns Q4_ERR_CUDA.
+ *  - No entry point traps, asserts or aborts.  Functions are thread-safe;
+ *    calls that share an output or workspace buffer must not overlap in time.
+ */
+#ifndef Q4_H
+#define Q4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define Q4_API __attribute__((visibility("default")))
+#else
+#define Q4_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum q4_status {
+    Q4_OK = 0,
+    Q4_ERR_INVALID_ARG = 1,        /* a required pointer is NULL, or an enum is out of range */
+    Q4_ERR_SHAPE = 2,              /* K not a positive multiple of 32, N < 0, M out of range */
+    Q4_ERR_ALIGN = 3,              /* a pointer violates its documented alignment */
+    Q4_ERR_DTYPE = 4,              /* unsupported data type for this entry point */
+    Q4_ERR_WORKSPACE = 5,          /* workspace missing or smaller than required */
+    Q4_ERR_CUDA = 6,               /* a CUDA runtime call or kernel launch failed */
+    Q4_ERR_UNSUPPORTED_DEVICE = 7  /* current device is not compute capability 10.0 */
+} q4_status;
+
+typedef enum q4_dtype {
+    Q4_F32 = 0,
+    Q4_BF16 = 1                    /* bfloat16, passed as its 16-bit pattern */
+} q4_dtype;
+
+#define Q4_FLAG_NONFINITE 1u
+#define Q4_FLAG_SCALE_OVERFLOW 2u
+
+#define Q4_GEMV_MAX_M 16
+
+/* Version of this ABI (incremented on any incompatible change). */
+Q4_API int q4_abi_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+Q4_API const char* q4_status_string(q4_status status);
+
+/*
+ * q4_quantize: encode W[N,K] (f32, device) into the Q4 format above.
+ *   W       device, f32 [N,K], 16-byte aligned.
+ *   N, K    N >= 0 (N == 0 enqueues nothing and returns Q4_OK);
+ *           K >= 32 and K % 32 == 0.
+ *   packed  device, uint8 [N, K/2], 16-byte aligned (output).
+ *   scales  device, binary16 bits [N, K/32], 2-byte aligned (output).
+ *   flags   device uint32 or NULL.  When given, the kernel ORs Q4_FLAG_* bits
+ *           into *flags; the caller clears it beforehand if it wants only this
+ *           call's flags.
+ * The result is bit-identical to the definition above for every input.
+ */
+Q4_API q4_status q4_quantize(const float* W, int64_t N, int64_t K,
+                      uint8_t* packed, uint16_t* scales, uint32_t* flags, void* stream);
+
+/*
+ * Bytes of workspace q4_gemv needs for this shape (0 when none).  When the
+ * shape is split along K across thread blocks, the workspace holds the f32
+ * partial sums and one arrival counter per block of rows.
+ */
+Q4_API size_t q4_gemv_workspace_size(int64_t M, int64_t N, int64_t K);
+
+/*
+ * q4_gemv: y = x . dequant(W)^T for M = 1..16 (decode).
+ *   x          device, [M,K] f32 or bfloat16 (x_dtype), 16-byte aligned.
+ *   M          0 .. Q4_GEMV_MAX_M (M == 0 or N == 0 enqueues nothing).
+ *   K, N       as for q4_quantize.
+ *   packed, scales  the Q4 encoding of W[N,K] (16-byte / 2-byte aligned).
+ *   y          device, f32 [M,N], 4-byte aligned (output, overwritten).
+ *   workspace  device, at least q4_gemv_workspace_size(M,N,K) bytes, 16-byte
+ *              aligned; may be NULL when that size is 0.  It must be zero-filled
+ *              before its first use.  Every completed call leaves the part that
+ *              must start at zero (the arrival counters) at zero again, so the
+ *              same workspace can be reused by later calls without clearing.
+ *              Calls that share a workspace must not overlap on the GPU.
+ * Arithmetic: codes are expanded exactly, each group's 32 products are summed in
+ * f32, multiplied by the group scale and accumulated in f32.
+ */
+Q4_API q4_status q4_gemv(const void* x, q4_dtype x_dtype, int64_t M, int64_t K,
+                  const uint8_t* packed, const uint16_t* scales, int64_t N,
+                  float* y, void* workspace, size_t workspace_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* Q4_H */

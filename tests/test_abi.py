@@ -1,0 +1,90 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports every
+symbol include/q4.h declares, and rejects bad arguments before touching a device."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from bit_weight_only_quantize_b200 import _lib, build
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "q4.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return re.findall(r"^Q4_API\s+[\w\s\*]+?\b(q4_\w+)\s*\(", text, flags=re.M)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _lib.load()
+
+
+def test_header_declares_expected(lib):
+    names = declared_functions()
+    assert set(names) == set(_lib.SIGNATURES), names
+
+
+def test_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
+
+
+def test_version_and_strings(lib):
+    assert lib.q4_abi_version() == 1
+    for code in range(8):
+        s = lib.q4_status_string(code).decode()
+        assert s.startswith(_lib.STATUS_NAMES[code])
+    assert lib.q4_status_string(99).decode() == "Q4_ERR_UNKNOWN"
+
+
+# Fake, never-dereferenced addresses: every call below fails validation first.
+A16 = 1 << 20
+A8 = A16 + 8
+
+
+def test_quantize_validation(lib):
+    S = None
+    assert lib.q4_quantize(A16, 4, 48, A16, A16, None, S) == 2          # K % 32
+    assert lib.q4_quantize(A16, 4, 0, A16, A16, None, S) == 2           # K == 0
+    assert lib.q4_quantize(A16, -1, 64, A16, A16, None, S) == 2         # N < 0
+    assert lib.q4_quantize(None, 4, 64, A16, A16, None, S) == 1         # NULL W
+    assert lib.q4_quantize(A16, 4, 64, None, A16, None, S) == 1
+    assert lib.q4_quantize(A8, 4, 64, A16, A16, None, S) == 3           # misaligned W
+    assert lib.q4_quantize(A16, 4, 64, A8, A16, None, S) == 3
+    assert lib.q4_quantize(A16, 4, 64, A16, A16 + 1, None, S) == 3
+    assert lib.q4_quantize(A16, 4, 64, A16, A16, A16 + 2, S) == 3
+    assert lib.q4_quantize(None, 0, 64, None, None, None, S) == 0       # empty: no-op
+
+
+def test_gemv_validation(lib):
+    S = None
+    assert lib.q4_gemv(A16, 7, 1, 64, A16, A16, 8, A16, None, 0, S) == 4        # dtype
+    assert lib.q4_gemv(A16, 1, 17, 64, A16, A16, 8, A16, None, 0, S) == 2       # M > 16
+    assert lib.q4_gemv(A16, 1, -1, 64, A16, A16, 8, A16, None, 0, S) == 2
+    assert lib.q4_gemv(A16, 1, 1, 40, A16, A16, 8, A16, None, 0, S) == 2        # K % 32
+    assert lib.q4_gemv(None, 1, 1, 64, A16, A16, 8, A16, None, 0, S) == 1
+    assert lib.q4_gemv(A16, 1, 1, 64, A16, A16, 8, None, None, 0, S) == 1
+    assert lib.q4_gemv(A8, 1, 1, 64, A16, A16, 8, A16, None, 0, S) == 3        # x alignment
+    assert lib.q4_gemv(A16, 1, 1, 64, A8, A16, 8, A16, None, 0, S) == 3        # packed alignment
+    assert lib.q4_gemv(A16, 1, 1, 64, A16, A16 + 1, 8, A16 + 2, None, 0, S) == 3
+    assert lib.q4_gemv(A16, 1, 1, 64, A16, A16, 8, A16, A8, 64, S) == 3       # workspace alignment
+    assert lib.q4_gemv(None, 1, 0, 64, None, None, 8, None, None, 0, S) == 0   # M == 0: no-op
+    assert lib.q4_gemv(None, 1, 3, 64, None, None, 0, None, None, 0, S) == 0   # N == 0: no-op
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_no_device_reports_cuda_error(lib):
+    assert lib.q4_quantize(A16, 4, 64, A16, A16, None, None) == 6
+    assert lib.q4_gemv(A16, 1, 1, 64, A16, A16, 8, A16, None, 0, None) == 6
+    assert lib.q4_gemv_workspace_size(1, 8, 64) == 0
+
+
+def test_binding_raises_without_gpu_tensors():
+    import bit_weight_only_quantize_b200 as q4
+    with pytest.raises(ValueError):
+        q4.quantize(torch.zeros(4, 64))
