@@ -17,6 +17,7 @@ the max over ranks.  --impl reference times the CPU oracle instead (rank 0 only)
 from __future__ import annotations
 
 import argparse
+import faulthandler
 import hashlib
 import json
 import os
@@ -31,6 +32,12 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 import synth_inputs  # noqa: E402
+
+faulthandler.enable()
+
+
+def log(msg):
+    print(f"[bench] {msg}", file=sys.stderr, flush=True)
 
 METRIC = "Q4 GEMV effective GB/s"
 UNIT = "GB/s"
@@ -92,8 +99,8 @@ class ClockSampler:
             import pynvml
             import torch
             pynvml.nvmlInit()
-            bus = torch.cuda.get_device_properties(torch_device).pci_bus_id
-            self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(torch_device).uuid)
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid.encode())
             self.nv = pynvml
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
             self.ok = True
@@ -220,28 +227,37 @@ def timed_graph(torch, launch, steps, period, stream):
 def measure_main(torch, q4, lib, args, world, rank, device, peaks, dist):
     props = torch.cuda.get_device_properties(device)
     l2 = int(getattr(props, "L2_cache_size", 126 * 2 ** 20))
+    log("setup: quantising the decode projections")
     step = DecodeStep(torch, q4, lib, rank, device, l2)
+    log(f"setup done: {step.copies} rotating copies")
     stream = torch.cuda.Stream(device=device)
     # warm-up (eager, through the same C ABI), then capture
     for i in range(args.warmup):
         step.launch(i, stream.cuda_stream)
     torch.cuda.synchronize(device)
+    log("warm-up done; capturing graphs")
     period = step.copies * max(1, 64 // step.copies)
     run, graphs = timed_graph(torch, step.launch, args.steps, period, stream)
-    run()                                  # one untimed pass of the graphs
+    log("captured; untimed replay")
+    with torch.cuda.stream(stream):
+        run()                              # one untimed pass of the graphs
     torch.cuda.synchronize(device)
+    log("replay ok; timing")
 
     clocks = ClockSampler(device)
+    log(f"clock sampler ok={clocks.ok}")
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize(device)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     clocks.start()
+    torch.cuda.nvtx.range_push("timed_main")
     e0.record(stream)
     with torch.cuda.stream(stream):
         run()
     e1.record(stream)
+    torch.cuda.nvtx.range_pop()
     clocks.sample()
     torch.cuda.synchronize(device)
     clocks.stop()
@@ -253,6 +269,7 @@ def measure_main(torch, q4, lib, args, world, rank, device, peaks, dist):
         t = torch.tensor([ms], dtype=torch.float64, device=device)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms_max = float(t.item())
+    log(f"timed {ms:.3f} ms; checking outputs")
     err = step.check()
     del graphs
     return step, ms_max, clocks.report(), err
@@ -306,13 +323,14 @@ def time_launches(torch, fn, n, device, stream):
         with torch.cuda.graph(g, stream=stream):
             for i in range(n):
                 fn(i)
-    g.replay()
-    torch.cuda.synchronize(device)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    g.replay()
-    e1.record(stream)
+    with torch.cuda.stream(stream):          # replay on the stream the events are recorded on
+        g.replay()
+        torch.cuda.synchronize(device)
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
     torch.cuda.synchronize(device)
     return e0.elapsed_time(e1) / n
 
@@ -335,6 +353,7 @@ def measure_rows(torch, q4, lib, device, peaks, l2):
         st = lib.q4_gemv(x.data_ptr(), 1, 1, w.K, packed.data_ptr(), scales.data_ptr(), w.N, y.data_ptr(),
                          ws.data_ptr(), ws.numel(), stream.cuda_stream)
         assert st == 0
+    log("rows: lm head")
     ms = time_launches(torch, lm, 20, device, stream)
     b = gemv_bytes(1, w.N, w.K)
     out["lm_head_gemv"] = {"workload": "M=1 K=2560 N=248320 bf16 x", "ms": ms, "GB/s": b / ms / 1e6,
@@ -349,6 +368,7 @@ def measure_rows(torch, q4, lib, device, peaks, l2):
     def qz(i):
         st = lib.q4_quantize(Wd.data_ptr(), w.N, w.K, pk2.data_ptr(), sc2.data_ptr(), None, stream.cuda_stream)
         assert st == 0
+    log("rows: quantize")
     ms = time_launches(torch, qz, 5, device, stream)
     b = w.N * w.K * 4 + w.N * w.K // 2 + w.N * (w.K // 32) * 2
     out["quantize"] = {"workload": "W f32 248320x2560 -> Q4", "ms": ms, "GB/s": b / ms / 1e6,
@@ -374,6 +394,7 @@ def measure_rows(torch, q4, lib, device, peaks, l2):
             st = lib.q4_gemv(xs.data_ptr(), 1, sw.M, sw.K, pks[c].data_ptr(), scs[c].data_ptr(), sw.N,
                              ys.data_ptr(), wss.data_ptr(), wss.numel(), stream.cuda_stream)
             assert st == 0
+        log(f"rows: gemv m={sw.M}")
         ms = time_launches(torch, sb, copies * 4, device, stream)
         b = gemv_bytes(sw.M, sw.N, sw.K)
         out[f"gemv_m{sw.M}"] = {"workload": f"M={sw.M} K=2560 N=4096 bf16 x", "ms": ms, "GB/s": b / ms / 1e6,
@@ -507,6 +528,7 @@ def main():
             "roofline": roofline, "gpu_launches": launches, "clocks": clocks}
     if dist is not None:
         dist.barrier()
+    log("e2e")
     line["e2e"] = measure_e2e(torch, q4, step, args.steps, device, dist, world)
     if world == 1:
         del step
@@ -514,7 +536,9 @@ def main():
         if args.rows == "all":
             props = torch.cuda.get_device_properties(device)
             l2 = int(getattr(props, "L2_cache_size", 126 * 2 ** 20))
+            log("other rows")
             line["rows"] = measure_rows(torch, q4, lib, device, peaks, l2)
+        log("cpu baseline")
         line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
     if rank == 0:
         print(json.dumps(line), flush=True)

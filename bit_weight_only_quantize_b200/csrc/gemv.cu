@@ -20,11 +20,13 @@
 //  * x is staged once per block in shared memory as f32; the eight 16-byte chunks
 //    of group g sit at slots c ^ (g & 7) so the 8 lanes of a load phase hit
 //    distinct banks.
-//  * Skinny shapes split K across blocks (grid.y).  Each block writes f32 partial
-//    sums to the workspace, then bumps the row block's arrival counter; the block
-//    that arrives last adds the partials in split order (a fixed order, so the
-//    result does not depend on timing), writes y and resets the counter.  Nobody
-//    waits on anybody.
+//  * Skinny shapes (fewer row blocks than SMs) split K across blocks (grid.y).
+//    Each block writes f32 partial sums to the workspace, then bumps the row
+//    block's arrival counter; the block that arrives last adds the partials in
+//    split order (a fixed order, so the result does not depend on timing), writes
+//    y and resets the counter.  Nobody waits on anybody.
+//  * When x for a split does not fit the shared-memory budget it is staged in
+//    pieces of whole chunks; the block restages when its work crosses a piece.
 #include "q4_common.cuh"
 
 namespace q4 {
@@ -47,7 +49,17 @@ struct GemvArgs {
     int ksg;               // groups per split
     int splits;
     int row_blocks;
+    int chunk;             // groups per work unit (<= kSlots * kTeam)
+    int xcap;              // groups of x held in shared memory at once (multiple of chunk)
 };
+
+// Workspace layout (shape independent, so one workspace serves every shape):
+// [0, kCounterBytes) arrival counters, one per row block of a split launch; they
+// must be zero before the first call and every call leaves them zero.  Splits
+// are only used when there are fewer row blocks than SMs, so kCounterSlots
+// bounds the count.  Partial sums follow.
+constexpr int kCounterSlots = 1024;
+constexpr size_t kCounterBytes = kCounterSlots * sizeof(unsigned);
 
 __device__ __forceinline__ uint4 load_weights(const uint8_t* p)
 {
@@ -87,10 +99,40 @@ __device__ __forceinline__ float4 load_x4(const void* x, size_t idx)
     }
 }
 
+// Loads of one work unit: row block rb, chunk ch (groups ch*chunk .. of this split).
+__device__ __forceinline__ void load_unit(const GemvArgs& a, int rb, int ch, int g0, int ng, int team, int lane16,
+                                          uint4 (&w)[kSlots], uint32_t (&sc)[kSlots])
+{
+    const int row = rb * kTeams + team;
+#pragma unroll
+    for (int j = 0; j < kSlots; ++j) {
+        const int lg = ch * a.chunk + j * kTeam + lane16;
+        if (row < a.N && j * kTeam < a.chunk && lg < ng) {
+            const size_t gg = (size_t)row * a.G + g0 + lg;
+            w[j] = load_weights(a.packed + gg * 16);
+            sc[j] = a.scales[gg];
+        }
+    }
+}
+
+// x[:, 32*gbase .. 32*(gbase+n)) -> shared memory as f32; rows m >= M are zero.
+template <int MT, bool XBF16>
+__device__ __forceinline__ void stage_x(const GemvArgs& a, float4* xs, int gbase, int n, int per_m, size_t K)
+{
+    for (int i = threadIdx.x; i < MT * n * 8; i += kThreads) {
+        const int m = i / (n * 8);
+        const int r = i - m * (n * 8);
+        const int lg = r >> 3, c = r & 7;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (m < a.M) v = load_x4<XBF16>(a.x, (size_t)m * K + (size_t)(gbase + lg) * 32 + c * 4);
+        xs[m * per_m + lg * 8 + (c ^ (lg & 7))] = v;
+    }
+}
+
 template <int MT, bool XBF16>
 __global__ void __launch_bounds__(kThreads, 2) gemv_ffma_kernel(const GemvArgs a)
 {
-    extern __shared__ float4 xs[];               // [MT][ng][8] float4, chunk-swizzled per group
+    extern __shared__ float4 xs[];               // [MT][xcap][8] float4, chunk-swizzled per group
     __shared__ int s_last;
 
     const int tid = threadIdx.x;
@@ -100,106 +142,122 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_ffma_kernel(const GemvArgs a
     const int g0 = split * a.ksg;
     const int ng = min(a.G - g0, a.ksg);
     const size_t K = (size_t)a.G * 32;
+    const int nchunks = (ng + a.chunk - 1) / a.chunk;
+    const int chunks_per_stage = a.xcap / a.chunk;
+    const int per_m = min(ng, a.xcap) * 8;       // float4 per x row in shared memory
 
     pdl_launch_dependents();
     pdl_wait();
+    int rb = blockIdx.x, ch = 0;
+    if (rb >= a.row_blocks) return;
 
-    // Stage x[:, 32*g0 .. 32*(g0+ng)) as f32; rows m >= M are zero.
-    const int per_m = ng * 8;
-    for (int i = tid; i < MT * per_m; i += kThreads) {
-        const int m = i / per_m;
-        const int r = i - m * per_m;
-        const int lg = r >> 3, c = r & 7;
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (m < a.M) v = load_x4<XBF16>(a.x, (size_t)m * K + (size_t)(g0 + lg) * 32 + c * 4);
-        xs[m * per_m + lg * 8 + (c ^ (lg & 7))] = v;
-    }
-    __syncthreads();
+    // The first unit's weight loads go out before x is staged, so the two
+    // latencies overlap; afterwards each unit's loads go out before the
+    // previous unit is computed.
+    uint4 w[kSlots];
+    uint32_t sc[kSlots];
+    load_unit(a, rb, ch, g0, ng, team, lane16, w, sc);
+    int staged = -1;
+    float yacc[MT];
+#pragma unroll
+    for (int m = 0; m < MT; ++m) yacc[m] = 0.f;
 
-    const int nchunks = (ng + kChunkGroups - 1) / kChunkGroups;
-    for (int rb = blockIdx.x; rb < a.row_blocks; rb += gridDim.x) {
+    while (true) {
+        const int stage = ch / chunks_per_stage;
+        if (stage != staged) {
+            if (staged >= 0) __syncthreads();    // the previous stage is no longer read
+            const int gb = stage * a.xcap;
+            stage_x<MT, XBF16>(a, xs, g0 + gb, min(a.xcap, ng - gb), per_m, K);
+            __syncthreads();
+            staged = stage;
+        }
+        int nrb = rb, nch = ch + 1;
+        if (nch == nchunks) {
+            nch = 0;
+            nrb += gridDim.x;
+        }
+        const bool has_next = nrb < a.row_blocks;
+        uint4 wn[kSlots];
+        uint32_t scn[kSlots];
+        if (has_next) load_unit(a, nrb, nch, g0, ng, team, lane16, wn, scn);
+
         const int row = rb * kTeams + team;
         const bool row_ok = row < a.N;
-        float yacc[MT];
 #pragma unroll
-        for (int m = 0; m < MT; ++m) yacc[m] = 0.f;
-
-        for (int ch = 0; ch < nchunks; ++ch) {
-            uint4 w[kSlots];
-            uint32_t sc[kSlots];
+        for (int j = 0; j < kSlots; ++j) {
+            const int lg = ch * a.chunk + j * kTeam + lane16;        // group within the split
+            if (row_ok && j * kTeam < a.chunk && lg < ng) {
+                const int ls = lg - stage * a.xcap;                    // group within the stage
+                const float s = __half2float(__ushort_as_half((unsigned short)sc[j]));
+                const float4* xg = xs + ls * 8;
+                const int sw = ls & 7;
+                float2 acc[MT];
 #pragma unroll
-            for (int j = 0; j < kSlots; ++j) {
-                const int lg = ch * kChunkGroups + j * kTeam + lane16;
-                if (row_ok && lg < ng) {
-                    const size_t gg = (size_t)row * a.G + g0 + lg;
-                    w[j] = load_weights(a.packed + gg * 16);
-                    sc[j] = a.scales[gg];
+                for (int m = 0; m < MT; ++m) acc[m] = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int wd = 0; wd < 4; ++wd) {
+                    const uint32_t v = wd == 0 ? w[j].x : wd == 1 ? w[j].y : wd == 2 ? w[j].z : w[j].w;
+                    float2 d01, d23, d45, d67;
+                    expand8(v, d01, d23, d45, d67);
+#pragma unroll
+                    for (int m = 0; m < MT; ++m) {
+                        const float4 xa = xg[m * per_m + ((2 * wd) ^ sw)];
+                        const float4 xb = xg[m * per_m + ((2 * wd + 1) ^ sw)];
+                        acc[m] = __ffma2_rn(make_float2(xa.x, xa.y), d01, acc[m]);
+                        acc[m] = __ffma2_rn(make_float2(xa.z, xa.w), d23, acc[m]);
+                        acc[m] = __ffma2_rn(make_float2(xb.x, xb.y), d45, acc[m]);
+                        acc[m] = __ffma2_rn(make_float2(xb.z, xb.w), d67, acc[m]);
+                    }
                 }
+#pragma unroll
+                for (int m = 0; m < MT; ++m) yacc[m] = fmaf(s, acc[m].x + acc[m].y, yacc[m]);
             }
+        }
+
+        if (nch == 0) {                          // row block rb is complete
+            // Team reduction: after it every lane of the team holds the row's sums.
 #pragma unroll
-            for (int j = 0; j < kSlots; ++j) {
-                const int lg = ch * kChunkGroups + j * kTeam + lane16;
-                if (row_ok && lg < ng) {
-                    const float s = __half2float(__ushort_as_half((unsigned short)sc[j]));
-                    const float4* xg = xs + lg * 8;
-                    const int sw = lg & 7;
-                    float2 acc[MT];
+            for (int m = 0; m < MT; ++m) {
 #pragma unroll
-                    for (int m = 0; m < MT; ++m) acc[m] = make_float2(0.f, 0.f);
+                for (int o = kTeam / 2; o > 0; o >>= 1) yacc[m] += __shfl_xor_sync(0xffffffffu, yacc[m], o);
+            }
+            float mine = 0.f;                    // lane m keeps output m
 #pragma unroll
-                    for (int wd = 0; wd < 4; ++wd) {
-                        const uint32_t v = wd == 0 ? w[j].x : wd == 1 ? w[j].y : wd == 2 ? w[j].z : w[j].w;
-                        float2 d01, d23, d45, d67;
-                        expand8(v, d01, d23, d45, d67);
-#pragma unroll
-                        for (int m = 0; m < MT; ++m) {
-                            const float4 xa = xg[m * per_m + ((2 * wd) ^ sw)];
-                            const float4 xb = xg[m * per_m + ((2 * wd + 1) ^ sw)];
-                            acc[m] = __ffma2_rn(make_float2(xa.x, xa.y), d01, acc[m]);
-                            acc[m] = __ffma2_rn(make_float2(xa.z, xa.w), d23, acc[m]);
-                            acc[m] = __ffma2_rn(make_float2(xb.x, xb.y), d45, acc[m]);
-                            acc[m] = __ffma2_rn(make_float2(xb.z, xb.w), d67, acc[m]);
+            for (int m = 0; m < MT; ++m) {
+                if (m == lane16) mine = yacc[m];
+                yacc[m] = 0.f;
+            }
+            if (a.splits == 1) {
+                if (row_ok && lane16 < a.M) a.y[(size_t)lane16 * a.N + row] = mine;
+            } else {
+                if (row_ok && lane16 < a.M) a.partial[((size_t)split * a.M + lane16) * a.N + row] = mine;
+                __threadfence();
+                __syncthreads();
+                if (tid == 0) s_last = atomicAdd(&a.counters[rb], 1u) == (unsigned)(a.splits - 1);
+                __syncthreads();
+                if (s_last) {
+                    __threadfence();
+                    for (int i = tid; i < kTeams * a.M; i += kThreads) {
+                        const int m = i / kTeams;
+                        const int r = rb * kTeams + (i - m * kTeams);
+                        if (r < a.N) {
+                            float sum = 0.f;
+                            for (int sp = 0; sp < a.splits; ++sp)
+                                sum += __ldcg(&a.partial[((size_t)sp * a.M + m) * a.N + r]);
+                            a.y[(size_t)m * a.N + r] = sum;
                         }
                     }
-#pragma unroll
-                    for (int m = 0; m < MT; ++m) yacc[m] = fmaf(s, acc[m].x + acc[m].y, yacc[m]);
+                    if (tid == 0) a.counters[rb] = 0u;
                 }
             }
         }
-
-        // Team reduction: after it every lane of the team holds the row's sums.
+        if (!has_next) break;
+        rb = nrb;
+        ch = nch;
 #pragma unroll
-        for (int m = 0; m < MT; ++m) {
-#pragma unroll
-            for (int o = kTeam / 2; o > 0; o >>= 1) yacc[m] += __shfl_xor_sync(0xffffffffu, yacc[m], o);
-        }
-        float mine = 0.f;                        // lane m keeps output m
-#pragma unroll
-        for (int m = 0; m < MT; ++m)
-            if (m == lane16) mine = yacc[m];
-
-        if (a.splits == 1) {
-            if (row_ok && lane16 < a.M) a.y[(size_t)lane16 * a.N + row] = mine;
-        } else {
-            if (row_ok && lane16 < a.M) a.partial[((size_t)split * a.M + lane16) * a.N + row] = mine;
-            __threadfence();
-            __syncthreads();
-            if (tid == 0) s_last = atomicAdd(&a.counters[rb], 1u) == (unsigned)(a.splits - 1);
-            __syncthreads();
-            if (s_last) {
-                __threadfence();
-                for (int i = tid; i < kTeams * a.M; i += kThreads) {
-                    const int m = i / kTeams;
-                    const int r = rb * kTeams + (i - m * kTeams);
-                    if (r < a.N) {
-                        float sum = 0.f;
-                        for (int sp = 0; sp < a.splits; ++sp)
-                            sum += __ldcg(&a.partial[((size_t)sp * a.M + m) * a.N + r]);
-                        a.y[(size_t)m * a.N + r] = sum;
-                    }
-                }
-                if (tid == 0) a.counters[rb] = 0u;
-            }
+        for (int j = 0; j < kSlots; ++j) {
+            w[j] = wn[j];
+            sc[j] = scn[j];
         }
     }
 }
@@ -229,18 +287,28 @@ bool plan_gemv(int64_t M, int64_t N, int64_t K, q4_dtype xt, const DeviceInfo& d
     const int mt = round_m(M);
     const int G = (int)(K / 32);
     const int row_blocks = (int)((N + kTeams - 1) / kTeams);
-    const int ksg_max = kSmemBudget / (mt * 128);
-    int splits = (G + ksg_max - 1) / ksg_max;
     // Skinny shapes: split K until every SM has a block, keeping >= 16 groups per split.
+    int splits = 1;
     while ((long long)row_blocks * splits < dev.sm_count && G / (splits + 1) >= kTeam) ++splits;
     const int ksg = (G + splits - 1) / splits;
     splits = (G + ksg - 1) / ksg;
+    if (splits > 1 && row_blocks > kCounterSlots) splits = 1;   // cannot happen while SMs < 1024
+
+    // x staging: as many groups as the shared-memory budget holds, in whole chunks.
+    const int cap_raw = kSmemBudget / (mt * 128);
+    int chunk = cap_raw >= kChunkGroups ? kChunkGroups : (cap_raw / kTeam) * kTeam;
+    if (chunk < kTeam) chunk = kTeam;
+    int xcap = (cap_raw / chunk) * chunk;
+    if (xcap < chunk) xcap = chunk;
+    const int held = ksg < xcap ? ksg : xcap;
 
     p->kernel = 0;
     p->splits = splits;
     p->groups_per_split = ksg;
     p->row_blocks = row_blocks;
-    p->smem_bytes = mt * ksg * 128;
+    p->chunk = chunk;
+    p->xcap = xcap;
+    p->smem_bytes = mt * held * 128;
     int per_sm = 2;
     const void* fn = pick_ffma(mt, xt == Q4_BF16);
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, p->smem_bytes) != cudaSuccess ||
@@ -255,10 +323,7 @@ bool plan_gemv(int64_t M, int64_t N, int64_t K, q4_dtype xt, const DeviceInfo& d
     if (gx < 1) gx = 1;
     p->grid_x = (int)gx;
     p->workspace_bytes = 0;
-    if (splits > 1) {
-        const size_t part = ((size_t)splits * (size_t)M * (size_t)N * sizeof(float) + 15) & ~(size_t)15;
-        p->workspace_bytes = part + (size_t)row_blocks * sizeof(unsigned);
-    }
+    if (splits > 1) p->workspace_bytes = kCounterBytes + (size_t)splits * (size_t)M * (size_t)N * sizeof(float);
     return true;
 }
 
@@ -274,9 +339,8 @@ q4_status launch_gemv(const void* x, q4_dtype xt, int64_t M, int64_t K, const ui
     a.partial = nullptr;
     a.counters = nullptr;
     if (plan.splits > 1) {
-        const size_t part = ((size_t)plan.splits * (size_t)M * (size_t)N * sizeof(float) + 15) & ~(size_t)15;
-        a.partial = reinterpret_cast<float*>(workspace);
-        a.counters = reinterpret_cast<unsigned*>(reinterpret_cast<char*>(workspace) + part);
+        a.counters = reinterpret_cast<unsigned*>(workspace);
+        a.partial = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) + kCounterBytes);
     }
     a.M = (int)M;
     a.N = (int)N;
@@ -284,6 +348,8 @@ q4_status launch_gemv(const void* x, q4_dtype xt, int64_t M, int64_t K, const ui
     a.ksg = plan.groups_per_split;
     a.splits = plan.splits;
     a.row_blocks = plan.row_blocks;
+    a.chunk = plan.chunk;
+    a.xcap = plan.xcap;
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)plan.grid_x, (unsigned)plan.splits);

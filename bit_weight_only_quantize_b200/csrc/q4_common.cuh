@@ -34,6 +34,8 @@ struct GemvPlan {
     int groups_per_split;   // 32-wide groups of K each split covers
     int row_blocks;         // blocks of rows
     int grid_x;             // thread blocks per split
+    int chunk;              // groups per work unit
+    int xcap;               // groups of x staged in shared memory at once
     int smem_bytes;         // dynamic shared memory per block
     size_t workspace_bytes; // partial sums + counters (0 when splits == 1)
 };

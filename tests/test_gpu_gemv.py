@@ -72,6 +72,32 @@ def test_split_k_reuses_workspace(M, N, K):
     assert rel_inf(gpu_gemv(x2, packed, scales, workspace=ws), ref2) <= 1e-5
 
 
+def test_one_workspace_shared_across_shapes():
+    """Split launches of different shapes through one workspace: the counters must
+    sit where no shape's partial sums land."""
+    import bit_weight_only_quantize_b200 as q4
+    shapes = [(1, 2048, 2560), (1, 1024, 2560), (3, 40, 4096), (1, 16, 8192), (16, 8, 2560)]
+    need = max(q4.gemv_workspace_size(*s) for s in shapes)
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    cases = []
+    for i, (M, N, K) in enumerate(shapes):
+        W = synth_inputs.weights("normal", N, K, seed=20 + i)
+        packed, scales, _ = oracle.quantize(W)
+        x = synth_inputs.activations(M, K, "bf16", seed=30 + i)
+        cases.append((x, packed, scales, oracle.matmul(x, packed, scales, threads=8)))
+    for _ in range(2):
+        for x, packed, scales, ref in cases + cases[::-1]:
+            assert rel_inf(gpu_gemv(x, packed, scales, workspace=ws), ref) <= 1e-5
+
+
+@pytest.mark.parametrize("M,N,K,x_dtype", [(1, 3000, 32768, "bf16"), (2, 2400, 16384, "f32"), (16, 300, 4096, "f32")])
+def test_x_restaged_in_chunks(M, N, K, x_dtype):
+    """K too long for one shared-memory stage of x: x is staged piecewise."""
+    W = synth_inputs.weights("outliers", N, K, seed=M + N)
+    x = synth_inputs.activations(M, K, x_dtype, seed=K)
+    check(x, W, x_dtype, tight=False)
+
+
 def test_too_small_workspace_rejected():
     import bit_weight_only_quantize_b200 as q4
     M, N, K = 1, 16, 8192
