@@ -124,6 +124,28 @@ Q4_API q4_status q4_gemv(const void* x, q4_dtype x_dtype, int64_t M, int64_t K,
                   const uint8_t* packed, const uint16_t* scales, int64_t N,
                   float* y, void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * q4_gemv_noalloc: q4_gemv for callers that cannot allocate device memory.
+ * The pages have no counterpart to this entry point; it exists for hosts that
+ * cannot hand the library a workspace (runtimes that own all device memory and
+ * give plugins no allocation hook, hosts that forbid allocation after start-up,
+ * code running while another thread captures a CUDA graph in global mode).
+ * Same inputs, outputs, layouts, alignment and arithmetic as q4_gemv; the
+ * split-K scratch is one library-owned device array of 1 MiB per device
+ * (held by every GPU that loads the library until the process exits) instead
+ * of a workspace argument.  It calls no cudaMalloc/cudaFree.
+ *  - The first call on a device performs a one-time set-up (looks up the
+ *    array's address, zero-fills it and waits for the device), so make that
+ *    first call before any stream capture on the device.
+ *  - All calls on a device share the array, which keeps the last call's
+ *    contents: calls that overlap on the GPU race.  Serialise them.
+ *  - A shape whose split needs more than 1 MiB of scratch returns
+ *    Q4_ERR_WORKSPACE (none with M <= 16 on a 148-SM B200).
+ */
+Q4_API q4_status q4_gemv_noalloc(const void* x, q4_dtype x_dtype, int64_t M, int64_t K,
+                                 const uint8_t* packed, const uint16_t* scales, int64_t N,
+                                 float* y, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
