@@ -474,6 +474,38 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+def run_profile_case(args):
+    """A few eager launches of one hot-path row, for ncu captures (no timing)."""
+    import torch
+    import bit_weight_only_quantize_b200 as q4
+    from bit_weight_only_quantize_b200 import _lib
+    lib = _lib.load()
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    stream = torch.cuda.current_stream(device).cuda_stream
+    case = args.profile
+    if case == "quantize":
+        w = synth_inputs.DECODE_PROJ[1]
+        Wd = torch.from_numpy(synth_inputs.weights(w.weights, w.N, w.K, 0)).to(device)
+        for _ in range(args.warmup + args.steps):
+            q4.quantize(Wd)
+    else:
+        w = {"decode": synth_inputs.DECODE_PROJ[1], "lm_head": synth_inputs.LM_HEAD,
+             "gemv_m4": synth_inputs.SMALL_BATCH[1], "decode_small": synth_inputs.DECODE_PROJ[2]}[case]
+        _, packed, scales = make_quantized(torch, q4, w, 0, device)
+        x = torch.from_numpy(synth_inputs.activations(w.M, w.K, "bf16", 0).view(np.int16)).view(
+            torch.bfloat16).to(device)
+        y = torch.empty((w.M, w.N), dtype=torch.float32, device=device)
+        need = q4.gemv_workspace_size(w.M, w.N, w.K)
+        ws = torch.zeros(max(need, 16), dtype=torch.uint8, device=device)
+        for _ in range(args.warmup + args.steps):
+            st = lib.q4_gemv(x.data_ptr(), 1, w.M, w.K, packed.data_ptr(), scales.data_ptr(), w.N, y.data_ptr(),
+                             ws.data_ptr(), ws.numel(), stream)
+            assert st == 0
+    torch.cuda.synchronize(device)
+    print(json.dumps({"profile_case": case, "launches": args.warmup + args.steps}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -482,7 +514,12 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--rows", choices=["all", "main"], default="all")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--profile", choices=["none", "decode", "decode_small", "lm_head", "gemv_m4", "quantize"],
+                    default="none", help="run a few untimed launches of one row (for ncu) and exit")
     args = ap.parse_args()
+    if args.profile != "none":
+        run_profile_case(args)
+        return
     if args.warmup < 3:
         args.warmup = 3
     world, rank, local = setup_dist(args)

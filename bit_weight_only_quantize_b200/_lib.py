@@ -29,6 +29,7 @@ _i64, _vp, _sz, _i32 = ctypes.c_int64, ctypes.c_void_p, ctypes.c_size_t, ctypes.
 SIGNATURES = {
     "q4_abi_version": (_i32, []),
     "q4_status_string": (ctypes.c_char_p, [_i32]),
+    "q4_device_error": (_i32, [_vp, _i32]),
     "q4_quantize": (_i32, [_vp, _i64, _i64, _vp, _vp, _vp, _vp]),
     "q4_gemv_workspace_size": (_sz, [_i64, _i64, _i64]),
     "q4_gemv": (_i32, [_vp, _i32, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _sz, _vp]),
@@ -69,6 +70,13 @@ def status_string(status: int) -> str:
         return load().q4_status_string(status).decode()
     except Exception:
         return STATUS_NAMES.get(status, f"status {status}")
+
+
+def device_error(clear: bool = True) -> int:
+    """The library's device error word for the current device (see q4_device_error)."""
+    out = ctypes.c_uint32(0)
+    check(load().q4_device_error(ctypes.byref(out), 1 if clear else 0), "q4_device_error")
+    return int(out.value)
 
 
 def check(status: int, where: str) -> None:

@@ -2,6 +2,8 @@
 // checks and dispatch to the kernels.  Every argument check happens before the
 // first CUDA call, so a bad call returns its status without touching the device.
 #include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
 
 #include <mutex>
 
@@ -46,6 +48,15 @@ q4_status current_device(DeviceInfo* out)
     std::call_once(g_once[dev], query, dev);
     *out = g_info[dev];
     return g_info_status[dev];
+}
+
+bool pdl_enabled()
+{
+    static const bool on = [] {
+        const char* v = getenv("Q4_NO_PDL");
+        return !(v && v[0] != '\0' && strcmp(v, "0") != 0);
+    }();
+    return on;
 }
 
 }  // namespace q4
@@ -102,11 +113,13 @@ size_t q4_gemv_workspace_size(int64_t M, int64_t N, int64_t K)
     if (M < 1 || M > Q4_GEMV_MAX_M || N < 1 || check_nk(N, K) != Q4_OK) return 0;
     q4::DeviceInfo dev;
     if (q4::current_device(&dev) != Q4_OK) return 0;
-    q4::GemvPlan plan;
-    if (!q4::plan_gemv(M, N, K, Q4_BF16, dev, &plan)) return 0;
-    q4::GemvPlan plan32;
-    if (!q4::plan_gemv(M, N, K, Q4_F32, dev, &plan32)) return 0;
-    return plan.workspace_bytes > plan32.workspace_bytes ? plan.workspace_bytes : plan32.workspace_bytes;
+    size_t need = 0;
+    for (q4_dtype t : {Q4_BF16, Q4_F32}) {
+        q4::GemvPlan plan;
+        if (!q4::plan_gemv(M, N, K, t, dev, nullptr, nullptr, &plan)) return 0;
+        if (plan.workspace_bytes > need) need = plan.workspace_bytes;
+    }
+    return need;
 }
 
 q4_status q4_gemv(const void* x, q4_dtype x_dtype, int64_t M, int64_t K, const uint8_t* packed,
@@ -125,7 +138,7 @@ q4_status q4_gemv(const void* x, q4_dtype x_dtype, int64_t M, int64_t K, const u
     q4::DeviceInfo dev;
     if ((st = q4::current_device(&dev)) != Q4_OK) return st;
     q4::GemvPlan plan;
-    if (!q4::plan_gemv(M, N, K, x_dtype, dev, &plan)) {
+    if (!q4::plan_gemv(M, N, K, x_dtype, dev, packed, scales, &plan)) {
         cudaGetLastError();
         return Q4_ERR_CUDA;
     }

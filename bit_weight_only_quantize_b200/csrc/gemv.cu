@@ -282,7 +282,8 @@ constexpr int kSmemBudget = 96 * 1024;          // x stage per block, keeps >= 2
 
 }  // namespace
 
-bool plan_gemv(int64_t M, int64_t N, int64_t K, q4_dtype xt, const DeviceInfo& dev, GemvPlan* p)
+namespace {
+bool plan_gemv_generic(int64_t M, int64_t N, int64_t K, q4_dtype xt, const DeviceInfo& dev, GemvPlan* p)
 {
     const int mt = round_m(M);
     const int G = (int)(K / 32);
@@ -326,11 +327,29 @@ bool plan_gemv(int64_t M, int64_t N, int64_t K, q4_dtype xt, const DeviceInfo& d
     if (splits > 1) p->workspace_bytes = kCounterBytes + (size_t)splits * (size_t)M * (size_t)N * sizeof(float);
     return true;
 }
+}  // namespace
+
+bool plan_gemv(int64_t M, int64_t N, int64_t K, q4_dtype xt, const DeviceInfo& dev, const void* packed,
+               const void* scales, GemvPlan* p)
+{
+    if (!packed && !scales) {              // sizing only: the larger workspace of the two families
+        GemvPlan g;
+        if (!plan_gemv_generic(M, N, K, xt, dev, &g)) return false;
+        GemvPlan t;
+        if (M == 1 && K % 256 == 0 && plan_gemv_tma(M, N, K, xt, dev, &t) && t.workspace_bytes > g.workspace_bytes)
+            g.workspace_bytes = t.workspace_bytes;
+        *p = g;
+        return true;
+    }
+    if (tma_gemv_eligible(M, K, packed, scales) && plan_gemv_tma(M, N, K, xt, dev, p)) return true;
+    return plan_gemv_generic(M, N, K, xt, dev, p);
+}
 
 q4_status launch_gemv(const void* x, q4_dtype xt, int64_t M, int64_t K, const uint8_t* packed,
                       const uint16_t* scales, int64_t N, float* y, void* workspace,
                       const GemvPlan& plan, cudaStream_t stream)
 {
+    if (plan.kernel == 1) return launch_gemv_tma(x, xt, K, packed, scales, N, y, workspace, plan, stream);
     GemvArgs a;
     a.x = x;
     a.packed = packed;
@@ -358,7 +377,7 @@ q4_status launch_gemv(const void* x, q4_dtype xt, int64_t M, int64_t K, const ui
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[0].val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     void* args[] = {&a};

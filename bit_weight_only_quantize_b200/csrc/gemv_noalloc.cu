@@ -79,7 +79,7 @@ extern "C" q4_status q4_gemv_noalloc(const void* x, q4_dtype x_dtype, int64_t M,
     if (g_setup_status[dev.device] != Q4_OK) return g_setup_status[dev.device];
 
     q4::GemvPlan plan;
-    if (!q4::plan_gemv(M, N, K, x_dtype, dev, &plan)) {
+    if (!q4::plan_gemv(M, N, K, x_dtype, dev, packed, scales, &plan)) {
         cudaGetLastError();
         return Q4_ERR_CUDA;
     }

@@ -107,7 +107,7 @@ q4_status launch_quantize(const float* W, int64_t N, int64_t K, uint8_t* packed,
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[0].val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     cudaError_t err = cudaLaunchKernelEx(&cfg, quantize_kernel, reinterpret_cast<const float4*>(W), nvec,

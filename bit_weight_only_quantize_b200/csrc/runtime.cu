@@ -1,0 +1,93 @@
+// Host-side runtime pieces shared by the kernels: TMA descriptor encoding through
+// the driver entry point, and the library's device error word.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "tma.cuh"
+
+namespace q4 {
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+void load_encode()
+{
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+        g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    else
+        cudaGetLastError();
+}
+
+// Bit 0: a bounded wait inside a kernel ran out (the kernel gave up and returned).
+__device__ unsigned g_device_error = 0;
+
+constexpr int kMaxDevices = 64;
+std::once_flag g_err_once[kMaxDevices];
+unsigned* g_err_addr[kMaxDevices];
+
+void lookup_err(int dev)
+{
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) {
+        cudaGetLastError();
+        p = nullptr;
+    }
+    g_err_addr[dev] = static_cast<unsigned*>(p);
+}
+
+}  // namespace
+
+bool encode_tma_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner, uint64_t outer,
+                   uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle)
+{
+    std::call_once(g_encode_once, load_encode);
+    if (!g_encode) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {pitch_bytes};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+unsigned* device_error_word()
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    std::call_once(g_err_once[dev], lookup_err, dev);
+    return g_err_addr[dev];
+}
+
+}  // namespace q4
+
+extern "C" q4_status q4_device_error(uint32_t* out, int clear)
+{
+    if (!out) return Q4_ERR_INVALID_ARG;
+    unsigned* p = q4::device_error_word();
+    if (!p) return Q4_ERR_CUDA;
+    unsigned v = 0;
+    if (cudaMemcpy(&v, p, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) {
+        cudaGetLastError();
+        return Q4_ERR_CUDA;
+    }
+    if (clear && v != 0) {
+        const unsigned zero = 0;
+        if (cudaMemcpy(p, &zero, sizeof zero, cudaMemcpyHostToDevice) != cudaSuccess) {
+            cudaGetLastError();
+            return Q4_ERR_CUDA;
+        }
+    }
+    *out = v;
+    return Q4_OK;
+}

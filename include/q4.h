@@ -82,6 +82,18 @@ Q4_API int q4_abi_version(void);
 /* Human-readable name of a status code (static string, never NULL). */
 Q4_API const char* q4_status_string(q4_status status);
 
+#define Q4_DEVICE_ERR_WAIT_TIMEOUT 1u
+
+/*
+ * Kernels never trap: a kernel whose bounded wait (on a TMA transfer, through an
+ * mbarrier) runs out records Q4_DEVICE_ERR_WAIT_TIMEOUT in a per-device error word,
+ * drains its own transfers and returns; its output is then undefined.
+ * q4_device_error reads that word for the current device into *out (synchronous,
+ * after all previously issued work that wrote it) and clears it when `clear` is
+ * non-zero.  Returns Q4_ERR_INVALID_ARG for a NULL out, Q4_ERR_CUDA on a failed copy.
+ */
+Q4_API q4_status q4_device_error(uint32_t* out, int clear);
+
 /*
  * q4_quantize: encode W[N,K] (f32, device) into the Q4 format above.
  *   W       device, f32 [N,K], 16-byte aligned.

@@ -77,6 +77,10 @@ def test_gemv_validation(lib):
     assert lib.q4_gemv(None, 1, 3, 64, None, None, 0, None, None, 0, S) == 0   # N == 0: no-op
 
 
+def test_device_error_rejects_null(lib):
+    assert lib.q4_device_error(None, 0) == 1
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
 def test_no_device_reports_cuda_error(lib):
     assert lib.q4_quantize(A16, 4, 64, A16, A16, None, None) == 6

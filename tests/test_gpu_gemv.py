@@ -98,11 +98,39 @@ def test_x_restaged_in_chunks(M, N, K, x_dtype):
     check(x, W, x_dtype, tight=False)
 
 
+@pytest.mark.parametrize("x_dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("N,K", [(1, 256), (31, 768), (33, 2560), (1000, 5120), (4097, 256), (100000, 256),
+                                 (2500, 16384), (70, 65536)])
+def test_tma_path_shapes(N, K, x_dtype):
+    """M = 1 with K % 256 == 0 takes the TMA kernel: ragged row blocks, idle warps
+    (fewer boxes than team warps), team sizes 1..8 and K splits across blocks."""
+    from bit_weight_only_quantize_b200 import _lib
+    W = synth_inputs.weights("outliers", N, K, seed=N % 97 + K)
+    x = synth_inputs.activations(1, K, x_dtype, seed=N)
+    check(x, W, x_dtype, tight=N * K <= 2 ** 26)
+    assert _lib.device_error() == 0
+
+
+def test_misaligned_scales_take_generic_path():
+    """Scales that are only 2-byte aligned cannot feed TMA; the generic kernel serves them."""
+    import bit_weight_only_quantize_b200 as q4
+    N, K = 64, 512
+    W = synth_inputs.weights("normal", N, K, seed=3)
+    packed, scales, _ = oracle.quantize(W)
+    x = synth_inputs.activations(1, K, "bf16", seed=3)
+    sc_store = torch.zeros(N * K // 32 + 8, dtype=torch.int16, device="cuda")
+    sc = sc_store[1:1 + N * K // 32].view(N, K // 32)
+    sc.copy_(torch.from_numpy(scales.view(np.int16)))
+    y = q4.gemv(to_dev_x(x), torch.from_numpy(packed).cuda(), sc)
+    torch.cuda.synchronize()
+    assert rel_inf(y.cpu().numpy(), oracle.matmul(x, packed, scales)) <= 1e-5
+
+
 def test_too_small_workspace_rejected():
     import bit_weight_only_quantize_b200 as q4
     M, N, K = 1, 16, 8192
-    need = q4.gemv_workspace_size(M, N, K)
-    ws = torch.zeros(need - 16, dtype=torch.uint8, device="cuda")
+    assert q4.gemv_workspace_size(M, N, K) > 16      # the shape splits K
+    ws = torch.zeros(16, dtype=torch.uint8, device="cuda")
     x = torch.zeros((M, K), dtype=torch.bfloat16, device="cuda")
     pk = torch.zeros((N, K // 2), dtype=torch.uint8, device="cuda")
     sc = torch.zeros((N, K // 32), dtype=torch.int16, device="cuda")
