@@ -14,7 +14,7 @@ from . import _lib
 from ._lib import Q4Error, FLAG_NONFINITE, FLAG_SCALE_OVERFLOW, GEMV_MAX_M  # noqa: F401
 
 __all__ = [
-    "quantize", "gemv", "gemv_workspace_size", "Q4Error", "FLAG_NONFINITE", "FLAG_SCALE_OVERFLOW",
+    "quantize", "gemv", "gemm", "gemv_workspace_size", "Q4Error", "FLAG_NONFINITE", "FLAG_SCALE_OVERFLOW",
     "GEMV_MAX_M",
 ]
 
@@ -96,4 +96,26 @@ def gemv(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, out: torch
         st = lib.q4_gemv(x.data_ptr(), xt, M, K, packed.data_ptr(), scales.data_ptr(), N,
                          out.data_ptr(), ws_ptr, ws_bytes, _stream())
     _lib.check(st, "q4_gemv")
+    return out
+
+
+def gemm(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    """y[M,N] (bf16) = x[M,K] (bf16) . dequant(W)^T on the tensor cores (prefill)."""
+    _need(x, "x", torch.bfloat16, 2)
+    _need(packed, "packed", torch.uint8, 2)
+    _need(scales, "scales", torch.int16, 2)
+    M, K = x.shape
+    N = packed.shape[0]
+    if packed.shape[1] * 2 != K or tuple(scales.shape) != (N, K // 32):
+        raise ValueError("shape mismatch between x, packed and scales")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    else:
+        _need(out, "out", torch.bfloat16, 2)
+        if tuple(out.shape) != (M, N):
+            raise ValueError("out has the wrong shape")
+    with torch.cuda.device(x.device):
+        st = _lib.load().q4_gemm(x.data_ptr(), M, K, packed.data_ptr(), scales.data_ptr(), N, out.data_ptr(),
+                                 _stream())
+    _lib.check(st, "q4_gemm")
     return out

@@ -34,6 +34,7 @@ SIGNATURES = {
     "q4_gemv_workspace_size": (_sz, [_i64, _i64, _i64]),
     "q4_gemv": (_i32, [_vp, _i32, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _sz, _vp]),
     "q4_gemv_noalloc": (_i32, [_vp, _i32, _i64, _i64, _vp, _vp, _i64, _vp, _vp]),
+    "q4_gemm": (_i32, [_vp, _i64, _i64, _vp, _vp, _i64, _vp, _vp]),
 }
 
 

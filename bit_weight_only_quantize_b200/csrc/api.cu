@@ -147,4 +147,19 @@ q4_status q4_gemv(const void* x, q4_dtype x_dtype, int64_t M, int64_t K, const u
                            static_cast<cudaStream_t>(stream));
 }
 
+q4_status q4_gemm(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed, const uint16_t* scales,
+                  int64_t N, uint16_t* y, void* stream)
+{
+    if (M < 0 || M > INT32_MAX) return Q4_ERR_SHAPE;
+    q4_status st = check_nk(N, K);
+    if (st != Q4_OK) return st;
+    if (M == 0 || N == 0) return Q4_OK;
+    if (!x || !packed || !scales || !y) return Q4_ERR_INVALID_ARG;
+    if (misaligned(x, 16) || misaligned(packed, 16) || misaligned(scales, 2) || misaligned(y, 2))
+        return Q4_ERR_ALIGN;
+    q4::DeviceInfo dev;
+    if ((st = q4::current_device(&dev)) != Q4_OK) return st;
+    return q4::launch_gemm(x, M, K, packed, scales, N, y, static_cast<cudaStream_t>(stream), dev);
+}
+
 }  // extern "C"

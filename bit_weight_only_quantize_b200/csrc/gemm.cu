@@ -1,0 +1,429 @@
+// q4_gemm: y[M,N] = bf16( x[M,K] . dequant(W)^T ), prefill shapes, on the 5th-generation
+// tensor cores (tcgen05, accumulators in tensor memory).
+//
+// The pages batch every prefill projection across the prompt's tokens into GEMMs
+// (QORA-4B thread, section "GPU 预填充优化"; QORA-LLM-0.8B model card, section
+// "Performance": batched prefill "processes all GEMM projections in parallel across
+// tokens").  Here each weight is dequantised once per tile into shared memory as
+// bf16 and fed to tcgen05.mma with f32 accumulation:
+//
+//   w_bf16 = bf16_rn((code - 8) * f32(scale))      (the f32 product is exact, one rounding)
+//
+// One persistent block per SM, warp-specialised:
+//   warp 0      TMA producer: x tiles (128 rows x 64 k, 128-byte swizzle) and the raw
+//               codes of the weight tile (BN rows x 32 bytes) into a ring of kStages.
+//   warp 1      allocates tensor memory; one thread issues the MMAs (128 x BN x 16
+//               per instruction, MA accumulators of 128 rows per tile) and commits.
+//   warps 2..5  epilogue: tcgen05.ld of the accumulator lanes, f32 -> bf16, stores.
+//   warps 6..13 dequantise: codes -> bf16 in the K-major 128-byte-swizzled layout the
+//               MMA descriptor expects, scales read from global (prefetched one
+//               k-block ahead), then fence.proxy.async and arrive on the stage.
+// Accumulators are double-buffered in tensor memory, so the epilogue of one tile
+// overlaps the MMAs of the next.  Every mbarrier wait is bounded; on a timeout the
+// block records kErrWaitTimeout, all roles stop, outstanding copies and MMAs are
+// waited for (bounded) and tensor memory is freed before the block exits.
+#include "tma.cuh"
+
+namespace q4 {
+namespace {
+
+constexpr int kBK = 64;                       // k per stage: one 128-byte swizzle row of bf16
+constexpr int kProducerWarp = 0;
+constexpr int kMmaWarp = 1;
+constexpr int kEpiWarp0 = 2;                  // warps 2..5
+constexpr int kDeqWarp0 = 6;                  // warps 6..13
+constexpr int kDeqWarps = 8;
+constexpr int kThreads = (kDeqWarp0 + kDeqWarps) * 32;   // 448
+constexpr uint64_t kWaitLimit = kWaitLimitNs;
+
+struct GemmArgs {
+    const uint16_t* scales;
+    uint16_t* y;
+    unsigned* err;
+    int M, N, K, G;
+    int tiles_m, tiles_n;
+    int kblocks;
+};
+
+// ---- tcgen05 wrappers (inline PTX) ----
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols)
+{
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish()
+{
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t accumulate)
+{
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void mma_commit(uint64_t* bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
+                 : "memory");
+}
+
+// 32 consecutive f32 columns of this warp's 32 accumulator lanes.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row core groups 1024 B apart.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr)
+{
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// Instruction descriptor: bf16 x bf16 -> f32, both operands K-major, M x N.
+__host__ __device__ constexpr uint32_t instr_desc(int m, int n)
+{
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
+{
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// Eight codes of one word -> eight bf16 values (code - 8) * s in k order, rounded once.
+__device__ __forceinline__ uint4 dequant8(uint32_t v, float s)
+{
+    const uint32_t u = v >> 12;
+    const float f0 = __uint_as_float((v & 0x0000000Fu) | 0x4B000000u);
+    const float f1 = __uint_as_float((v & 0x000000F0u) | 0x49000000u);
+    const float f2 = __uint_as_float((v & 0x00000F00u) | 0x47000000u);
+    const float f3 = __uint_as_float((v & 0x0000F000u) | 0x45000000u);
+    const float f4 = __uint_as_float((v & 0x000F0000u) | 0x43000000u);
+    const float f5 = __uint_as_float((u & 0x00000F00u) | 0x47000000u);
+    const float f6 = __uint_as_float((u & 0x0000F000u) | 0x45000000u);
+    const float f7 = __uint_as_float((u & 0x000F0000u) | 0x43000000u);
+    const float2 ss = make_float2(s, s);
+    const float2 d01 = __fmul2_rn(__fadd2_rn(make_float2(f0, f1), make_float2(-8388616.0f, -524296.0f)), ss);
+    const float2 d23 = __fmul2_rn(__fadd2_rn(make_float2(f2, f3), make_float2(-32776.0f, -2056.0f)), ss);
+    const float2 d45 = __fmul2_rn(__fadd2_rn(make_float2(f4, f5), make_float2(-136.0f, -32776.0f)), ss);
+    const float2 d67 = __fmul2_rn(__fadd2_rn(make_float2(f6, f7), make_float2(-2056.0f, -136.0f)), ss);
+    return make_uint4(pack_bf16x2(d01.x, d01.y), pack_bf16x2(d23.x, d23.y), pack_bf16x2(d45.x, d45.y),
+                      pack_bf16x2(d67.x, d67.y));
+}
+
+template <int MA, int BN>
+struct GemmCfg {
+    static constexpr int kStages = MA == 2 ? 4 : (BN == 128 ? 5 : 7);
+    static constexpr uint32_t kABytes = 128 * kBK * 2;            // one 128-row x tile: 16 KiB
+    static constexpr uint32_t kBBytes = BN * kBK * 2;             // dequantised weight tile
+    static constexpr uint32_t kRawBytes = BN * (kBK / 2);         // raw codes
+    static constexpr uint32_t kStageBytes = MA * kABytes + kBBytes + kRawBytes;
+    static constexpr uint32_t kTxBytes = MA * kABytes + kRawBytes;
+    static constexpr uint32_t kTmemCols = 2 * MA * BN;            // double-buffered accumulators
+    static constexpr size_t kSmem = 1024 + (size_t)kStages * kStageBytes + 256;
+    static_assert(kTmemCols == 128 || kTmemCols == 256 || kTmemCols == 512, "tensor memory columns");
+};
+
+template <int MA, int BN>
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_codes,
+               const GemmArgs a)
+{
+    using C = GemmCfg<MA, BN>;
+    constexpr int S = C::kStages;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* smem =
+        reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // Per stage: [MA x A tile][B tile][raw codes]; A and B tiles are 1024-byte aligned.
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes);
+    uint64_t* full = bars;               // producer -> dequant   (TMA bytes)
+    uint64_t* bready = bars + S;         // dequant -> MMA        (kDeqWarps arrivals)
+    uint64_t* empty = bars + 2 * S;      // MMA -> producer       (commit)
+    uint64_t* accfull = bars + 3 * S;    // MMA -> epilogue, 2 buffers (commit)
+    uint64_t* accempty = accfull + 2;    // epilogue -> MMA, 2 buffers (4 warp arrivals)
+    uint64_t* drain = accempty + 2;      // final commit on abort
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tiles = a.tiles_m * a.tiles_n;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&bready[s], kDeqWarps);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&accfull[b], 1);
+            mbar_init(&accempty[b], 4);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&tm_x);
+        tma_prefetch_desc(&tm_codes);
+    }
+    if (warp == kMmaWarp) {
+        tmem_alloc(tmem_slot, C::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    pdl_launch_dependents();
+    pdl_wait();
+
+    auto fail = [&]() {
+        *abort_flag = 1;
+        atomicOr(a.err, kErrWaitTimeout);
+    };
+
+    if (warp == kProducerWarp) {
+        if (lane == 0) {
+            int it = 0;
+            int last_phase[16];
+            for (int s = 0; s < S; ++s) last_phase[s] = -1;
+            for (int t = blockIdx.x; t < tiles && !*abort_flag; t += gridDim.x) {
+                const int m0 = (t % a.tiles_m) * (128 * MA);
+                const int n0 = (t / a.tiles_m) * BN;
+                for (int kb = 0; kb < a.kblocks; ++kb, ++it) {
+                    const int s = it % S;
+                    const uint32_t ph = (uint32_t)(it / S) & 1u;
+                    if (!mbar_wait_bounded(&empty[s], ph ^ 1u, kWaitLimit)) { fail(); break; }
+                    if (*abort_flag) break;
+                    unsigned char* st = smem + s * C::kStageBytes;
+                    mbar_arrive_expect_tx(&full[s], C::kTxBytes);
+                    for (int am = 0; am < MA; ++am)
+                        tma_load_2d(st + am * C::kABytes, &tm_x, kb * kBK, m0 + am * 128, &full[s]);
+                    tma_load_2d(st + MA * C::kABytes + C::kBBytes, &tm_codes, kb * (kBK / 2), n0, &full[s]);
+                    last_phase[s] = (int)ph;
+                }
+            }
+            if (*abort_flag)      // copies still in flight land before the block can exit
+                for (int s = 0; s < S; ++s)
+                    if (last_phase[s] >= 0) mbar_wait_bounded(&full[s], (uint32_t)last_phase[s], kWaitLimit);
+        }
+    } else if (warp == kMmaWarp) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = instr_desc(128, BN);
+            int it = 0, tcount = 0;
+            bool issued_any = false;
+            for (int t = blockIdx.x; t < tiles && !*abort_flag; t += gridDim.x, ++tcount) {
+                const int buf = tcount & 1;
+                if (!mbar_wait_bounded(&accempty[buf], ((uint32_t)(tcount >> 1) & 1u) ^ 1u, kWaitLimit)) { fail(); break; }
+                tc_fence_after();
+                bool ok = true;
+                for (int kb = 0; kb < a.kblocks; ++kb, ++it) {
+                    const int s = it % S;
+                    if (!mbar_wait_bounded(&bready[s], (uint32_t)(it / S) & 1u, kWaitLimit)) { fail(); ok = false; break; }
+                    if (*abort_flag) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t st = smem_addr(smem + s * C::kStageBytes);
+                    const uint32_t b_addr = st + MA * C::kABytes;
+#pragma unroll
+                    for (int am = 0; am < MA; ++am) {
+                        const uint32_t d = tmem_base + (uint32_t)((buf * MA + am) * BN);
+                        const uint32_t a_addr = st + am * C::kABytes;
+#pragma unroll
+                        for (int j = 0; j < kBK / 16; ++j)
+                            mma_bf16(d, sw128_desc(a_addr + j * 32), sw128_desc(b_addr + j * 32), idesc,
+                                     (kb > 0 || j > 0) ? 1u : 0u);
+                    }
+                    mma_commit(&empty[s]);     // stage reusable once these MMAs have read it
+                    issued_any = true;
+                }
+                if (!ok) break;
+                mma_commit(&accfull[buf]);     // accumulator complete
+            }
+            if (*abort_flag && issued_any) {   // every MMA issued so far completes before tensor memory is freed
+                mma_commit(drain);
+                mbar_wait_bounded(drain, 0, kWaitLimit);
+            }
+        }
+    } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 4) {
+        const int quad = warp & 3;             // tensor-memory lanes 32*quad .. 32*quad+31
+        int tcount = 0;
+        const bool vec_ok = (a.N % 8) == 0 && (reinterpret_cast<uintptr_t>(a.y) & 15) == 0;
+        for (int t = blockIdx.x; t < tiles && !*abort_flag; t += gridDim.x, ++tcount) {
+            const int buf = tcount & 1;
+            if (!mbar_wait_bounded(&accfull[buf], (uint32_t)(tcount >> 1) & 1u, kWaitLimit)) { fail(); break; }
+            tc_fence_after();
+            const int m0 = (t % a.tiles_m) * (128 * MA);
+            const int n0 = (t / a.tiles_m) * BN;
+#pragma unroll 1
+            for (int am = 0; am < MA; ++am) {
+                const int row = m0 + am * 128 + quad * 32 + lane;
+#pragma unroll 1
+                for (int c0 = 0; c0 < BN; c0 += 32) {
+                    uint32_t r[32];
+                    tmem_ld32(tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)((buf * MA + am) * BN + c0), r);
+                    const int col = n0 + c0;
+                    if (row < a.M) {
+                        uint16_t* dst = a.y + (size_t)row * a.N + col;
+                        if (vec_ok && col + 32 <= a.N) {
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) {
+                                uint4 o;
+                                o.x = pack_bf16x2(__uint_as_float(r[8 * q + 0]), __uint_as_float(r[8 * q + 1]));
+                                o.y = pack_bf16x2(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3]));
+                                o.z = pack_bf16x2(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5]));
+                                o.w = pack_bf16x2(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7]));
+                                *reinterpret_cast<uint4*>(dst + 8 * q) = o;
+                            }
+                        } else {
+#pragma unroll
+                            for (int q = 0; q < 32; ++q)
+                                if (col + q < a.N) dst[q] = (uint16_t)(pack_bf16x2(__uint_as_float(r[q]), 0.f) & 0xFFFFu);
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&accempty[buf]);
+        }
+    } else {
+        // Dequantise: each thread owns BN*8/256 chunks (row n, 16-byte k chunk c) of every stage.
+        const int dt = threadIdx.x - kDeqWarp0 * 32;
+        constexpr int kChunks = BN * 8 / (kDeqWarps * 32);
+        int it = 0;
+        for (int t = blockIdx.x; t < tiles && !*abort_flag; t += gridDim.x) {
+            const int n0 = (t / a.tiles_m) * BN;
+            float sc[kChunks];
+            auto load_scales = [&](int kb) {
+#pragma unroll
+                for (int q = 0; q < kChunks; ++q) {
+                    const int idx = dt + q * kDeqWarps * 32;
+                    const int n = n0 + idx / 8, g = kb * 2 + (idx & 7) / 4;
+                    sc[q] = (n < a.N && g < a.G) ? __half2float(__ushort_as_half(__ldg(a.scales + (size_t)n * a.G + g)))
+                                                 : 0.f;
+                }
+            };
+            load_scales(0);
+            bool ok = true;
+            for (int kb = 0; kb < a.kblocks; ++kb, ++it) {
+                const int s = it % S;
+                if (!mbar_wait_bounded(&full[s], (uint32_t)(it / S) & 1u, kWaitLimit)) { fail(); ok = false; break; }
+                if (*abort_flag) { ok = false; break; }
+                unsigned char* st = smem + s * C::kStageBytes;
+                unsigned char* bt = st + MA * C::kABytes;
+                const unsigned char* raw = bt + C::kBBytes;
+                float cur[kChunks];
+#pragma unroll
+                for (int q = 0; q < kChunks; ++q) cur[q] = sc[q];
+                if (kb + 1 < a.kblocks) load_scales(kb + 1);
+#pragma unroll
+                for (int q = 0; q < kChunks; ++q) {
+                    const int idx = dt + q * kDeqWarps * 32;
+                    const int n = idx >> 3, c = idx & 7;
+                    const uint32_t v = *reinterpret_cast<const uint32_t*>(raw + n * 32 + c * 4);
+                    *reinterpret_cast<uint4*>(bt + n * 128 + ((c ^ (n & 7)) << 4)) = dequant8(v, cur[q]);
+                }
+                fence_proxy_async_smem();      // generic-proxy writes -> tensor-core reads
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bready[s]);
+            }
+            if (!ok) break;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == kMmaWarp) tmem_dealloc(tmem_base, C::kTmemCols);
+}
+
+template <int MA, int BN>
+bool setup_kernel(size_t* smem)
+{
+    *smem = GemmCfg<MA, BN>::kSmem;
+    if (cudaFuncSetAttribute(gemm_tc_kernel<MA, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)*smem) !=
+        cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return true;
+}
+
+}  // namespace
+
+q4_status launch_gemm(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed, const uint16_t* scales,
+                      int64_t N, uint16_t* y, cudaStream_t stream, const DeviceInfo& dev)
+{
+    // Tile shape: 256 x 128 when that still gives every SM a tile, else 128 x 128, else 128 x 64.
+    const long long t256 = ((M + 255) / 256) * ((N + 127) / 128);
+    const long long t128 = ((M + 127) / 128) * ((N + 127) / 128);
+    int MA = 1, BN = 64;
+    if (t256 >= dev.sm_count) { MA = 2; BN = 128; }
+    else if (t128 >= dev.sm_count) { MA = 1; BN = 128; }
+
+    CUtensorMap tm_x, tm_codes;
+    if (!encode_tma_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_UINT16, x, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, kBK, 128,
+                       CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_tma_2d(&tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2,
+                       kBK / 2, (uint32_t)BN, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return Q4_ERR_CUDA;
+    unsigned* err = device_error_word();
+    if (!err) return Q4_ERR_CUDA;
+
+    GemmArgs a;
+    a.scales = scales;
+    a.y = y;
+    a.err = err;
+    a.M = (int)M;
+    a.N = (int)N;
+    a.K = (int)K;
+    a.G = (int)(K / 32);
+    a.tiles_m = (int)((M + 128 * MA - 1) / (128 * MA));
+    a.tiles_n = (int)((N + BN - 1) / BN);
+    a.kblocks = (int)((K + kBK - 1) / kBK);
+    const int tiles = a.tiles_m * a.tiles_n;
+
+    size_t smem = 0;
+    bool ok = MA == 2 ? setup_kernel<2, 128>(&smem) : BN == 128 ? setup_kernel<1, 128>(&smem)
+                                                                : setup_kernel<1, 64>(&smem);
+    if (!ok) return Q4_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(tiles < dev.sm_count ? tiles : dev.sm_count));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e;
+    if (MA == 2) e = cudaLaunchKernelEx(&cfg, gemm_tc_kernel<2, 128>, tm_x, tm_codes, a);
+    else if (BN == 128) e = cudaLaunchKernelEx(&cfg, gemm_tc_kernel<1, 128>, tm_x, tm_codes, a);
+    else e = cudaLaunchKernelEx(&cfg, gemm_tc_kernel<1, 64>, tm_x, tm_codes, a);
+    return e == cudaSuccess ? Q4_OK : Q4_ERR_CUDA;
+}
+
+}  // namespace q4

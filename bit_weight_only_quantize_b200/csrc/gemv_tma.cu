@@ -32,7 +32,7 @@ constexpr int kThreads = kWarps * 32;
 constexpr int kStages = 2;
 constexpr uint32_t kCodeBox = kRows * 128;   // bytes of codes per box (8 groups)
 constexpr uint32_t kScaleBox = kRows * 16;   // bytes of scales per box
-constexpr uint32_t kWaitLimit = 1u << 22;
+constexpr uint64_t kWaitLimit = kWaitLimitNs;
 constexpr int kCounterSlots = 1024;          // must match the generic kernel's workspace layout
 constexpr size_t kCounterBytes = kCounterSlots * sizeof(unsigned);
 

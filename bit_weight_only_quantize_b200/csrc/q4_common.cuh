@@ -50,12 +50,18 @@ bool plan_gemv_tma(int64_t M, int64_t N, int64_t K, q4_dtype xt, const DeviceInf
 q4_status launch_gemv_tma(const void* x, q4_dtype xt, int64_t K, const uint8_t* packed, const uint16_t* scales,
                           int64_t N, float* y, void* workspace, const GemvPlan& plan, cudaStream_t stream);
 
+q4_status launch_gemm(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed, const uint16_t* scales,
+                      int64_t N, uint16_t* y, cudaStream_t stream, const DeviceInfo& dev);
+
 // Programmatic dependent launch is on unless the environment sets Q4_NO_PDL=1
 // (read once per process; useful under tools that do not follow such launches).
 bool pdl_enabled();
 q4_status launch_gemv(const void* x, q4_dtype xt, int64_t M, int64_t K, const uint8_t* packed,
                       const uint16_t* scales, int64_t N, float* y, void* workspace,
                       const GemvPlan& plan, cudaStream_t stream);
+
+q4_status launch_gemm(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed, const uint16_t* scales,
+                      int64_t N, uint16_t* y, cudaStream_t stream, const DeviceInfo& dev);
 
 // Programmatic dependent launch: a kernel launched with the programmatic
 // stream-serialisation attribute may start before its predecessor finishes;

@@ -44,13 +44,32 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity)
     return ok != 0;
 }
 
-// Bounded wait on an mbarrier phase: returns false if the phase did not complete
-// within `limit` polls (each poll itself blocks for a hardware-defined interval).
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint32_t limit)
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar)
 {
-    for (uint32_t i = 0; i < limit; ++i)
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ uint64_t global_ns()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Every wait in the library's kernels gives up after this long (all legitimate waits
+// last microseconds).
+constexpr uint64_t kWaitLimitNs = 1000000000ull;
+
+// Bounded wait on an mbarrier phase: false if the phase has not completed within
+// limit_ns nanoseconds of global time.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint64_t limit_ns)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    while (true) {
         if (mbar_try_wait(bar, parity)) return true;
-    return false;
+        if (global_ns() - t0 > limit_ns) return false;
+    }
 }
 
 // Order this thread's earlier generic-proxy shared-memory accesses before later

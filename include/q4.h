@@ -25,7 +25,9 @@
  * (model card, "Weight Format"; "File Structure": GEMV/GEMM kernels for Q4,
  * prefill).  Here:
  *   y[m, n] = sum_k x[m, k] * w'[n, k]        (x row-major [M,K], y row-major [M,N])
- * q4_gemv serves decode (M = 1..16: one token, or a few tokens verified together).
+ * q4_gemv serves decode (M = 1..16: one token, or a few tokens verified together);
+ * q4_gemm serves prefill (large M: projections batched across the prompt's tokens,
+ * QORA-4B thread, section "GPU 预填充优化").
  *
  * Conventions for every entry point:
  *  - Pointers named d_* / documented as device pointers must point to device
@@ -135,6 +137,23 @@ Q4_API size_t q4_gemv_workspace_size(int64_t M, int64_t N, int64_t K);
 Q4_API q4_status q4_gemv(const void* x, q4_dtype x_dtype, int64_t M, int64_t K,
                   const uint8_t* packed, const uint16_t* scales, int64_t N,
                   float* y, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * q4_gemm: y = bf16( x . dequant(W)^T ) for prefill (any M >= 0; tuned for M >= 512).
+ * The pages batch the prefill projections across tokens into GEMMs (QORA-4B thread,
+ * section "GPU 预填充优化"; QORA-LLM-0.8B model card, section "Performance").
+ *   x        device, bfloat16 [M,K], 16-byte aligned.
+ *   K, N     as for q4_quantize (K % 32 == 0, K >= 32; N >= 0).
+ *   packed, scales  the Q4 encoding of W[N,K] (16-byte / 2-byte aligned).
+ *   y        device, bfloat16 [M,N], 2-byte aligned (output, overwritten); stores are
+ *            vectorised when y is 16-byte aligned and N % 8 == 0.
+ * Arithmetic: each weight becomes bf16_rn((code - 8) * f32(scale)) (one rounding of an
+ * exact product), products run on the tensor cores (tcgen05) with f32 accumulation,
+ * and each f32 output is rounded to nearest-even bfloat16.  M == 0 or N == 0 is a
+ * no-op.  No workspace.
+ */
+Q4_API q4_status q4_gemm(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed,
+                         const uint16_t* scales, int64_t N, uint16_t* y, void* stream);
 
 /*
  * q4_gemv_noalloc: q4_gemv for callers that cannot allocate device memory.

@@ -77,6 +77,20 @@ def test_gemv_validation(lib):
     assert lib.q4_gemv(None, 1, 3, 64, None, None, 0, None, None, 0, S) == 0   # N == 0: no-op
 
 
+def test_gemm_validation(lib):
+    S = None
+    assert lib.q4_gemm(A16, 4, 48, A16, A16, 8, A16, S) == 2           # K % 32
+    assert lib.q4_gemm(A16, -1, 64, A16, A16, 8, A16, S) == 2          # M < 0
+    assert lib.q4_gemm(None, 4, 64, A16, A16, 8, A16, S) == 1
+    assert lib.q4_gemm(A16, 4, 64, A16, A16, 8, None, S) == 1
+    assert lib.q4_gemm(A8, 4, 64, A16, A16, 8, A16, S) == 3            # x alignment
+    assert lib.q4_gemm(A16, 4, 64, A8, A16, 8, A16, S) == 3            # packed alignment
+    assert lib.q4_gemm(A16, 4, 64, A16, A16 + 1, 8, A16, S) == 3
+    assert lib.q4_gemm(A16, 4, 64, A16, A16, 8, A16 + 1, S) == 3
+    assert lib.q4_gemm(None, 0, 64, None, None, 8, None, S) == 0       # M == 0: no-op
+    assert lib.q4_gemm(None, 4, 64, None, None, 0, None, S) == 0       # N == 0: no-op
+
+
 def test_device_error_rejects_null(lib):
     assert lib.q4_device_error(None, 0) == 1
 
