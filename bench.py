@@ -400,6 +400,33 @@ def measure_rows(torch, q4, lib, device, peaks, l2):
         out[f"gemv_m{sw.M}"] = {"workload": f"M={sw.M} K=2560 N=4096 bf16 x", "ms": ms, "GB/s": b / ms / 1e6,
                                 "frac_hbm": b / ms / 1e6 / hbm, "bytes": b, "launches": copies * 4}
         del pks, scs
+    # Prefill q4_gemm (bf16 x, bf16 y, f32 accumulate); inputs rotated to exceed 3x L2.
+    for gw in synth_inputs.PREFILL:
+        _, packed, scales = make_quantized(torch, q4, gw, 0, device)
+        xs = torch.from_numpy(synth_inputs.activations(gw.M, gw.K, "bf16", 0).view(np.int16)).view(
+            torch.bfloat16).to(device)
+        setb = packed.numel() + scales.numel() * 2 + xs.numel() * 2
+        copies = max(2, -(-3 * l2 // setb) + 1)
+        pks = [packed] + [packed.clone() for _ in range(copies - 1)]
+        scs = [scales] + [scales.clone() for _ in range(copies - 1)]
+        xss = [xs] + [xs.clone() for _ in range(copies - 1)]
+        yg = torch.empty((gw.M, gw.N), dtype=torch.bfloat16, device=device)
+
+        def gm(i, pks=pks, scs=scs, xss=xss, yg=yg, gw=gw, copies=copies):
+            c = i % copies
+            st = lib.q4_gemm(xss[c].data_ptr(), gw.M, gw.K, pks[c].data_ptr(), scs[c].data_ptr(), gw.N,
+                             yg.data_ptr(), stream.cuda_stream)
+            assert st == 0
+        log(f"rows: gemm m={gw.M} n={gw.N}")
+        n_launch = max(copies, 8)
+        ms = time_launches(torch, gm, n_launch, device, stream)
+        flops = 2.0 * gw.M * gw.N * gw.K
+        tf = flops / ms / 1e9
+        out[gw.name] = {"workload": f"M={gw.M} K={gw.K} N={gw.N} bf16 x, bf16 y", "ms": ms, "TFLOP/s": tf,
+                        "frac_bf16_burst": tf / peaks["bf16_tflops"],
+                        "frac_bf16_sustained": tf / peaks["bf16_tflops_sustained"],
+                        "flops": flops, "launches": n_launch, "l2": f"{copies} rotating input copies"}
+        del pks, scs, xss
     torch.cuda.synchronize(device)
     return out
 
@@ -490,6 +517,19 @@ def run_profile_case(args):
         for _ in range(args.warmup + args.steps):
             q4.quantize(Wd)
     else:
+        if case.startswith("gemm"):
+            gw = synth_inputs.PREFILL[-2] if case == "gemm" else synth_inputs.PREFILL[2]
+            _, packed, scales = make_quantized(torch, q4, gw, 0, device)
+            x = torch.from_numpy(synth_inputs.activations(gw.M, gw.K, "bf16", 0).view(np.int16)).view(
+                torch.bfloat16).to(device)
+            y = torch.empty((gw.M, gw.N), dtype=torch.bfloat16, device=device)
+            for _ in range(args.warmup + args.steps):
+                st = lib.q4_gemm(x.data_ptr(), gw.M, gw.K, packed.data_ptr(), scales.data_ptr(), gw.N, y.data_ptr(),
+                                 stream)
+                assert st == 0
+            torch.cuda.synchronize(device)
+            print(json.dumps({"profile_case": case, "launches": args.warmup + args.steps}))
+            return
         w = {"decode": synth_inputs.DECODE_PROJ[1], "lm_head": synth_inputs.LM_HEAD,
              "gemv_m4": synth_inputs.SMALL_BATCH[1], "decode_small": synth_inputs.DECODE_PROJ[2]}[case]
         _, packed, scales = make_quantized(torch, q4, w, 0, device)
@@ -514,7 +554,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--rows", choices=["all", "main"], default="all")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    ap.add_argument("--profile", choices=["none", "decode", "decode_small", "lm_head", "gemv_m4", "quantize"],
+    ap.add_argument("--profile", choices=["none", "decode", "decode_small", "lm_head", "gemv_m4", "quantize", "gemm", "gemm_m2048"],
                     default="none", help="run a few untimed launches of one row (for ncu) and exit")
     args = ap.parse_args()
     if args.profile != "none":

@@ -15,9 +15,9 @@
 //   warp 1      allocates tensor memory; one thread issues the MMAs (128 x BN x 16
 //               per instruction, MA accumulators of 128 rows per tile) and commits.
 //   warps 2..5  epilogue: tcgen05.ld of the accumulator lanes, f32 -> bf16, stores.
-//   warps 6..13 dequantise: codes -> bf16 in the K-major 128-byte-swizzled layout the
-//               MMA descriptor expects, scales read from global (prefetched one
-//               k-block ahead), then fence.proxy.async and arrive on the stage.
+//   warps 6..21 dequantise: codes -> bf16 in the K-major 128-byte-swizzled layout the
+//               MMA descriptor expects, scales read from global (prefetched two
+//               k-blocks ahead), then fence.proxy.async and arrive on the stage.
 // Accumulators are double-buffered in tensor memory, so the epilogue of one tile
 // overlaps the MMAs of the next.  Every mbarrier wait is bounded; on a timeout the
 // block records kErrWaitTimeout, all roles stop, outstanding copies and MMAs are
@@ -31,9 +31,9 @@ constexpr int kBK = 64;                       // k per stage: one 128-byte swizz
 constexpr int kProducerWarp = 0;
 constexpr int kMmaWarp = 1;
 constexpr int kEpiWarp0 = 2;                  // warps 2..5
-constexpr int kDeqWarp0 = 6;                  // warps 6..13
-constexpr int kDeqWarps = 8;
-constexpr int kThreads = (kDeqWarp0 + kDeqWarps) * 32;   // 448
+constexpr int kDeqWarp0 = 6;                  // warps 6..21
+constexpr int kDeqWarps = 16;
+constexpr int kThreads = (kDeqWarp0 + kDeqWarps) * 32;   // 704
 constexpr uint64_t kWaitLimit = kWaitLimitNs;
 
 struct GemmArgs {
@@ -315,39 +315,44 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         int it = 0;
         for (int t = blockIdx.x; t < tiles && !*abort_flag; t += gridDim.x) {
             const int n0 = (t / a.tiles_m) * BN;
-            float sc[kChunks];
-            auto load_scales = [&](int kb) {
+            // Scales for k-blocks kb+1 and kb+2 are in flight while kb is dequantised.
+            float sc0[kChunks], sc1[kChunks], sc2[kChunks];
+            auto load_scales = [&](int kb, float (&dst)[kChunks]) {
 #pragma unroll
                 for (int q = 0; q < kChunks; ++q) {
                     const int idx = dt + q * kDeqWarps * 32;
                     const int n = n0 + idx / 8, g = kb * 2 + (idx & 7) / 4;
-                    sc[q] = (n < a.N && g < a.G) ? __half2float(__ushort_as_half(__ldg(a.scales + (size_t)n * a.G + g)))
-                                                 : 0.f;
+                    dst[q] = (kb < a.kblocks && n < a.N && g < a.G)
+                                 ? __half2float(__ushort_as_half(__ldg(a.scales + (size_t)n * a.G + g)))
+                                 : 0.f;
                 }
             };
-            load_scales(0);
+            load_scales(0, sc0);
+            load_scales(1, sc1);
             bool ok = true;
             for (int kb = 0; kb < a.kblocks; ++kb, ++it) {
+                load_scales(kb + 2, sc2);
                 const int s = it % S;
                 if (!mbar_wait_bounded(&full[s], (uint32_t)(it / S) & 1u, kWaitLimit)) { fail(); ok = false; break; }
                 if (*abort_flag) { ok = false; break; }
                 unsigned char* st = smem + s * C::kStageBytes;
                 unsigned char* bt = st + MA * C::kABytes;
                 const unsigned char* raw = bt + C::kBBytes;
-                float cur[kChunks];
-#pragma unroll
-                for (int q = 0; q < kChunks; ++q) cur[q] = sc[q];
-                if (kb + 1 < a.kblocks) load_scales(kb + 1);
 #pragma unroll
                 for (int q = 0; q < kChunks; ++q) {
                     const int idx = dt + q * kDeqWarps * 32;
                     const int n = idx >> 3, c = idx & 7;
                     const uint32_t v = *reinterpret_cast<const uint32_t*>(raw + n * 32 + c * 4);
-                    *reinterpret_cast<uint4*>(bt + n * 128 + ((c ^ (n & 7)) << 4)) = dequant8(v, cur[q]);
+                    *reinterpret_cast<uint4*>(bt + n * 128 + ((c ^ (n & 7)) << 4)) = dequant8(v, sc0[q]);
                 }
                 fence_proxy_async_smem();      // generic-proxy writes -> tensor-core reads
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bready[s]);
+#pragma unroll
+                for (int q = 0; q < kChunks; ++q) {
+                    sc0[q] = sc1[q];
+                    sc1[q] = sc2[q];
+                }
             }
             if (!ok) break;
         }

@@ -41,3 +41,14 @@ def f32_sum_bound(x: np.ndarray, deq: np.ndarray, roundings: int) -> np.ndarray:
     xa = np.abs(x.astype(np.float64) if x.dtype != np.uint16 else
                 (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64))
     return gamma * (xa @ np.abs(deq).T)
+
+
+def offset_path_bound(x: np.ndarray, scales: np.ndarray, roundings: int) -> np.ndarray:
+    """Bound for the bf16-activation decode path, which sums x_k * (128 + code_k) and
+    removes 136 * sum(x) per half group: every rounded partial is at most
+    144 * s_k * |x_k| per term, so |y - y_ref| <= gamma_n * sum_k |x_k| * 144 * s_k."""
+    u = 2.0 ** -24
+    gamma = roundings * u / (1 - roundings * u)
+    xa = np.abs((x.astype(np.uint32) << 16).view(np.float32).astype(np.float64))
+    s = np.repeat(scales.view(np.float16).astype(np.float64), 32, axis=1)
+    return gamma * (xa @ (144.0 * s).T)

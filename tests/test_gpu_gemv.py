@@ -7,7 +7,7 @@ import torch
 
 import oracle
 import synth_inputs
-from tests._parity import f32_sum_bound, rel_inf, to_dev_x
+from tests._parity import f32_sum_bound, offset_path_bound, rel_inf, to_dev_x
 
 pytestmark = pytest.mark.gpu
 
@@ -38,6 +38,8 @@ def check(x, W, x_dtype, tight=True):
     assert err <= TOL[x_dtype], err
     if tight:
         bound = f32_sum_bound(x, oracle.dequantize(packed, scales), roundings(W.shape[1]))
+        if x_dtype == "bf16":
+            bound = np.maximum(bound, offset_path_bound(x, scales, roundings(W.shape[1])))
         assert np.all(np.abs(y - ref) <= bound + 1e-30)
     return y, ref
 
