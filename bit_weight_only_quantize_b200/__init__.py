@@ -14,7 +14,7 @@ from . import _lib
 from ._lib import Q4Error, FLAG_NONFINITE, FLAG_SCALE_OVERFLOW, GEMV_MAX_M  # noqa: F401
 
 __all__ = [
-    "quantize", "gemv", "gemm", "gemv_workspace_size", "Q4Error", "FLAG_NONFINITE", "FLAG_SCALE_OVERFLOW",
+    "quantize", "gemv", "gemv_multi", "gemm", "gemv_workspace_size", "gemv_multi_workspace_size", "Q4Error", "FLAG_NONFINITE", "FLAG_SCALE_OVERFLOW",
     "GEMV_MAX_M",
 ]
 
@@ -97,6 +97,54 @@ def gemv(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, out: torch
                          out.data_ptr(), ws_ptr, ws_bytes, _stream())
     _lib.check(st, "q4_gemv")
     return out
+
+
+def gemv_multi_workspace_size(M: int, K: int, Ns) -> int:
+    import ctypes
+    arr = (ctypes.c_int64 * len(Ns))(*Ns)
+    return int(_lib.load().q4_gemv_multi_workspace_size(M, K, ctypes.cast(arr, ctypes.c_void_p), len(Ns)))
+
+
+def gemv_multi(x: torch.Tensor, weights, outs=None, workspace: torch.Tensor | None = None,
+               weights_static: bool = False):
+    """[y_i = x . dequant(W_i)^T for (packed_i, scales_i) in weights] in one launch.
+
+    ``weights_static=True`` declares that no kernel still running on the stream writes
+    these weights, so they may be streamed before the preceding kernel finishes.
+    """
+    import ctypes
+    if x.dtype == torch.float32:
+        xt = _lib.Q4_F32
+    elif x.dtype == torch.bfloat16:
+        xt = _lib.Q4_BF16
+    else:
+        raise TypeError("x must be float32 or bfloat16")
+    _need(x, "x", x.dtype, 2)
+    M, K = x.shape
+    if not 1 <= len(weights) <= _lib.MULTI_MAX:
+        raise ValueError(f"between 1 and {_lib.MULTI_MAX} weight matrices")
+    if outs is None:
+        outs = [torch.empty((M, p.shape[0]), dtype=torch.float32, device=x.device) for p, _ in weights]
+    arr = (_lib.Weight * len(weights))()
+    for i, ((packed, scales), y) in enumerate(zip(weights, outs)):
+        _need(packed, "packed", torch.uint8, 2)
+        _need(scales, "scales", torch.int16, 2)
+        _need(y, "out", torch.float32, 2)
+        N = packed.shape[0]
+        if packed.shape[1] * 2 != K or tuple(scales.shape) != (N, K // 32) or tuple(y.shape) != (M, N):
+            raise ValueError("shape mismatch between x, packed, scales and out")
+        arr[i] = _lib.Weight(packed.data_ptr(), scales.data_ptr(), N, y.data_ptr())
+    lib = _lib.load()
+    with torch.cuda.device(x.device):
+        need = gemv_multi_workspace_size(M, K, [p.shape[0] for p, _ in weights])
+        if need and workspace is None:
+            workspace = torch.zeros(need, dtype=torch.uint8, device=x.device)
+        ws_ptr = workspace.data_ptr() if workspace is not None else None
+        ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+        st = lib.q4_gemv_multi(x.data_ptr(), xt, M, K, ctypes.cast(arr, ctypes.c_void_p), len(weights),
+                               _lib.WEIGHTS_STATIC if weights_static else 0, ws_ptr, ws_bytes, _stream())
+    _lib.check(st, "q4_gemv_multi")
+    return outs
 
 
 def gemm(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:

@@ -23,6 +23,14 @@ Q4_BF16 = 1
 FLAG_NONFINITE = 1
 FLAG_SCALE_OVERFLOW = 2
 GEMV_MAX_M = 16
+MULTI_MAX = 4
+WEIGHTS_STATIC = 1
+
+
+class Weight(ctypes.Structure):
+    """struct q4_weight of include/q4.h."""
+    _fields_ = [("packed", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("N", ctypes.c_int64),
+                ("y", ctypes.c_void_p)]
 
 # Every symbol include/q4.h declares, with (restype, argtypes).
 _i64, _vp, _sz, _i32 = ctypes.c_int64, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
@@ -35,6 +43,8 @@ SIGNATURES = {
     "q4_gemv": (_i32, [_vp, _i32, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _sz, _vp]),
     "q4_gemv_noalloc": (_i32, [_vp, _i32, _i64, _i64, _vp, _vp, _i64, _vp, _vp]),
     "q4_gemm": (_i32, [_vp, _i64, _i64, _vp, _vp, _i64, _vp, _vp]),
+    "q4_gemv_multi_workspace_size": (_sz, [_i64, _i64, _vp, _i32]),
+    "q4_gemv_multi": (_i32, [_vp, _i32, _i64, _i64, _vp, _i32, ctypes.c_uint32, _vp, _sz, _vp]),
 }
 
 

@@ -108,43 +108,99 @@ q4_status q4_quantize(const float* W, int64_t N, int64_t K, uint8_t* packed, uin
     return q4::launch_quantize(W, N, K, packed, scales, flags, static_cast<cudaStream_t>(stream), dev);
 }
 
-size_t q4_gemv_workspace_size(int64_t M, int64_t N, int64_t K)
+namespace {
+
+// Validates a matrix list and keeps the matrices with N > 0.
+q4_status collect(const q4_weight* mats, int count, int64_t K, q4_weight* out, int* kept, bool need_pointers)
 {
-    if (M < 1 || M > Q4_GEMV_MAX_M || N < 1 || check_nk(N, K) != Q4_OK) return 0;
+    if (!mats || count < 1 || count > Q4_MULTI_MAX) return Q4_ERR_INVALID_ARG;
+    int n = 0;
+    for (int i = 0; i < count; ++i) {
+        q4_status st = check_nk(mats[i].N, K);
+        if (st != Q4_OK) return st;
+        if (mats[i].N == 0) continue;
+        if (need_pointers) {
+            if (!mats[i].packed || !mats[i].scales || !mats[i].y) return Q4_ERR_INVALID_ARG;
+            if (misaligned(mats[i].packed, 16) || misaligned(mats[i].scales, 2) || misaligned(mats[i].y, 4))
+                return Q4_ERR_ALIGN;
+        }
+        out[n++] = mats[i];
+    }
+    *kept = n;
+    return Q4_OK;
+}
+
+size_t workspace_for(int64_t M, int64_t K, const q4_weight* mats, int count)
+{
     q4::DeviceInfo dev;
     if (q4::current_device(&dev) != Q4_OK) return 0;
     size_t need = 0;
     for (q4_dtype t : {Q4_BF16, Q4_F32}) {
         q4::GemvPlan plan;
-        if (!q4::plan_gemv(M, N, K, t, dev, nullptr, nullptr, &plan)) return 0;
+        if (!q4::plan_gemv(M, mats, count, K, t, dev, true, &plan)) return 0;
         if (plan.workspace_bytes > need) need = plan.workspace_bytes;
     }
     return need;
+}
+
+q4_status gemv_common(const void* x, q4_dtype x_dtype, int64_t M, int64_t K, const q4_weight* mats, int count,
+                      uint32_t flags, void* workspace, size_t workspace_bytes, void* stream)
+{
+    if (x_dtype != Q4_F32 && x_dtype != Q4_BF16) return Q4_ERR_DTYPE;
+    if (M < 0 || M > Q4_GEMV_MAX_M) return Q4_ERR_SHAPE;
+    if (K < 32 || (K % 32) != 0 || K > INT32_MAX) return Q4_ERR_SHAPE;
+    if (flags & ~Q4_WEIGHTS_STATIC) return Q4_ERR_INVALID_ARG;
+    q4_weight kept[Q4_MULTI_MAX];
+    int n = 0;
+    q4_status st = collect(mats, count, K, kept, &n, M > 0);
+    if (st != Q4_OK) return st;
+    if (M == 0 || n == 0) return Q4_OK;
+    if (!x) return Q4_ERR_INVALID_ARG;
+    if (misaligned(x, 16) || (workspace && misaligned(workspace, 16))) return Q4_ERR_ALIGN;
+    q4::DeviceInfo dev;
+    if ((st = q4::current_device(&dev)) != Q4_OK) return st;
+    q4::GemvPlan plan;
+    if (!q4::plan_gemv(M, kept, n, K, x_dtype, dev, false, &plan)) {
+        cudaGetLastError();
+        return Q4_ERR_CUDA;
+    }
+    if (plan.workspace_bytes > 0 && (!workspace || workspace_bytes < plan.workspace_bytes)) return Q4_ERR_WORKSPACE;
+    return q4::launch_gemv(x, x_dtype, M, K, kept, n, flags, workspace, plan, static_cast<cudaStream_t>(stream));
+}
+
+}  // namespace
+
+size_t q4_gemv_workspace_size(int64_t M, int64_t N, int64_t K)
+{
+    if (M < 1 || M > Q4_GEMV_MAX_M || N < 1 || check_nk(N, K) != Q4_OK) return 0;
+    const q4_weight w = {nullptr, nullptr, N, nullptr};
+    return workspace_for(M, K, &w, 1);
+}
+
+size_t q4_gemv_multi_workspace_size(int64_t M, int64_t K, const int64_t* Ns, int count)
+{
+    if (M < 1 || M > Q4_GEMV_MAX_M || !Ns || count < 1 || count > Q4_MULTI_MAX) return 0;
+    q4_weight mats[Q4_MULTI_MAX];
+    int n = 0;
+    for (int i = 0; i < count; ++i) {
+        if (check_nk(Ns[i], K) != Q4_OK) return 0;
+        if (Ns[i] > 0) mats[n++] = q4_weight{nullptr, nullptr, Ns[i], nullptr};
+    }
+    return n ? workspace_for(M, K, mats, n) : 0;
 }
 
 q4_status q4_gemv(const void* x, q4_dtype x_dtype, int64_t M, int64_t K, const uint8_t* packed,
                   const uint16_t* scales, int64_t N, float* y, void* workspace, size_t workspace_bytes,
                   void* stream)
 {
-    if (x_dtype != Q4_F32 && x_dtype != Q4_BF16) return Q4_ERR_DTYPE;
-    if (M < 0 || M > Q4_GEMV_MAX_M) return Q4_ERR_SHAPE;
-    q4_status st = check_nk(N, K);
-    if (st != Q4_OK) return st;
-    if (M == 0 || N == 0) return Q4_OK;
-    if (!x || !packed || !scales || !y) return Q4_ERR_INVALID_ARG;
-    if (misaligned(x, 16) || misaligned(packed, 16) || misaligned(scales, 2) || misaligned(y, 4) ||
-        (workspace && misaligned(workspace, 16)))
-        return Q4_ERR_ALIGN;
-    q4::DeviceInfo dev;
-    if ((st = q4::current_device(&dev)) != Q4_OK) return st;
-    q4::GemvPlan plan;
-    if (!q4::plan_gemv(M, N, K, x_dtype, dev, packed, scales, &plan)) {
-        cudaGetLastError();
-        return Q4_ERR_CUDA;
-    }
-    if (plan.workspace_bytes > 0 && (!workspace || workspace_bytes < plan.workspace_bytes)) return Q4_ERR_WORKSPACE;
-    return q4::launch_gemv(x, x_dtype, M, K, packed, scales, N, y, workspace, plan,
-                           static_cast<cudaStream_t>(stream));
+    const q4_weight w = {packed, scales, N, y};
+    return gemv_common(x, x_dtype, M, K, &w, 1, 0u, workspace, workspace_bytes, stream);
+}
+
+q4_status q4_gemv_multi(const void* x, q4_dtype x_dtype, int64_t M, int64_t K, const q4_weight* mats, int count,
+                        uint32_t flags, void* workspace, size_t workspace_bytes, void* stream)
+{
+    return gemv_common(x, x_dtype, M, K, mats, count, flags, workspace, workspace_bytes, stream);
 }
 
 q4_status q4_gemm(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed, const uint16_t* scales,

@@ -329,27 +329,11 @@ bool plan_gemv_generic(int64_t M, int64_t N, int64_t K, q4_dtype xt, const Devic
 }
 }  // namespace
 
-bool plan_gemv(int64_t M, int64_t N, int64_t K, q4_dtype xt, const DeviceInfo& dev, const void* packed,
-               const void* scales, GemvPlan* p)
+namespace {
+q4_status launch_gemv_generic(const void* x, q4_dtype xt, int64_t M, int64_t K, const uint8_t* packed,
+                              const uint16_t* scales, int64_t N, float* y, void* workspace,
+                              const GemvPlan& plan, cudaStream_t stream)
 {
-    if (!packed && !scales) {              // sizing only: the larger workspace of the two families
-        GemvPlan g;
-        if (!plan_gemv_generic(M, N, K, xt, dev, &g)) return false;
-        GemvPlan t;
-        if (M == 1 && K % 256 == 0 && plan_gemv_tma(M, N, K, xt, dev, &t) && t.workspace_bytes > g.workspace_bytes)
-            g.workspace_bytes = t.workspace_bytes;
-        *p = g;
-        return true;
-    }
-    if (tma_gemv_eligible(M, K, packed, scales) && plan_gemv_tma(M, N, K, xt, dev, p)) return true;
-    return plan_gemv_generic(M, N, K, xt, dev, p);
-}
-
-q4_status launch_gemv(const void* x, q4_dtype xt, int64_t M, int64_t K, const uint8_t* packed,
-                      const uint16_t* scales, int64_t N, float* y, void* workspace,
-                      const GemvPlan& plan, cudaStream_t stream)
-{
-    if (plan.kernel == 1) return launch_gemv_tma(x, xt, K, packed, scales, N, y, workspace, plan, stream);
     GemvArgs a;
     a.x = x;
     a.packed = packed;
@@ -383,6 +367,54 @@ q4_status launch_gemv(const void* x, q4_dtype xt, int64_t M, int64_t K, const ui
     void* args[] = {&a};
     const cudaError_t err = cudaLaunchKernelExC(&cfg, pick_ffma(round_m(M), xt == Q4_BF16), args);
     return err == cudaSuccess ? Q4_OK : Q4_ERR_CUDA;
+}
+}  // namespace
+
+bool plan_gemv(int64_t M, const q4_weight* mats, int count, int64_t K, q4_dtype xt, const DeviceInfo& dev,
+               bool sizing_only, GemvPlan* p)
+{
+    if (count < 1 || count > Q4_MULTI_MAX) return false;
+    // Workspace the generic kernel needs for the largest of the matrices (it serves
+    // them one launch each when the TMA kernels cannot).
+    size_t generic_ws = 0;
+    GemvPlan g = {};
+    for (int i = 0; i < count; ++i) {
+        if (!plan_gemv_generic(M, mats[i].N, K, xt, dev, &g)) return false;
+        if (g.workspace_bytes > generic_ws) generic_ws = g.workspace_bytes;
+    }
+    bool eligible = true;
+    for (int i = 0; i < count; ++i)
+        eligible = eligible && (sizing_only ? tma_gemv_eligible(M, K, xt, nullptr, nullptr)
+                                            : tma_gemv_eligible(M, K, xt, mats[i].packed, mats[i].scales));
+    int64_t Ns[Q4_MULTI_MAX];
+    for (int i = 0; i < count; ++i) Ns[i] = mats[i].N;
+    if (eligible && plan_gemv_tma(M, Ns, count, K, xt, dev, p)) {
+        if (sizing_only && generic_ws > p->workspace_bytes) p->workspace_bytes = generic_ws;
+        return true;
+    }
+    *p = g;
+    p->kernel = 0;
+    p->workspace_bytes = generic_ws;
+    return true;
+}
+
+q4_status launch_gemv(const void* x, q4_dtype xt, int64_t M, int64_t K, const q4_weight* mats, int count,
+                      uint32_t flags, void* workspace, const GemvPlan& plan, cudaStream_t stream)
+{
+    if (plan.kernel == 1)
+        return launch_gemv_tma(x, xt, M, K, mats, count, (flags & Q4_WEIGHTS_STATIC) ? 1 : 0, workspace, plan,
+                               stream);
+    DeviceInfo dev;
+    q4_status st = current_device(&dev);
+    if (st != Q4_OK) return st;
+    for (int i = 0; i < count; ++i) {        // one generic launch per matrix, in order on the stream
+        GemvPlan g;
+        if (!plan_gemv_generic(M, mats[i].N, K, xt, dev, &g)) return Q4_ERR_CUDA;
+        st = launch_gemv_generic(x, xt, M, K, mats[i].packed, mats[i].scales, mats[i].N, mats[i].y, workspace, g,
+                                 stream);
+        if (st != Q4_OK) return st;
+    }
+    return Q4_OK;
 }
 
 }  // namespace q4

@@ -78,12 +78,13 @@ extern "C" q4_status q4_gemv_noalloc(const void* x, q4_dtype x_dtype, int64_t M,
     std::call_once(g_setup_once[dev.device], setup_device, dev.device);
     if (g_setup_status[dev.device] != Q4_OK) return g_setup_status[dev.device];
 
+    const q4_weight w = {packed, scales, N, y};
     q4::GemvPlan plan;
-    if (!q4::plan_gemv(M, N, K, x_dtype, dev, packed, scales, &plan)) {
+    if (!q4::plan_gemv(M, &w, 1, K, x_dtype, dev, false, &plan)) {
         cudaGetLastError();
         return Q4_ERR_CUDA;
     }
     if (plan.workspace_bytes > kScratchBytes) return Q4_ERR_WORKSPACE;
-    return q4::launch_gemv(x, x_dtype, M, K, packed, scales, N, y, g_scratch_addr[dev.device], plan,
+    return q4::launch_gemv(x, x_dtype, M, K, &w, 1, 0u, g_scratch_addr[dev.device], plan,
                            static_cast<cudaStream_t>(stream));
 }

@@ -40,15 +40,19 @@ struct GemvPlan {
     size_t workspace_bytes; // partial sums + counters (0 when splits == 1)
 };
 
-// Chooses the kernel for a shape.  packed/scales may be NULL (sizing only: the
-// plan then assumes the pointers the TMA kernel needs and reports the larger
-// workspace of the two kernel families).
-bool plan_gemv(int64_t M, int64_t N, int64_t K, q4_dtype xt, const DeviceInfo& dev, const void* packed,
-               const void* scales, GemvPlan* plan);
-bool tma_gemv_eligible(int64_t M, int64_t K, const void* packed, const void* scales);
-bool plan_gemv_tma(int64_t M, int64_t N, int64_t K, q4_dtype xt, const DeviceInfo& dev, GemvPlan* plan);
-q4_status launch_gemv_tma(const void* x, q4_dtype xt, int64_t K, const uint8_t* packed, const uint16_t* scales,
-                          int64_t N, float* y, void* workspace, const GemvPlan& plan, cudaStream_t stream);
+// Chooses the kernels for one or more weight matrices sharing x (all N > 0).
+// With sizing_only the pointers are not looked at: the plan assumes pointers the TMA
+// kernels accept and reports the largest workspace either kernel family may need.
+bool plan_gemv(int64_t M, const q4_weight* mats, int count, int64_t K, q4_dtype xt, const DeviceInfo& dev,
+               bool sizing_only, GemvPlan* plan);
+q4_status launch_gemv(const void* x, q4_dtype xt, int64_t M, int64_t K, const q4_weight* mats, int count,
+                      uint32_t flags, void* workspace, const GemvPlan& plan, cudaStream_t stream);
+
+bool tma_gemv_eligible(int64_t M, int64_t K, q4_dtype xt, const void* packed, const void* scales);
+bool plan_gemv_tma(int64_t M, const int64_t* Ns, int count, int64_t K, q4_dtype xt, const DeviceInfo& dev,
+                   GemvPlan* plan);
+q4_status launch_gemv_tma(const void* x, q4_dtype xt, int64_t M, int64_t K, const q4_weight* mats, int count,
+                          int prefetch, void* workspace, const GemvPlan& plan, cudaStream_t stream);
 
 q4_status launch_gemm(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed, const uint16_t* scales,
                       int64_t N, uint16_t* y, cudaStream_t stream, const DeviceInfo& dev);
@@ -56,12 +60,6 @@ q4_status launch_gemm(const uint16_t* x, int64_t M, int64_t K, const uint8_t* pa
 // Programmatic dependent launch is on unless the environment sets Q4_NO_PDL=1
 // (read once per process; useful under tools that do not follow such launches).
 bool pdl_enabled();
-q4_status launch_gemv(const void* x, q4_dtype xt, int64_t M, int64_t K, const uint8_t* packed,
-                      const uint16_t* scales, int64_t N, float* y, void* workspace,
-                      const GemvPlan& plan, cudaStream_t stream);
-
-q4_status launch_gemm(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed, const uint16_t* scales,
-                      int64_t N, uint16_t* y, cudaStream_t stream, const DeviceInfo& dev);
 
 // Programmatic dependent launch: a kernel launched with the programmatic
 // stream-serialisation attribute may start before its predecessor finishes;

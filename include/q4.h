@@ -77,6 +77,8 @@ typedef enum q4_dtype {
 #define Q4_FLAG_SCALE_OVERFLOW 2u
 
 #define Q4_GEMV_MAX_M 16
+#define Q4_MULTI_MAX 4
+#define Q4_WEIGHTS_STATIC 1u
 
 /* Version of this ABI (incremented on any incompatible change). */
 Q4_API int q4_abi_version(void);
@@ -137,6 +139,34 @@ Q4_API size_t q4_gemv_workspace_size(int64_t M, int64_t N, int64_t K);
 Q4_API q4_status q4_gemv(const void* x, q4_dtype x_dtype, int64_t M, int64_t K,
                   const uint8_t* packed, const uint16_t* scales, int64_t N,
                   float* y, void* workspace, size_t workspace_bytes, void* stream);
+
+/* One weight matrix of a q4_gemv_multi call and its output. */
+typedef struct q4_weight {
+    const uint8_t* packed;    /* device, codes [N, K/2], 16-byte aligned */
+    const uint16_t* scales;   /* device, binary16 bits [N, K/32], 2-byte aligned */
+    int64_t N;                /* output features (rows), >= 0 */
+    float* y;                 /* device, f32 [M, N], 4-byte aligned (output, overwritten) */
+} q4_weight;
+
+/* Workspace bytes for q4_gemv_multi with these row counts (0 when none). */
+Q4_API size_t q4_gemv_multi_workspace_size(int64_t M, int64_t K, const int64_t* Ns, int count);
+
+/*
+ * q4_gemv_multi: y_i = x . dequant(W_i)^T for up to Q4_MULTI_MAX weight matrices that
+ * share x (the several projections of one token, e.g. query/key/value or gate/up, as in
+ * the fused gate+up decode of the QORA-LLM-0.8B model card, section "AVX-512 SIMD
+ * Acceleration"), in one launch.  Same arithmetic, layouts and alignment as q4_gemv,
+ * which is the count == 1 case.  Matrices with N == 0 are skipped.
+ *   mats     host array of `count` (1..Q4_MULTI_MAX) q4_weight; all share K.
+ *   flags    0, or Q4_WEIGHTS_STATIC: the caller guarantees no kernel still in flight
+ *            on `stream` writes any packed/scales buffer of `mats`, which lets the
+ *            kernel stream the weights while its predecessor on the stream finishes
+ *            (x and the outputs are only touched after the predecessor completes).
+ *   workspace  as for q4_gemv, sized by q4_gemv_multi_workspace_size.
+ */
+Q4_API q4_status q4_gemv_multi(const void* x, q4_dtype x_dtype, int64_t M, int64_t K,
+                               const q4_weight* mats, int count, uint32_t flags,
+                               void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * q4_gemm: y = bf16( x . dequant(W)^T ) for prefill (any M >= 0; tuned for M >= 512).

@@ -91,6 +91,23 @@ def test_gemm_validation(lib):
     assert lib.q4_gemm(None, 4, 64, None, None, 0, None, S) == 0       # N == 0: no-op
 
 
+def test_gemv_multi_validation(lib):
+    W = _lib.Weight
+    good = (W * 2)(W(A16, A16, 8, A16), W(A16, A16, 16, A16))
+    vp = ctypes.cast(good, ctypes.c_void_p)
+    assert lib.q4_gemv_multi(A16, 1, 1, 64, None, 1, 0, None, 0, None) == 1          # no matrices
+    assert lib.q4_gemv_multi(A16, 1, 1, 64, vp, 0, 0, None, 0, None) == 1            # count 0
+    assert lib.q4_gemv_multi(A16, 1, 1, 64, vp, 5, 0, None, 0, None) == 1            # count > max
+    assert lib.q4_gemv_multi(A16, 1, 1, 64, vp, 2, 4, None, 0, None) == 1            # unknown flag
+    assert lib.q4_gemv_multi(A16, 1, 1, 48, vp, 2, 0, None, 0, None) == 2            # K % 32
+    bad = (W * 2)(W(A16, A16, 8, A16), W(A8, A16, 16, A16))
+    assert lib.q4_gemv_multi(A16, 1, 1, 64, ctypes.cast(bad, ctypes.c_void_p), 2, 0, None, 0, None) == 3
+    nul = (W * 2)(W(A16, A16, 8, A16), W(None, A16, 16, A16))
+    assert lib.q4_gemv_multi(A16, 1, 1, 64, ctypes.cast(nul, ctypes.c_void_p), 2, 0, None, 0, None) == 1
+    empty = (W * 2)(W(None, None, 0, None), W(None, None, 0, None))
+    assert lib.q4_gemv_multi(A16, 1, 1, 64, ctypes.cast(empty, ctypes.c_void_p), 2, 0, None, 0, None) == 0
+
+
 def test_device_error_rejects_null(lib):
     assert lib.q4_device_error(None, 0) == 1
 
