@@ -541,6 +541,16 @@ def run_profile_case(args):
             torch.cuda.synchronize(device)
             print(json.dumps({"profile_case": case, "launches": args.warmup + args.steps}))
             return
+        if case == "decode_multi":
+            mats = [make_quantized(torch, q4, w, 0, device) for w in MAIN]
+            x = torch.from_numpy(synth_inputs.activations(1, 2560, "bf16", 0).view(np.int16)).view(
+                torch.bfloat16).to(device)
+            weights = [(p, s) for _, p, s in mats]
+            for _ in range(args.warmup + args.steps):
+                q4.gemv_multi(x, weights, weights_static=True)
+            torch.cuda.synchronize(device)
+            print(json.dumps({"profile_case": case, "launches": args.warmup + args.steps}))
+            return
         w = {"decode": synth_inputs.DECODE_PROJ[1], "lm_head": synth_inputs.LM_HEAD,
              "gemv_m4": synth_inputs.SMALL_BATCH[1], "decode_small": synth_inputs.DECODE_PROJ[2]}[case]
         _, packed, scales = make_quantized(torch, q4, w, 0, device)
@@ -565,7 +575,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--rows", choices=["all", "main"], default="all")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    ap.add_argument("--profile", choices=["none", "decode", "decode_small", "lm_head", "gemv_m4", "quantize", "gemm", "gemm_m2048"],
+    ap.add_argument("--profile", choices=["none", "decode", "decode_small", "decode_multi", "lm_head", "gemv_m4", "quantize", "gemm",
+                             "gemm_m2048"],
                     default="none", help="run a few untimed launches of one row (for ncu) and exit")
     args = ap.parse_args()
     if args.profile != "none":

@@ -1,36 +1,38 @@
 // q4_gemv / q4_gemv_multi for the shapes the TMA path serves (K % 256 == 0, scales
-// 16-byte aligned; M = 1 with f32 or bf16 x, M = 2..16 with bf16 x).
+// 16-byte aligned; M = 1 with f32 or bf16 x, M = 1..16 with bf16 x).
 //
 // Decode streams every weight once, so the kernels are built around keeping HBM busy
 // and spending few instructions per weight (QORA-LLM-0.8B model card, section "AVX-512
 // SIMD Acceleration": a Q4 GEMV whose nibbles go through a 16-entry table; QORA-4B
 // thread, section "量化与内存管理": GEMV over Q4 weights on a thread pool):
 //
-//  * Weights stream as TMA boxes of 16 rows x 8 groups: 2 KiB of codes (128-byte
-//    swizzled) plus 256 B of binary16 scales, into a per-warp ring of kStages stages
-//    guarded by mbarriers.  Each warp issues its own boxes (lane 0), so no producer
-//    warp is needed and a block keeps warps * kStages boxes in flight.
+//  * Weights stream as TMA boxes of 16 rows x 8 groups (2 KiB of codes, 128-byte
+//    swizzled); a ring stage holds kBoxesPerStage consecutive boxes plus one box of
+//    their binary16 scales under one mbarrier.  Each warp keeps its own ring of kStages
+//    stages and issues its own copies (lane 0), so every warp has about 9 KiB in flight.
 //  * Work is cut into row blocks of 16 rows, enumerated over one or more weight
 //    matrices that share x (one launch for a set of projections of the same token).
 //    Teams of P warps own sequences of row blocks; the P warps of a team take
 //    disjoint K ranges of each block and add their partial sums in a fixed order.
-//    Skinny shapes also split K across blocks (last-arriver reduction, no waiting).
+//    Skinny shapes may also split K across blocks (last-arriver reduction, no
+//    waiting).  The plan picks splits, P and teams per block with a small cost model.
 //  * Arithmetic per mode:
 //      f32 x, M = 1:  nibble p OR-ed into the mantissa of 2^(23-4p) is exactly
 //                     2^(23-4p) + code; a packed f32x2 add leaves code - 8; packed
 //                     f32x2 FMAs accumulate each group in f32.  Two lanes per row.
-//      bf16 x, M = 1: nibble pair (j, j+4) OR-ed into 0x4300 is the bf16 pair
-//                     (128 + c_j, 128 + c_{j+4}); fma.rn.f32.bf16 multiplies it by the
-//                     bf16 x pair exactly and accumulates in f32; 136 * sum(x) of the
-//                     half group (an f64 sum rounded once) is subtracted afterwards.
-//      bf16 x, M = 2..16: the same bf16 pairs are the A operand of
-//                     mma.sync.m16n8k16 (f32 accumulate), x rows the B operand, in a
-//                     permuted k order that matches the pairs; 136 * sum(x) per group
-//                     and x row is subtracted from each group's MMA result.
+//      bf16 x, M = 1..16: nibble pair (j, j+4) of a word OR-ed into 0x4300 (one LOP3)
+//                     is the bf16 pair (128 + c_j, 128 + c_{j+4}); such pairs, read
+//                     with ldmatrix, are the A operand of mma.sync.m16n8k16 (f32
+//                     accumulate) and x rows the B operand, in a permuted k order that
+//                     matches the pairs.  The MMA's C operand is -136 * sum(x) of the
+//                     group (an f64 sum rounded once), so each result is the exact
+//                     group dot product up to f32 accumulation.
 //    In every mode each group's sum is scaled by its binary16 scale and added in f32.
 //  * Every mbarrier wait is bounded.  If one runs out the kernel records
 //    kErrWaitTimeout in the library error word, stops issuing and computing, waits
 //    (bounded) for its own copies still in flight and returns (see q4_device_error).
+#include <algorithm>
+
 #include "tma.cuh"
 
 namespace q4 {
@@ -39,13 +41,24 @@ namespace {
 constexpr int kRows = 16;                    // rows per row block
 constexpr int kMaxWarps = 16;
 constexpr int kStages = 2;
+constexpr int kBoxesPerStage = 2;            // code boxes per ring stage (one mbarrier)
 constexpr uint32_t kCodeBox = kRows * 128;   // bytes of codes per box (8 groups)
 constexpr uint32_t kScaleBox = kRows * 16;   // bytes of scales per box
+constexpr uint32_t kStageCodes = kBoxesPerStage * kCodeBox;
+constexpr uint32_t kStageScales = kBoxesPerStage * kScaleBox;   // one box of 8 * kBoxesPerStage groups
 constexpr uint64_t kWaitLimit = kWaitLimitNs;
 constexpr int kCounterSlots = 1024;          // same workspace layout as the generic kernel
+// Plan cost model, in units of the time one warp takes for a stage unit when 16 warps
+// share the SM (measured on B200: about 2.7 us).  A warp with fewer neighbours is
+// faster only down to the pace of kMinWarpShare warps (its own dependency chains and
+// memory latency bound it); the row-block epilogue (team reduction, stores) and the
+// split-K reduction (partials through L2 and an atomic per row block) add fixed costs.
+constexpr double kMinWarpShare = 12.0;
+constexpr double kEpilogueCost = 0.1;
+constexpr double kSplitCost = 0.9;
 constexpr size_t kCounterBytes = kCounterSlots * sizeof(unsigned);
 
-enum Mode { kF32M1 = 0, kBf16M1 = 1, kMma8 = 2, kMma16 = 3 };
+enum Mode { kF32M1 = 0, kMma8 = 1, kMma16 = 2 };
 
 struct TmaMaps {
     CUtensorMap codes[Q4_MULTI_MAX];
@@ -125,42 +138,56 @@ __device__ __forceinline__ float2 word_dot_f32(uint32_t v, const float4* xw, con
     return acc;
 }
 
-// d = a * b + c with bfloat16 a, b (exact product) and f32 c, d: one rounding.
-__device__ __forceinline__ float fma_bf16(uint16_t a, uint16_t b, float c)
+// (a & m) | c as one LOP3; m and c are kept in registers (pinned) by the callers, since the
+// instruction takes a single immediate.
+__device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t m, uint32_t c)
 {
-    float d;
-    asm("fma.rn.f32.bf16 %0, %1, %2, %3;" : "=f"(d) : "h"(a), "h"(b), "f"(c));
-    return d;
+    uint32_t r;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(a), "r"(m), "r"(c));
+    return r;
 }
 
-// Nibble pair (j, j+4) of a word as the bf16 pair (128 + c_j, 128 + c_{j+4}).
-__device__ __forceinline__ uint32_t nib_pair(uint32_t v, int j)
+__device__ __forceinline__ uint32_t pinned_u32(uint32_t v)
 {
-    return ((v >> (4 * j)) & 0x000F000Fu) | 0x43004300u;
+    uint32_t r;
+    asm volatile("mov.b32 %0, %1;" : "=r"(r) : "r"(v));
+    return r;
 }
 
-// bf16 x: sum_j x_j * (128 + c_j) over the 8 weights of one word; xp holds the x pairs
-// (x_j, x_{j+4}) matching nib_pair.  Every product is exact in f32.
-__device__ __forceinline__ float word_dot_bf16(uint32_t v, uint4 xp, float acc)
+// Nibble pair (j, j+4) of a word as the bf16 pair (128 + c_j, 128 + c_{j+4}); mask and
+// magic are the registers holding 0x000F000F and 0x43004300.
+__device__ __forceinline__ uint32_t nib_pair(uint32_t v, int j, uint32_t mask, uint32_t magic)
 {
-    const uint32_t xs[4] = {xp.x, xp.y, xp.z, xp.w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const uint32_t t = nib_pair(v, j);
-        acc = fma_bf16((uint16_t)(t & 0xFFFFu), (uint16_t)(xs[j] & 0xFFFFu), acc);
-        acc = fma_bf16((uint16_t)(t >> 16), (uint16_t)(xs[j] >> 16), acc);
-    }
-    return acc;
+    return and_or(v >> (4 * j), mask, magic);
 }
 
+// Four 8x8 b16 matrices from shared memory; lane 8i + r supplies the address of row r of
+// matrix i and lane (g, t) receives the 32-bit word (row g, columns 2t, 2t+1) of each.
+__device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+
+// d = A . B + c for one m16n8k16 tile (bf16 inputs, f32 accumulate).
+__device__ __forceinline__ void mma_bf16_16816_c(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                                 uint32_t b0, uint32_t b1, const float4 c)
+{
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%10,%11,%12,%13};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(c.x), "f"(c.y), "f"(c.z), "f"(c.w));
+}
+
+// d += A . B for one m16n8k16 tile (bf16 inputs, f32 accumulate).
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                                uint32_t b0, uint32_t b1)
 {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%10,%11,%12,%13};"
-        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.f), "f"(0.f), "f"(0.f), "f"(0.f));
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
 __device__ __forceinline__ float scale_at(const uint4& s8, int c)
@@ -188,9 +215,9 @@ __device__ __forceinline__ double sum8_bf16(const uint4 raw)
 
 template <int MODE>
 struct ModeCfg {
-    static constexpr int MP = MODE == kMma16 ? 16 : MODE == kMma8 ? 8 : 1;   // padded x rows
+    static constexpr int MP = MODE == kMma16 ? 16 : MODE == kMma8 ? 8 : 1;   // x rows of the MMA tiles
     static constexpr int NT = MP >= 8 ? MP / 8 : 1;                          // n-tiles of 8 x rows
-    static constexpr int kMinBlocks = MODE <= kBf16M1 ? 2 : 1;
+    static constexpr int kMinBlocks = 1;
 };
 
 template <int MODE>
@@ -204,9 +231,9 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
     const int W = blockDim.x >> 5;
     unsigned char* smem =
         reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    unsigned char* codes = smem;                                          // [warp][stage][2048]
-    unsigned char* scl = codes + W * kStages * kCodeBox;                  // [warp][stage][256]
-    uint64_t* bars = reinterpret_cast<uint64_t*>(scl + W * kStages * kScaleBox);   // [warp][stage]
+    unsigned char* codes = smem;                                          // [warp][stage][box][2048]
+    unsigned char* scl = codes + W * kStages * kStageCodes;               // [warp][stage][16 rows][8 * boxes]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(scl + W * kStages * kStageScales);   // [warp][stage]
     float* red = reinterpret_cast<float*>(bars + W * kStages);            // [warp][16 rows][MP]
     unsigned char* xst = reinterpret_cast<unsigned char*>(red + W * kRows * MP);   // staged x (16-byte aligned)
 
@@ -219,7 +246,8 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
     const int ng = min(a.G - g0, a.ksg);
     const int nb = (ng + 7) >> 3;                                         // boxes of this split
     const int ngp = nb * 8;                                               // groups, padded
-    const int b0 = wt * nb / P, nbw = (wt + 1) * nb / P - b0;             // this warp's boxes
+    const int nu = (nb + kBoxesPerStage - 1) / kBoxesPerStage;            // stage units of this split
+    const int u0 = wt * nu / P, nbw = (wt + 1) * nu / P - u0;             // this warp's units
     const int first_rb = blockIdx.x * a.teams + team;
     const int rb_stride = gridDim.x * a.teams;
     const int nrb = (active && first_rb < a.row_blocks) ? (a.row_blocks - first_rb + rb_stride - 1) / rb_stride : 0;
@@ -232,20 +260,31 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
         fence_mbar_init();
     }
     __syncwarp();
-    const ExpandConsts kc = {make_float2(pinned(-8388616.0f), pinned(-524296.0f)),
-                             make_float2(pinned(-32776.0f), pinned(-2056.0f)),
-                             make_float2(pinned(-136.0f), pinned(-32776.0f)),
-                             make_float2(pinned(-2056.0f), pinned(-136.0f))};
+    ExpandConsts kc = {};
+    if constexpr (MODE == kF32M1)
+        kc = {make_float2(pinned(-8388616.0f), pinned(-524296.0f)), make_float2(pinned(-32776.0f), pinned(-2056.0f)),
+              make_float2(pinned(-136.0f), pinned(-32776.0f)), make_float2(pinned(-2056.0f), pinned(-136.0f))};
 
+    // Job j: unit (u0 + j % nbw) of the warp's (j / nbw)-th row block; a unit is up to
+    // kBoxesPerStage consecutive code boxes plus one scale box spanning all of them.  Jobs
+    // are issued in order, so a cursor (unit, row block) replaces the division.
+    int iss_u = 0, iss_rb = first_rb;
     auto issue = [&](int j) {
         const int s = j % kStages;
-        const int rb = first_rb + (j / nbw) * rb_stride;
-        const int b = b0 + j % nbw;
+        const int rb = iss_rb;
+        const int bf = (u0 + iss_u) * kBoxesPerStage;
+        if (++iss_u == nbw) {
+            iss_u = 0;
+            iss_rb += rb_stride;
+        }
+        const int nbox = min(kBoxesPerStage, nb - bf);
         const int mi = matrix_of(a, rb);
         const int lrow = (rb - a.rb_begin[mi]) * kRows;
-        mbar_arrive_expect_tx(&my_bars[s], kCodeBox + kScaleBox);
-        tma_load_2d(codes + (warp * kStages + s) * kCodeBox, &maps.codes[mi], (g0 + 8 * b) * 16, lrow, &my_bars[s]);
-        tma_load_2d(scl + (warp * kStages + s) * kScaleBox, &maps.scales[mi], g0 + 8 * b, lrow, &my_bars[s]);
+        mbar_arrive_expect_tx(&my_bars[s], nbox * kCodeBox + kStageScales);
+        for (int q = 0; q < nbox; ++q)
+            tma_load_2d(codes + ((warp * kStages + s) * kBoxesPerStage + q) * kCodeBox, &maps.codes[mi],
+                        (g0 + 8 * (bf + q)) * 16, lrow, &my_bars[s]);
+        tma_load_2d(scl + (warp * kStages + s) * kStageScales, &maps.scales[mi], g0 + 8 * bf, lrow, &my_bars[s]);
     };
     int issued = min(kStages, njobs);
     // Weights that no kernel still in flight writes may stream before the dependency
@@ -257,12 +296,15 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
     if (!a.prefetch && lane == 0)
         for (int j = 0; j < issued; ++j) issue(j);
 
-    // ---- stage x for this split (zero past the split, past K and past M) ----
-    //  kF32M1 : f32 [group][32]
-    //  kBf16M1: bf16 pairs [group][word][4] + f32 sums of each half group
-    //  kMma*  : bf16 pairs [m][group][word][4] + f32 sums [group][m]
-    // Sums are of the bf16 values in f64, rounded once; neighbouring lanes combine words.
-    float* xsum = nullptr;
+    // ---- stage x for this split (zero past the split and past K) ----
+    //  kF32M1: f32 [group][32]
+    //  kMma* : bf16 pairs [m][group][word][4] for m < M, then one zero row that lanes
+    //          of x rows >= M read; each row is padded by one group so that lanes of
+    //          neighbouring x rows fall on different banks.  Beside it, per group, -136 *
+    //          sum(x) of the group for each x row (an f64 sum of the bf16 values, rounded
+    //          once), laid out [group][n-tile][t] as the accumulator fragment of lane (g, t).
+    float* xoff = nullptr;
+    const int rs = (ngp + 1) * 4;                                         // uint4 per staged x row
     if constexpr (MODE == kF32M1) {
         float4* xf = reinterpret_cast<float4*>(xst);
         for (int i = threadIdx.x; i < ngp * 8; i += blockDim.x) {
@@ -274,8 +316,8 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
         }
     } else {
         uint4* xp = reinterpret_cast<uint4*>(xst);
-        xsum = reinterpret_cast<float*>(xp + MP * ngp * 4);
-        const int total = MP * ngp * 4;
+        xoff = reinterpret_cast<float*>(xp + (a.M + 1) * rs);
+        const int total = (a.M + 1) * ngp * 4;
         for (int i0 = threadIdx.x - lane; i0 < total; i0 += blockDim.x) {    // warp-uniform trips
             const int i = i0 + lane;
             const int m = i / (ngp * 4);
@@ -285,24 +327,42 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
             if (i < total && m < a.M && lg < ng)
                 raw = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(a.x) + (size_t)m * K +
                                                       (size_t)(g0 + lg) * 32 + wd * 8);
-            if (i < total) xp[i] = pairs_of(raw);
+            if (i < total) xp[m * rs + rem] = pairs_of(raw);
             double sum = sum8_bf16(raw);
             sum += __shfl_xor_sync(0xffffffffu, sum, 1);                    // words (0,1) and (2,3)
-            if constexpr (MODE == kBf16M1) {
-                if (i < total && (wd & 1) == 0) xsum[lg * 2 + (wd >> 1)] = (float)sum;
-            } else {
-                sum += __shfl_xor_sync(0xffffffffu, sum, 2);                // all four words
-                if (i < total && wd == 0) xsum[lg * MP + m] = (float)sum;
+            sum += __shfl_xor_sync(0xffffffffu, sum, 2);                    // all four words
+            if (i < total && wd == 0 && m < a.M) {
+                // the accumulator fragment of lane (g, t) holds columns 2t, 2t+1 in both row halves
+                const float o = (float)(-136.0 * sum);
+                const int n = m >> 3, col = m & 7;
+                float* q = xoff + (((size_t)lg * NT + n) * 4 + (col >> 1)) * 4 + (col & 1);
+                q[0] = o;
+                q[2] = o;
+            }
+        }
+        for (int i = threadIdx.x; i < ngp * MP; i += blockDim.x) {
+            const int lg = i / MP, m = i - lg * MP;
+            if (m >= a.M) {
+                const int n = m >> 3, col = m & 7;
+                float* q = xoff + (((size_t)lg * NT + n) * 4 + (col >> 1)) * 4 + (col & 1);
+                q[0] = 0.f;
+                q[2] = 0.f;
             }
         }
     }
     __syncthreads();
 
+    const uint32_t kmask = pinned_u32(0x000F000Fu), kmagic = pinned_u32(0x43004300u);
+    // MMA modes: lane (g, t) supplies the B operand of x row n * 8 + g (the zero row past M).
+    const uint4* xrow[NT];
+#pragma unroll
+    for (int n = 0; n < NT; ++n) xrow[n] = reinterpret_cast<const uint4*>(xst) + min(n * 8 + (lane >> 2), a.M) * rs;
+
     bool ok = true;
     int consumed = 0;
     for (int rbi = 0; rbi < nrb; ++rbi) {
         const int rb = first_rb + rbi * rb_stride;
-        float yacc = 0.f;     // M = 1 modes: row (lane & 15), half (lane >> 4)
+        float yacc = 0.f;     // kF32M1: row (lane & 15), half (lane >> 4)
         float acc[NT][4];     // MMA modes: rows g, g+8; x rows n*8 + 2t, +1
 #pragma unroll
         for (int n = 0; n < NT; ++n)
@@ -315,55 +375,81 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
             if (ok) ok = mbar_wait_bounded(&my_bars[s], (uint32_t)(j / kStages) & 1u, kWaitLimit);
             if (ok) {
                 consumed = j + 1;
-                const unsigned char* cb = codes + (warp * kStages + s) * kCodeBox;
-                const unsigned char* sb = scl + (warp * kStages + s) * kScaleBox;
-                const int gb = (b0 + jb) * 8;                                 // first group of the box
-                if constexpr (MODE == kF32M1 || MODE == kBf16M1) {
-                    const int r = lane & 15, h = lane >> 4;
-                    const unsigned char* rowp = cb + r * 128 + h * 8;
-                    const uint4 s8 = *reinterpret_cast<const uint4*>(sb + r * 16);
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        const uint2 w2 = *reinterpret_cast<const uint2*>(rowp + ((c ^ (r & 7)) << 4));
-                        float part;
+                const int bf = (u0 + jb) * kBoxesPerStage;
+                const int nbox = min(kBoxesPerStage, nb - bf);
+#pragma unroll 1
+                for (int q = 0; q < nbox; ++q) {
+                    {
+                        const unsigned char* cb = codes + ((warp * kStages + s) * kBoxesPerStage + q) * kCodeBox;
+                        const unsigned char* sb = scl + (warp * kStages + s) * kStageScales + q * 16;
+                        constexpr int kScaleRow = 16 * kBoxesPerStage;   // bytes per row of the scale box
+                        const int gb = (bf + q) * 8;                     // first group of the box
                         if constexpr (MODE == kF32M1) {
-                            const float4* xg = reinterpret_cast<const float4*>(xst) + (gb + c) * 8 + h * 4;
-                            const float2 q = __fadd2_rn(word_dot_f32(w2.x, xg, kc), word_dot_f32(w2.y, xg + 2, kc));
-                            part = q.x + q.y;
+                            const int r = lane & 15, h = lane >> 4;
+                            const unsigned char* rowp = cb + r * 128 + h * 8;
+                            const uint4 s8 = *reinterpret_cast<const uint4*>(sb + r * kScaleRow);
+#pragma unroll
+                            for (int c = 0; c < 8; ++c) {
+                                const uint2 w2 = *reinterpret_cast<const uint2*>(rowp + ((c ^ (r & 7)) << 4));
+                                const float4* xg = reinterpret_cast<const float4*>(xst) + (gb + c) * 8 + h * 4;
+                                const float2 d2 =
+                                    __fadd2_rn(word_dot_f32(w2.x, xg, kc), word_dot_f32(w2.y, xg + 2, kc));
+                                yacc = fmaf(scale_at(s8, c), d2.x + d2.y, yacc);
+                            }
                         } else {
-                            const uint4* xpg = reinterpret_cast<const uint4*>(xst) + (gb + c) * 4 + h * 2;
-                            const float a0 = word_dot_bf16(w2.x, xpg[0], 0.f);
-                            const float a1 = word_dot_bf16(w2.y, xpg[1], 0.f);
-                            part = fmaf(-136.0f, xsum[(gb + c) * 2 + h], a0 + a1);   // remove 128 + 8
-                        }
-                        yacc = fmaf(scale_at(s8, c), part, yacc);
-                    }
-                } else {
-                    const int g = lane >> 2, t = lane & 3;
-                    const uint4 sg = *reinterpret_cast<const uint4*>(sb + g * 16);
-                    const uint4 sg8 = *reinterpret_cast<const uint4*>(sb + (g + 8) * 16);
-                    const uint4* xp = reinterpret_cast<const uint4*>(xst);
+                            const int g = lane >> 2, t = lane & 3;
+                            const uint4 sg = *reinterpret_cast<const uint4*>(sb + g * kScaleRow);
+                            const uint4 sg8 = *reinterpret_cast<const uint4*>(sb + (g + 8) * kScaleRow);
+                            // ldmatrix rows: lane 8i + r -> weight row 8 (i & 1) + r of group
+                            // 2 cp + (i >> 1); with the 128-byte swizzle the chunk of group c in
+                            // row r sits at (c ^ (r & 7)) * 16, so group pair cp is one XOR away.
+                            const int lr = lane & 7, li = lane >> 3;
+                            const uint32_t abase =
+                                smem_addr(cb) + ((li & 1) * 8 + lr) * 128 + (((li >> 1) ^ lr) << 4);
+                            // All MMAs of a batch of groups are issued before any result is
+                            // read, so the tensor-core latency overlaps across groups.
+                            constexpr int GB = NT == 1 ? 8 : 4;            // groups per batch
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        const int off = ((c ^ g) << 4) + 4 * t;                 // (g & 7) == g
-                        const uint32_t w0 = *reinterpret_cast<const uint32_t*>(cb + g * 128 + off);
-                        const uint32_t w1 = *reinterpret_cast<const uint32_t*>(cb + (g + 8) * 128 + off);
-                        const uint32_t A0 = nib_pair(w0, 0), A1 = nib_pair(w1, 0), A2 = nib_pair(w0, 1),
-                                       A3 = nib_pair(w1, 1);
-                        const uint32_t A4 = nib_pair(w0, 2), A5 = nib_pair(w1, 2), A6 = nib_pair(w0, 3),
-                                       A7 = nib_pair(w1, 3);
-                        const float s0 = scale_at(sg, c), s1 = scale_at(sg8, c);
+                            for (int c0 = 0; c0 < 8; c0 += GB) {
+                                float d[GB][NT][4];
 #pragma unroll
-                        for (int n = 0; n < NT; ++n) {
-                            const uint4 bx = xp[((n * 8 + g) * ngp + gb + c) * 4 + t];
-                            float d0[4], d1[4];
-                            mma_bf16_16816(d0, A0, A1, A2, A3, bx.x, bx.y);
-                            mma_bf16_16816(d1, A4, A5, A6, A7, bx.z, bx.w);
-                            const float2 xs2 = *reinterpret_cast<const float2*>(xsum + (gb + c) * MP + n * 8 + 2 * t);
-                            acc[n][0] = fmaf(s0, fmaf(-136.0f, xs2.x, d0[0] + d1[0]), acc[n][0]);
-                            acc[n][1] = fmaf(s0, fmaf(-136.0f, xs2.y, d0[1] + d1[1]), acc[n][1]);
-                            acc[n][2] = fmaf(s1, fmaf(-136.0f, xs2.x, d0[2] + d1[2]), acc[n][2]);
-                            acc[n][3] = fmaf(s1, fmaf(-136.0f, xs2.y, d0[3] + d1[3]), acc[n][3]);
+                                for (int cp = c0 / 2; cp < (c0 + GB) / 2; ++cp) {
+                                    uint32_t r0, r1, r2, r3;  // word t of rows g, g+8 for groups 2cp, 2cp+1
+                                    ldmatrix_x4(abase ^ (uint32_t)(cp << 5), r0, r1, r2, r3);
+#pragma unroll
+                                    for (int h = 0; h < 2; ++h) {
+                                        const int c = 2 * cp + h;
+                                        const uint32_t w0 = h ? r2 : r0, w1 = h ? r3 : r1;
+                                        const uint32_t A0 = nib_pair(w0, 0, kmask, kmagic);
+                                        const uint32_t A1 = nib_pair(w1, 0, kmask, kmagic);
+                                        const uint32_t A2 = nib_pair(w0, 1, kmask, kmagic);
+                                        const uint32_t A3 = nib_pair(w1, 1, kmask, kmagic);
+                                        const uint32_t A4 = nib_pair(w0, 2, kmask, kmagic);
+                                        const uint32_t A5 = nib_pair(w1, 2, kmask, kmagic);
+                                        const uint32_t A6 = nib_pair(w0, 3, kmask, kmagic);
+                                        const uint32_t A7 = nib_pair(w1, 3, kmask, kmagic);
+#pragma unroll
+                                        for (int n = 0; n < NT; ++n) {
+                                            const uint4 bx = xrow[n][(gb + c) * 4 + t];
+                                            const float4 o4 = reinterpret_cast<const float4*>(
+                                                xoff)[((gb + c) * NT + n) * 4 + t];      // -136 * sum(x)
+                                            mma_bf16_16816_c(d[c - c0][n], A0, A1, A2, A3, bx.x, bx.y, o4);
+                                            mma_bf16_16816(d[c - c0][n], A4, A5, A6, A7, bx.z, bx.w);
+                                        }
+                                    }
+                                }
+#pragma unroll
+                                for (int c = c0; c < c0 + GB; ++c) {
+                                    const float s0 = scale_at(sg, c), s1 = scale_at(sg8, c);
+#pragma unroll
+                                    for (int n = 0; n < NT; ++n) {
+                                        acc[n][0] = fmaf(s0, d[c - c0][n][0], acc[n][0]);
+                                        acc[n][1] = fmaf(s0, d[c - c0][n][1], acc[n][1]);
+                                        acc[n][2] = fmaf(s1, d[c - c0][n][2], acc[n][2]);
+                                        acc[n][3] = fmaf(s1, d[c - c0][n][3], acc[n][3]);
+                                    }
+                                }
+                            }
                         }
                     }
                 }
@@ -380,7 +466,7 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
 
         // ---- row block rb complete: partials -> red[warp][row][m], team sum in warp order ----
         float* my_red = red + warp * kRows * MP;
-        if constexpr (MODE == kF32M1 || MODE == kBf16M1) {
+        if constexpr (MODE == kF32M1) {
             yacc += __shfl_xor_sync(0xffffffffu, yacc, 16);           // the two halves of each row
             if (lane < 16) my_red[lane] = yacc;
         } else {
@@ -434,24 +520,31 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
     if (!ok) {
         if (lane == 0) atomicOr(a.err, kErrWaitTimeout);
         for (int j = consumed; j < issued; ++j)    // copies still in flight into this warp's ring
-            mbar_wait_bounded(&my_bars[j % kStages], (uint32_t)(j / kStages) & 1u, kWaitLimit);
+            if (!mbar_wait_bounded(&my_bars[j % kStages], (uint32_t)(j / kStages) & 1u, kWaitLimit)) break;
     }
 }
 
-size_t smem_bytes(int mode, int warps, int nb)
+size_t per_warp_bytes(int mode)
 {
     const int mp = mode == kMma16 ? 16 : mode == kMma8 ? 8 : 1;
-    const size_t ring = (size_t)warps * kStages * (kCodeBox + kScaleBox) + warps * kStages * sizeof(uint64_t);
-    const size_t red = (size_t)warps * kRows * mp * sizeof(float);
+    return (size_t)kStages * (kStageCodes + kStageScales + sizeof(uint64_t)) + (size_t)kRows * mp * sizeof(float);
+}
+
+size_t x_stage_bytes(int mode, int nb, int64_t M)
+{
+    const int mp = mode == kMma16 ? 16 : mode == kMma8 ? 8 : 1;
     const size_t ngp = (size_t)nb * 8;
-    const size_t xs = mode == kF32M1 ? ngp * 32 * sizeof(float)
-                                     : (size_t)mp * ngp * 64 + ngp * (mode == kBf16M1 ? 2 : mp) * sizeof(float);
-    return 1024 + ring + red + xs;
+    return mode == kF32M1 ? ngp * 32 * sizeof(float) : (size_t)(M + 1) * (ngp + 1) * 64 + ngp * (mp / 8) * 64;
+}
+
+size_t smem_bytes(int mode, int warps, int nb, int64_t M)
+{
+    return 1024 + (size_t)warps * per_warp_bytes(mode) + x_stage_bytes(mode, nb, M);
 }
 
 int mode_for(int64_t M, q4_dtype xt)
 {
-    if (M == 1) return xt == Q4_BF16 ? kBf16M1 : kF32M1;
+    if (M == 1 && xt == Q4_F32) return kF32M1;
     return M <= 8 ? kMma8 : kMma16;
 }
 
@@ -459,7 +552,6 @@ const void* kernel_for(int mode)
 {
     switch (mode) {
     case kF32M1: return reinterpret_cast<const void*>(&gemv_tma_kernel<kF32M1>);
-    case kBf16M1: return reinterpret_cast<const void*>(&gemv_tma_kernel<kBf16M1>);
     case kMma8: return reinterpret_cast<const void*>(&gemv_tma_kernel<kMma8>);
     default: return reinterpret_cast<const void*>(&gemv_tma_kernel<kMma16>);
     }
@@ -484,27 +576,59 @@ bool plan_gemv_tma(int64_t M, const int64_t* Ns, int count, int64_t K, q4_dtype 
     if (rbl < 1 || rbl > INT32_MAX / kRows) return false;
     const int row_blocks = (int)rbl;
     const int boxes = (G + 7) / 8;
-    const long long warp_slots = (long long)dev.sm_count * (mode <= kBf16M1 ? 2 : 1) * kMaxWarps;
-    // Team size: enough warps per row block to fill the SMs, at most one per box.
-    int P = 1;
-    if ((long long)row_blocks < warp_slots) {
-        const long long want = (warp_slots + row_blocks - 1) / row_blocks;
-        P = (int)(want < boxes ? want : boxes);
-        if (P > kMaxWarps) P = kMaxWarps;
-        if (P < 1) P = 1;
+    const int units = (boxes + kBoxesPerStage - 1) / kBoxesPerStage;
+    const size_t pw = per_warp_bytes(mode);
+    const size_t budget = (size_t)dev.max_smem_optin - 512;   // room for the kernel's static arrays
+    // Boxes of the widest split when K is cut into `sp` splits of whole units.
+    auto split_boxes = [&](int sp) {
+        const int b = (units + sp - 1) / sp * kBoxesPerStage;
+        return b < boxes ? b : boxes;
+    };
+    // Splits forced by shared memory: the staged x of one split leaves room for 4 warps.
+    int splits_min = 1;
+    while (1024 + 4 * pw + x_stage_bytes(mode, split_boxes(splits_min), M) > budget) {
+        if (split_boxes(splits_min) <= kBoxesPerStage) return false;
+        ++splits_min;
     }
-    // Still short of work: split K across blocks (each warp keeps >= 1 box).
-    int splits = 1;
-    while ((long long)row_blocks * P * splits < warp_slots / 2 && boxes / (splits + 1) >= P &&
-           row_blocks <= kCounterSlots)
-        ++splits;
-    const int ksg = ((G + splits - 1) / splits + 7) / 8 * 8;
-    splits = (G + ksg - 1) / ksg;
-    const int nb = (ksg + 7) / 8;
-    const int teams = P == 1 ? kMaxWarps : (kMaxWarps / P > 0 ? kMaxWarps / P : 1);
+    // Choose the K splits, the team size P and the teams per block by a cost model of the
+    // busiest block: rounds of row blocks x units per warp x warps sharing the SM, plus
+    // the row-block epilogue and, for a split K, the reduction of partial sums.  Teams
+    // per block are capped so that small problems spread over all SMs.
+    int splits = 0, P = 0, teams = 0;
+    double best = 0.0;
+    const int max_splits = row_blocks <= kCounterSlots ? units : splits_min;
+    for (int sp = splits_min; sp <= max_splits; ++sp) {
+        const int nbs = split_boxes(sp);
+        if ((boxes + nbs - 1) / nbs != sp) continue;                  // same cut as fewer splits
+        const size_t xs = x_stage_bytes(mode, nbs, M);
+        if (1024 + pw + xs > budget) continue;
+        const size_t fitw = (budget - 1024 - xs) / pw;
+        const int wbs = (int)(fitw < (size_t)kMaxWarps ? fitw : (size_t)kMaxWarps);
+        const int nus = (nbs + kBoxesPerStage - 1) / kBoxesPerStage;
+        const long long sms = dev.sm_count / sp > 0 ? dev.sm_count / sp : 1;   // blocks of one split
+        for (int pp = 1; pp <= nus && pp <= wbs; ++pp) {
+            const int pwu = (nus + pp - 1) / pp;                          // units per warp per row block
+            long long tm = wbs / pp;
+            const long long spread = ((long long)row_blocks + sms - 1) / sms;
+            if (tm > spread) tm = spread;
+            const long long gxs = std::min(((long long)row_blocks + tm - 1) / tm, sms);
+            const long long rounds = ((long long)row_blocks + gxs * tm - 1) / (gxs * tm);
+            const double share = std::max((double)(tm * pp), kMinWarpShare) / 16.0;
+            const double cost = (double)rounds * (pwu + kEpilogueCost) * share + (sp > 1 ? kSplitCost : 0.0);
+            if (splits == 0 || cost < best - 1e-9) {
+                splits = sp;
+                P = pp;
+                teams = (int)tm;
+                best = cost;
+            }
+        }
+    }
+    if (splits == 0) return false;
+    const int ksg = split_boxes(splits) * 8;
+    const int nb = ksg / 8;
     const int warps = P * teams;
-    const size_t smem = smem_bytes(mode, warps, nb);
-    if (smem > (size_t)dev.max_smem_optin) return false;
+    const size_t smem = smem_bytes(mode, warps, nb, M);
+    if (smem > budget) return false;
     const void* fn = kernel_for(mode);
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) {
         cudaGetLastError();
@@ -516,7 +640,7 @@ bool plan_gemv_tma(int64_t M, const int64_t* Ns, int count, int64_t K, q4_dtype 
         return false;
     }
     const long long blocks_needed = ((long long)row_blocks + teams - 1) / teams;
-    long long gx = ((long long)dev.sm_count * per_sm + splits - 1) / splits;
+    long long gx = (long long)dev.sm_count * per_sm / splits;
     if (gx > blocks_needed) gx = blocks_needed;
     if (gx < 1) gx = 1;
     p->kernel = 1;
@@ -543,7 +667,7 @@ q4_status launch_gemv_tma(const void* x, q4_dtype xt, int64_t M, int64_t K, cons
         if (!encode_tma_2d(&maps.codes[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, mats[i].packed, (uint64_t)K / 2,
                            (uint64_t)mats[i].N, (uint64_t)K / 2, 128, kRows, CU_TENSOR_MAP_SWIZZLE_128B) ||
             !encode_tma_2d(&maps.scales[i], CU_TENSOR_MAP_DATA_TYPE_UINT16, mats[i].scales, G, (uint64_t)mats[i].N,
-                           G * 2, 8, kRows, CU_TENSOR_MAP_SWIZZLE_NONE))
+                           G * 2, 8 * kBoxesPerStage, kRows, CU_TENSOR_MAP_SWIZZLE_NONE))
             return Q4_ERR_CUDA;
         a.y[i] = mats[i].y;
         a.N[i] = (int)mats[i].N;

@@ -130,7 +130,7 @@ def test_misaligned_scales_take_generic_path():
 
 def test_too_small_workspace_rejected():
     import bit_weight_only_quantize_b200 as q4
-    M, N, K = 1, 16, 8192
+    M, N, K = 1, 16, 32768
     assert q4.gemv_workspace_size(M, N, K) > 16      # the shape splits K
     ws = torch.zeros(16, dtype=torch.uint8, device="cuda")
     x = torch.zeros((M, K), dtype=torch.bfloat16, device="cuda")
