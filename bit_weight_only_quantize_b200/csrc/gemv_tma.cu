@@ -267,24 +267,29 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
 
     // Job j: unit (u0 + j % nbw) of the warp's (j / nbw)-th row block; a unit is up to
     // kBoxesPerStage consecutive code boxes plus one scale box spanning all of them.  Jobs
-    // are issued in order, so a cursor (unit, row block) replaces the division.
-    int iss_u = 0, iss_rb = first_rb;
+    // are issued in order, so a cursor (unit, row block and its matrix) replaces the
+    // division and the matrix lookup.
+    int iss_u = 0, iss_rb = first_rb, iss_mi = 0, iss_lrow = 0;
+    auto locate = [&]() {
+        iss_mi = matrix_of(a, iss_rb);
+        iss_lrow = (iss_rb - a.rb_begin[iss_mi]) * kRows;
+    };
+    if (lane == 0 && njobs > 0) locate();
     auto issue = [&](int j) {
         const int s = j % kStages;
-        const int rb = iss_rb;
         const int bf = (u0 + iss_u) * kBoxesPerStage;
+        const int nbox = min(kBoxesPerStage, nb - bf);
+        uint64_t* bar = &my_bars[s];
+        const CUtensorMap* cmap = &maps.codes[iss_mi];
+        unsigned char* dst = codes + (warp * kStages + s) * kStageCodes;
+        mbar_arrive_expect_tx(bar, nbox * kCodeBox + kStageScales);
+        for (int q = 0; q < nbox; ++q) tma_load_2d(dst + q * kCodeBox, cmap, (g0 + 8 * (bf + q)) * 16, iss_lrow, bar);
+        tma_load_2d(scl + (warp * kStages + s) * kStageScales, &maps.scales[iss_mi], g0 + 8 * bf, iss_lrow, bar);
         if (++iss_u == nbw) {
             iss_u = 0;
             iss_rb += rb_stride;
+            if (j + 1 < njobs) locate();
         }
-        const int nbox = min(kBoxesPerStage, nb - bf);
-        const int mi = matrix_of(a, rb);
-        const int lrow = (rb - a.rb_begin[mi]) * kRows;
-        mbar_arrive_expect_tx(&my_bars[s], nbox * kCodeBox + kStageScales);
-        for (int q = 0; q < nbox; ++q)
-            tma_load_2d(codes + ((warp * kStages + s) * kBoxesPerStage + q) * kCodeBox, &maps.codes[mi],
-                        (g0 + 8 * (bf + q)) * 16, lrow, &my_bars[s]);
-        tma_load_2d(scl + (warp * kStages + s) * kStageScales, &maps.scales[mi], g0 + 8 * bf, lrow, &my_bars[s]);
     };
     int issued = min(kStages, njobs);
     // Weights that no kernel still in flight writes may stream before the dependency
@@ -485,11 +490,11 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
             const int nrow = a.N[mi];
             const int lrow0 = (rb - a.rb_begin[mi]) * kRows;
             const size_t vrows = (size_t)a.row_blocks * kRows;            // padded rows over all matrices
-            for (int e = lane; e < kRows * MP; e += 32) {
-                const int rr = e / MP, m = e - rr * MP;
+            for (int e = lane; e < kRows * a.M; e += 32) {           // x row major: coalesced y
+                const int m = e / kRows, rr = e - m * kRows;
                 float total = 0.f;
-                for (int w = 0; w < P; ++w) total += red[(team * P + w) * kRows * MP + e];
-                if (m < a.M && lrow0 + rr < nrow) {
+                for (int w = 0; w < P; ++w) total += red[(team * P + w) * kRows * MP + rr * MP + m];
+                if (lrow0 + rr < nrow) {
                     if (a.splits == 1) a.y[mi][(size_t)m * nrow + lrow0 + rr] = total;
                     else a.partial[((size_t)split * a.M + m) * vrows + (size_t)rb * kRows + rr] = total;
                 }
