@@ -10,14 +10,16 @@
 //   w_bf16 = bf16_rn((code - 8) * f32(scale))      (the f32 product is exact, one rounding)
 //
 // One persistent block per SM, warp-specialised:
-//   warp 0      TMA producer: x tiles (128 rows x 64 k, 128-byte swizzle) and the raw
-//               codes of the weight tile (BN rows x 32 bytes) into a ring of kStages.
+//   warp 0      TMA producer: x tiles (128 rows x 64 k, 128-byte swizzle), the raw
+//               codes of the weight tile (BN rows x 32 bytes) and, when K % 256 == 0,
+//               the 16-byte row of scales around the stage's two groups into a ring of
+//               kStages.
 //   warp 1      allocates tensor memory; one thread issues the MMAs (128 x BN x 16
 //               per instruction, MA accumulators of 128 rows per tile) and commits.
 //   warps 2..5  epilogue: tcgen05.ld of the accumulator lanes, f32 -> bf16, stores.
 //   warps 6..21 dequantise: codes -> bf16 in the K-major 128-byte-swizzled layout the
-//               MMA descriptor expects, scales read from global (prefetched two
-//               k-blocks ahead), then fence.proxy.async and arrive on the stage.
+//               MMA descriptor expects, scales from the stage (or, for other K, read
+//               from global two k-blocks ahead), then fence.proxy.async and arrive.
 // Accumulators are double-buffered in tensor memory, so the epilogue of one tile
 // overlaps the MMAs of the next.  Every mbarrier wait is bounded; on a timeout the
 // block records kErrWaitTimeout, all roles stop, outstanding copies and MMAs are
@@ -38,6 +40,7 @@ constexpr uint64_t kWaitLimit = kWaitLimitNs;
 
 struct GemmArgs {
     const uint16_t* scales;
+    int scale_tma;                    // scales arrive by TMA with each stage (needs K % 256 == 0)
     uint16_t* y;
     unsigned* err;
     int M, N, K, G;
@@ -140,7 +143,8 @@ struct GemmCfg {
     static constexpr uint32_t kABytes = 128 * kBK * 2;            // one 128-row x tile: 16 KiB
     static constexpr uint32_t kBBytes = BN * kBK * 2;             // dequantised weight tile
     static constexpr uint32_t kRawBytes = BN * (kBK / 2);         // raw codes
-    static constexpr uint32_t kStageBytes = MA * kABytes + kBBytes + kRawBytes;
+    static constexpr uint32_t kScaleBytes = BN * 16;              // scales: 8 groups x BN rows
+    static constexpr uint32_t kStageBytes = MA * kABytes + kBBytes + kRawBytes + kScaleBytes;
     static constexpr uint32_t kTxBytes = MA * kABytes + kRawBytes;
     static constexpr uint32_t kTmemCols = 2 * MA * BN;            // double-buffered accumulators
     static constexpr size_t kSmem = 1024 + (size_t)kStages * kStageBytes + 256;
@@ -150,14 +154,15 @@ struct GemmCfg {
 template <int MA, int BN>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_codes,
-               const GemmArgs a)
+               const __grid_constant__ CUtensorMap tm_scales, const GemmArgs a)
 {
     using C = GemmCfg<MA, BN>;
     constexpr int S = C::kStages;
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem =
         reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    // Per stage: [MA x A tile][B tile][raw codes]; A and B tiles are 1024-byte aligned.
+    // Per stage: [MA x A tile][B tile][raw codes][scales]; A and B tiles are 1024-byte
+    // aligned.  The scale box holds the 8 groups around the stage's 2 (a 16-byte row).
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes);
     uint64_t* full = bars;               // producer -> dequant   (TMA bytes)
     uint64_t* bready = bars + S;         // dequant -> MMA        (kDeqWarps arrivals)
@@ -186,6 +191,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         fence_mbar_init();
         tma_prefetch_desc(&tm_x);
         tma_prefetch_desc(&tm_codes);
+        if (a.scale_tma) tma_prefetch_desc(&tm_scales);
     }
     if (warp == kMmaWarp) {
         tmem_alloc(tmem_slot, C::kTmemCols);
@@ -218,10 +224,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                     if (!mbar_wait_bounded(&empty[s], ph ^ 1u, kWaitLimit)) { fail(); break; }
                     if (*abort_flag) break;
                     unsigned char* st = smem + s * C::kStageBytes;
-                    mbar_arrive_expect_tx(&full[s], C::kTxBytes);
+                    mbar_arrive_expect_tx(&full[s], C::kTxBytes + (a.scale_tma ? C::kScaleBytes : 0u));
                     for (int am = 0; am < MA; ++am)
                         tma_load_2d(st + am * C::kABytes, &tm_x, kb * kBK, m0 + am * 128, &full[s]);
                     tma_load_2d(st + MA * C::kABytes + C::kBBytes, &tm_codes, kb * (kBK / 2), n0, &full[s]);
+                    if (a.scale_tma)           // 16-byte aligned: group (2 kb) rounded down to 8
+                        tma_load_2d(st + MA * C::kABytes + C::kBBytes + C::kRawBytes, &tm_scales, (kb * 2) & ~7, n0,
+                                    &full[s]);
                     last_phase[s] = (int)ph;
                 }
             }
@@ -327,23 +336,27 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                                  : 0.f;
                 }
             };
-            load_scales(0, sc0);
-            load_scales(1, sc1);
+            if (!a.scale_tma) {
+                load_scales(0, sc0);
+                load_scales(1, sc1);
+            }
             bool ok = true;
             for (int kb = 0; kb < a.kblocks; ++kb, ++it) {
-                load_scales(kb + 2, sc2);
+                if (!a.scale_tma) load_scales(kb + 2, sc2);
                 const int s = it % S;
                 if (!mbar_wait_bounded(&full[s], (uint32_t)(it / S) & 1u, kWaitLimit)) { fail(); ok = false; break; }
                 if (*abort_flag) { ok = false; break; }
                 unsigned char* st = smem + s * C::kStageBytes;
                 unsigned char* bt = st + MA * C::kABytes;
                 const unsigned char* raw = bt + C::kBBytes;
+                const __half* sst = reinterpret_cast<const __half*>(raw + C::kRawBytes);
 #pragma unroll
                 for (int q = 0; q < kChunks; ++q) {
                     const int idx = dt + q * kDeqWarps * 32;
                     const int n = idx >> 3, c = idx & 7;
                     const uint32_t v = *reinterpret_cast<const uint32_t*>(raw + n * 32 + c * 4);
-                    *reinterpret_cast<uint4*>(bt + n * 128 + ((c ^ (n & 7)) << 4)) = dequant8(v, sc0[q]);
+                    const float sc = a.scale_tma ? __half2float(sst[n * 8 + ((kb * 2 + c / 4) & 7)]) : sc0[q];
+                    *reinterpret_cast<uint4*>(bt + n * 128 + ((c ^ (n & 7)) << 4)) = dequant8(v, sc);
                 }
                 fence_proxy_async_smem();      // generic-proxy writes -> tensor-core reads
                 __syncwarp();
@@ -394,11 +407,18 @@ q4_status launch_gemm(const uint16_t* x, int64_t M, int64_t K, const uint8_t* pa
         !encode_tma_2d(&tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2,
                        kBK / 2, (uint32_t)BN, CU_TENSOR_MAP_SWIZZLE_NONE))
         return Q4_ERR_CUDA;
+    // Scales by TMA when a row of them is a whole number of 16-byte units and 16-byte aligned.
+    CUtensorMap tm_scales = tm_codes;
+    const bool scale_tma = (K / 32) % 8 == 0 && (reinterpret_cast<uintptr_t>(scales) & 15) == 0;
+    if (scale_tma && !encode_tma_2d(&tm_scales, CU_TENSOR_MAP_DATA_TYPE_UINT16, scales, (uint64_t)(K / 32),
+                                    (uint64_t)N, (uint64_t)(K / 32) * 2, 8, (uint32_t)BN, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return Q4_ERR_CUDA;
     unsigned* err = device_error_word();
     if (!err) return Q4_ERR_CUDA;
 
     GemmArgs a;
     a.scales = scales;
+    a.scale_tma = scale_tma ? 1 : 0;
     a.y = y;
     a.err = err;
     a.M = (int)M;
@@ -425,9 +445,9 @@ q4_status launch_gemm(const uint16_t* x, int64_t M, int64_t K, const uint8_t* pa
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     cudaError_t e;
-    if (MA == 2) e = cudaLaunchKernelEx(&cfg, gemm_tc_kernel<2, 128>, tm_x, tm_codes, a);
-    else if (BN == 128) e = cudaLaunchKernelEx(&cfg, gemm_tc_kernel<1, 128>, tm_x, tm_codes, a);
-    else e = cudaLaunchKernelEx(&cfg, gemm_tc_kernel<1, 64>, tm_x, tm_codes, a);
+    if (MA == 2) e = cudaLaunchKernelEx(&cfg, gemm_tc_kernel<2, 128>, tm_x, tm_codes, tm_scales, a);
+    else if (BN == 128) e = cudaLaunchKernelEx(&cfg, gemm_tc_kernel<1, 128>, tm_x, tm_codes, tm_scales, a);
+    else e = cudaLaunchKernelEx(&cfg, gemm_tc_kernel<1, 64>, tm_x, tm_codes, tm_scales, a);
     return e == cudaSuccess ? Q4_OK : Q4_ERR_CUDA;
 }
 
