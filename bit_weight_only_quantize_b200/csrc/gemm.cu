@@ -116,18 +116,51 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
     return r;
 }
 
+// (a & m) | c as one LOP3 with all three operands in registers (the instruction takes a
+// single immediate, so constant masks and magics are kept in registers by the caller).
+__device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t m, uint32_t c)
+{
+    uint32_t r;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(a), "r"(m), "r"(c));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t pinned_u32(uint32_t v)
+{
+    uint32_t r;
+    asm volatile("mov.b32 %0, %1;" : "=r"(r) : "r"(v));
+    return r;
+}
+
+// Constants of dequant8 held in registers: nibble masks 0xF << 4i and the exponents
+// 2^(23-4i) whose mantissa a nibble at bit 4i lands in.
+struct DequantConsts {
+    uint32_t mask[5], magic[5];
+    __device__ __forceinline__ DequantConsts()
+    {
+#pragma unroll
+        for (int i = 0; i < 5; ++i) {
+            mask[i] = pinned_u32(0xFu << (4 * i));
+            magic[i] = pinned_u32((uint32_t)(150 - 4 * i) << 23);
+        }
+    }
+};
+
 // Eight codes of one word -> eight bf16 values (code - 8) * s in k order, rounded once.
-__device__ __forceinline__ uint4 dequant8(uint32_t v, float s)
+// Nibble i OR-ed into the mantissa of 2^(23-4i) is exactly 2^(23-4i) + code; a packed
+// add removes 2^(23-4i) + 8 exactly, the packed multiply by s is exact (a 4-bit integer
+// times a binary16 value fits in f32), and cvt.rn.bf16x2 rounds once.
+__device__ __forceinline__ uint4 dequant8(uint32_t v, float s, const DequantConsts& k)
 {
     const uint32_t u = v >> 12;
-    const float f0 = __uint_as_float((v & 0x0000000Fu) | 0x4B000000u);
-    const float f1 = __uint_as_float((v & 0x000000F0u) | 0x49000000u);
-    const float f2 = __uint_as_float((v & 0x00000F00u) | 0x47000000u);
-    const float f3 = __uint_as_float((v & 0x0000F000u) | 0x45000000u);
-    const float f4 = __uint_as_float((v & 0x000F0000u) | 0x43000000u);
-    const float f5 = __uint_as_float((u & 0x00000F00u) | 0x47000000u);
-    const float f6 = __uint_as_float((u & 0x0000F000u) | 0x45000000u);
-    const float f7 = __uint_as_float((u & 0x000F0000u) | 0x43000000u);
+    const float f0 = __uint_as_float(and_or(v, k.mask[0], k.magic[0]));   // 2^23 + c0
+    const float f1 = __uint_as_float(and_or(v, k.mask[1], k.magic[1]));   // 2^19 + c1
+    const float f2 = __uint_as_float(and_or(v, k.mask[2], k.magic[2]));   // 2^15 + c2
+    const float f3 = __uint_as_float(and_or(v, k.mask[3], k.magic[3]));   // 2^11 + c3
+    const float f4 = __uint_as_float(and_or(v, k.mask[4], k.magic[4]));   // 2^7  + c4
+    const float f5 = __uint_as_float(and_or(u, k.mask[2], k.magic[2]));   // 2^15 + c5
+    const float f6 = __uint_as_float(and_or(u, k.mask[3], k.magic[3]));   // 2^11 + c6
+    const float f7 = __uint_as_float(and_or(u, k.mask[4], k.magic[4]));   // 2^7  + c7
     const float2 ss = make_float2(s, s);
     const float2 d01 = __fmul2_rn(__fadd2_rn(make_float2(f0, f1), make_float2(-8388616.0f, -524296.0f)), ss);
     const float2 d23 = __fmul2_rn(__fadd2_rn(make_float2(f2, f3), make_float2(-32776.0f, -2056.0f)), ss);
@@ -321,6 +354,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         // Dequantise: each thread owns BN*8/256 chunks (row n, 16-byte k chunk c) of every stage.
         const int dt = threadIdx.x - kDeqWarp0 * 32;
         constexpr int kChunks = BN * 8 / (kDeqWarps * 32);
+        const DequantConsts dk;
         int it = 0;
         for (int t = blockIdx.x; t < tiles && !*abort_flag; t += gridDim.x) {
             const int n0 = (t / a.tiles_m) * BN;
@@ -356,7 +390,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                     const int n = idx >> 3, c = idx & 7;
                     const uint32_t v = *reinterpret_cast<const uint32_t*>(raw + n * 32 + c * 4);
                     const float sc = a.scale_tma ? __half2float(sst[n * 8 + ((kb * 2 + c / 4) & 7)]) : sc0[q];
-                    *reinterpret_cast<uint4*>(bt + n * 128 + ((c ^ (n & 7)) << 4)) = dequant8(v, sc);
+                    *reinterpret_cast<uint4*>(bt + n * 128 + ((c ^ (n & 7)) << 4)) = dequant8(v, sc, dk);
                 }
                 fence_proxy_async_smem();      // generic-proxy writes -> tensor-core reads
                 __syncwarp();
