@@ -58,7 +58,7 @@ constexpr double kEpilogueCost = 0.1;
 constexpr double kSplitCost = 0.9;
 constexpr size_t kCounterBytes = kCounterSlots * sizeof(unsigned);
 
-enum Mode { kF32M1 = 0, kMma8 = 1, kMma16 = 2 };
+enum Mode { kF32M1 = 0, kMma8 = 1, kMma16 = 2, kMma1 = 3 };   // kMma1: kMma8 with one x row
 
 struct TmaMaps {
     CUtensorMap codes[Q4_MULTI_MAX];
@@ -109,35 +109,6 @@ __device__ __forceinline__ float pinned(float v)
     return r;
 }
 
-struct ExpandConsts {
-    float2 c01, c23, c45, c67;
-};
-
-// f32 x: eight codes of one word dotted with eight x values (exact code - 8).
-__device__ __forceinline__ float2 word_dot_f32(uint32_t v, const float4* xw, const ExpandConsts& k)
-{
-    const uint32_t u = v >> 12;
-    const float f0 = __uint_as_float((v & 0x0000000Fu) | 0x4B000000u);   // 2^23 + c0
-    const float f1 = __uint_as_float((v & 0x000000F0u) | 0x49000000u);   // 2^19 + c1
-    const float f2 = __uint_as_float((v & 0x00000F00u) | 0x47000000u);   // 2^15 + c2
-    const float f3 = __uint_as_float((v & 0x0000F000u) | 0x45000000u);   // 2^11 + c3
-    const float f4 = __uint_as_float((v & 0x000F0000u) | 0x43000000u);   // 2^7  + c4
-    const float f5 = __uint_as_float((u & 0x00000F00u) | 0x47000000u);   // 2^15 + c5
-    const float f6 = __uint_as_float((u & 0x0000F000u) | 0x45000000u);   // 2^11 + c6
-    const float f7 = __uint_as_float((u & 0x000F0000u) | 0x43000000u);   // 2^7  + c7
-    const float2 d01 = __fadd2_rn(make_float2(f0, f1), k.c01);
-    const float2 d23 = __fadd2_rn(make_float2(f2, f3), k.c23);
-    const float2 d45 = __fadd2_rn(make_float2(f4, f5), k.c45);
-    const float2 d67 = __fadd2_rn(make_float2(f6, f7), k.c67);
-    const float4 xa = xw[0];
-    const float4 xb = xw[1];
-    float2 acc = __fmul2_rn(make_float2(xa.x, xa.y), d01);
-    acc = __ffma2_rn(make_float2(xa.z, xa.w), d23, acc);
-    acc = __ffma2_rn(make_float2(xb.x, xb.y), d45, acc);
-    acc = __ffma2_rn(make_float2(xb.z, xb.w), d67, acc);
-    return acc;
-}
-
 // (a & m) | c as one LOP3; m and c are kept in registers (pinned) by the callers, since the
 // instruction takes a single immediate.
 __device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t m, uint32_t c)
@@ -152,6 +123,38 @@ __device__ __forceinline__ uint32_t pinned_u32(uint32_t v)
     uint32_t r;
     asm volatile("mov.b32 %0, %1;" : "=r"(r) : "r"(v));
     return r;
+}
+
+// Constants of word_dot_f32 held in registers: the offsets 2^(23-4p) + 8 to remove, the
+// nibble masks 0xF << 4i and the exponents 2^(23-4i) a nibble at bit 4i is OR-ed into.
+struct ExpandConsts {
+    float2 c01, c23, c45, c67;
+    uint32_t mask[5], magic[5];
+};
+
+// f32 x: eight codes of one word dotted with eight x values (exact code - 8).
+__device__ __forceinline__ float2 word_dot_f32(uint32_t v, const float4* xw, const ExpandConsts& k)
+{
+    const uint32_t u = v >> 12;
+    const float f0 = __uint_as_float(and_or(v, k.mask[0], k.magic[0]));   // 2^23 + c0
+    const float f1 = __uint_as_float(and_or(v, k.mask[1], k.magic[1]));   // 2^19 + c1
+    const float f2 = __uint_as_float(and_or(v, k.mask[2], k.magic[2]));   // 2^15 + c2
+    const float f3 = __uint_as_float(and_or(v, k.mask[3], k.magic[3]));   // 2^11 + c3
+    const float f4 = __uint_as_float(and_or(v, k.mask[4], k.magic[4]));   // 2^7  + c4
+    const float f5 = __uint_as_float(and_or(u, k.mask[2], k.magic[2]));   // 2^15 + c5
+    const float f6 = __uint_as_float(and_or(u, k.mask[3], k.magic[3]));   // 2^11 + c6
+    const float f7 = __uint_as_float(and_or(u, k.mask[4], k.magic[4]));   // 2^7  + c7
+    const float2 d01 = __fadd2_rn(make_float2(f0, f1), k.c01);
+    const float2 d23 = __fadd2_rn(make_float2(f2, f3), k.c23);
+    const float2 d45 = __fadd2_rn(make_float2(f4, f5), k.c45);
+    const float2 d67 = __fadd2_rn(make_float2(f6, f7), k.c67);
+    const float4 xa = xw[0];
+    const float4 xb = xw[1];
+    float2 acc = __fmul2_rn(make_float2(xa.x, xa.y), d01);
+    acc = __ffma2_rn(make_float2(xa.z, xa.w), d23, acc);
+    acc = __ffma2_rn(make_float2(xb.x, xb.y), d45, acc);
+    acc = __ffma2_rn(make_float2(xb.z, xb.w), d67, acc);
+    return acc;
 }
 
 // Nibble pair (j, j+4) of a word as the bf16 pair (128 + c_j, 128 + c_{j+4}); mask and
@@ -215,7 +218,7 @@ __device__ __forceinline__ double sum8_bf16(const uint4 raw)
 
 template <int MODE>
 struct ModeCfg {
-    static constexpr int MP = MODE == kMma16 ? 16 : MODE == kMma8 ? 8 : 1;   // x rows of the MMA tiles
+    static constexpr int MP = MODE == kMma16 ? 16 : (MODE == kMma8 || MODE == kMma1) ? 8 : 1;   // MMA x rows
     static constexpr int NT = MP >= 8 ? MP / 8 : 1;                          // n-tiles of 8 x rows
     static constexpr int kMinBlocks = 1;
 };
@@ -261,9 +264,17 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
     }
     __syncwarp();
     ExpandConsts kc = {};
-    if constexpr (MODE == kF32M1)
-        kc = {make_float2(pinned(-8388616.0f), pinned(-524296.0f)), make_float2(pinned(-32776.0f), pinned(-2056.0f)),
-              make_float2(pinned(-136.0f), pinned(-32776.0f)), make_float2(pinned(-2056.0f), pinned(-136.0f))};
+    if constexpr (MODE == kF32M1) {
+        kc.c01 = make_float2(pinned(-8388616.0f), pinned(-524296.0f));
+        kc.c23 = make_float2(pinned(-32776.0f), pinned(-2056.0f));
+        kc.c45 = make_float2(pinned(-136.0f), pinned(-32776.0f));
+        kc.c67 = make_float2(pinned(-2056.0f), pinned(-136.0f));
+#pragma unroll
+        for (int i = 0; i < 5; ++i) {
+            kc.mask[i] = pinned_u32(0xFu << (4 * i));
+            kc.magic[i] = pinned_u32((uint32_t)(150 - 4 * i) << 23);
+        }
+    }
 
     // Job j: unit (u0 + j % nbw) of the warp's (j / nbw)-th row block; a unit is up to
     // kBoxesPerStage consecutive code boxes plus one scale box spanning all of them.  Jobs
@@ -449,9 +460,11 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
 #pragma unroll
                                     for (int n = 0; n < NT; ++n) {
                                         acc[n][0] = fmaf(s0, d[c - c0][n][0], acc[n][0]);
-                                        acc[n][1] = fmaf(s0, d[c - c0][n][1], acc[n][1]);
                                         acc[n][2] = fmaf(s1, d[c - c0][n][2], acc[n][2]);
-                                        acc[n][3] = fmaf(s1, d[c - c0][n][3], acc[n][3]);
+                                        if constexpr (MODE != kMma1) {          // columns 2t + 1
+                                            acc[n][1] = fmaf(s0, d[c - c0][n][1], acc[n][1]);
+                                            acc[n][3] = fmaf(s1, d[c - c0][n][3], acc[n][3]);
+                                        }
                                     }
                                 }
                             }
@@ -531,13 +544,13 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
 
 size_t per_warp_bytes(int mode)
 {
-    const int mp = mode == kMma16 ? 16 : mode == kMma8 ? 8 : 1;
+    const int mp = mode == kMma16 ? 16 : (mode == kMma8 || mode == kMma1) ? 8 : 1;
     return (size_t)kStages * (kStageCodes + kStageScales + sizeof(uint64_t)) + (size_t)kRows * mp * sizeof(float);
 }
 
 size_t x_stage_bytes(int mode, int nb, int64_t M)
 {
-    const int mp = mode == kMma16 ? 16 : mode == kMma8 ? 8 : 1;
+    const int mp = mode == kMma16 ? 16 : (mode == kMma8 || mode == kMma1) ? 8 : 1;
     const size_t ngp = (size_t)nb * 8;
     return mode == kF32M1 ? ngp * 32 * sizeof(float) : (size_t)(M + 1) * (ngp + 1) * 64 + ngp * (mp / 8) * 64;
 }
@@ -550,7 +563,7 @@ size_t smem_bytes(int mode, int warps, int nb, int64_t M)
 int mode_for(int64_t M, q4_dtype xt)
 {
     if (M == 1 && xt == Q4_F32) return kF32M1;
-    return M <= 8 ? kMma8 : kMma16;
+    return M == 1 ? kMma1 : M <= 8 ? kMma8 : kMma16;
 }
 
 const void* kernel_for(int mode)
@@ -558,6 +571,7 @@ const void* kernel_for(int mode)
     switch (mode) {
     case kF32M1: return reinterpret_cast<const void*>(&gemv_tma_kernel<kF32M1>);
     case kMma8: return reinterpret_cast<const void*>(&gemv_tma_kernel<kMma8>);
+    case kMma1: return reinterpret_cast<const void*>(&gemv_tma_kernel<kMma1>);
     default: return reinterpret_cast<const void*>(&gemv_tma_kernel<kMma16>);
     }
 }
