@@ -176,7 +176,13 @@ class DecodeStep:
         x = synth_inputs.activations(1, 2560, "bf16", rank)
         self.x_np = x
         self.x = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(device)
-        self.y = [torch.empty((1, w.N), dtype=torch.float32, device=device) for (w, *_) in self.mats]
+        # the projections' outputs are views of one buffer, so a step's result leaves the
+        # device in a single copy
+        self.y_all = torch.empty((sum(w.N for (w, *_) in self.mats),), dtype=torch.float32, device=device)
+        self.y, off = [], 0
+        for (w, *_) in self.mats:
+            self.y.append(self.y_all[off:off + w.N].view(1, w.N))
+            off += w.N
         need = q4.gemv_multi_workspace_size(1, 2560, [w.N for w in MAIN])
         self.ws = torch.zeros(max(need, 16), dtype=torch.uint8, device=device)
         import ctypes
@@ -290,17 +296,15 @@ def measure_e2e(torch, q4, step, steps, device, dist=None, world=1):
     the three GEMVs, outputs -> pinned host, host waits for the result."""
     n = max(1, min(steps, 2000))
     x_host = torch.from_numpy(step.x_np.view(np.int16)).view(torch.bfloat16).pin_memory()
-    y_host = [torch.empty(y.shape, dtype=y.dtype).pin_memory() for y in step.y]
+    y_host = torch.empty(step.y_all.shape, dtype=step.y_all.dtype).pin_memory()
     x_dev = torch.empty_like(step.x)
     stream = torch.cuda.current_stream(device)
+    weights = [[(step.pk[j][c], step.sc[j][c]) for j in range(len(step.mats))] for c in range(step.copies)]
 
     def one(i):
-        c = i % step.copies
         x_dev.copy_(x_host, non_blocking=True)
-        q4.gemv_multi(x_dev, [(step.pk[j][c], step.sc[j][c]) for j in range(len(step.mats))], step.y,
-                      workspace=step.ws, weights_static=True)
-        for j in range(len(step.mats)):
-            y_host[j].copy_(step.y[j], non_blocking=True)
+        q4.gemv_multi(x_dev, weights[i % step.copies], step.y, workspace=step.ws, weights_static=True)
+        y_host.copy_(step.y_all, non_blocking=True)
         stream.synchronize()
 
     for i in range(3):
@@ -319,7 +323,7 @@ def measure_e2e(torch, q4, step, steps, device, dist=None, world=1):
         ms = float(t.item())
     return {"value": world * STEP_BYTES / (ms * 1e-3) / 1e9, "unit": UNIT,
             "h2d_bytes_per_step": x_host.numel() * 2,
-            "d2h_bytes_per_step": sum(y.numel() * 4 for y in y_host),
+            "d2h_bytes_per_step": y_host.numel() * 4,
             "steps": n, "ms_per_step": ms,
             "api": "bit_weight_only_quantize_b200.gemv_multi, pinned host x in, host y out, sync per step"}
 

@@ -8,6 +8,9 @@ QORA-LLM-0.8B model card, section "Weight Format").
 """
 from __future__ import annotations
 
+import contextlib
+import ctypes
+
 import torch
 
 from . import _lib
@@ -21,6 +24,13 @@ __all__ = [
 
 def _stream() -> int:
     return torch.cuda.current_stream().cuda_stream
+
+
+def _on(device: torch.device):
+    """Make ``device`` current for the call (a no-op context when it already is)."""
+    if device.index is None or device.index == torch.cuda.current_device():
+        return contextlib.nullcontext()
+    return torch.cuda.device(device)
 
 
 def _need(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int) -> None:
@@ -50,7 +60,7 @@ def quantize(W: torch.Tensor, flags: torch.Tensor | None = None):
     if flags is not None:
         _need(flags, "flags", torch.int32, 1)
         fptr = flags.data_ptr()
-    with torch.cuda.device(W.device):
+    with _on(W.device):
         st = _lib.load().q4_quantize(W.data_ptr(), N, K, packed.data_ptr(), scales.data_ptr(), fptr, _stream())
     _lib.check(st, "q4_quantize")
     return packed, scales
@@ -87,10 +97,11 @@ def gemv(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, out: torch
         if tuple(out.shape) != (M, N):
             raise ValueError("out has the wrong shape")
     lib = _lib.load()
-    with torch.cuda.device(x.device):
-        need = int(lib.q4_gemv_workspace_size(M, N, K))
-        if need and workspace is None:
-            workspace = torch.zeros(need, dtype=torch.uint8, device=x.device)
+    with _on(x.device):
+        if workspace is None:
+            need = int(lib.q4_gemv_workspace_size(M, N, K))
+            if need:
+                workspace = torch.zeros(need, dtype=torch.uint8, device=x.device)
         ws_ptr = workspace.data_ptr() if workspace is not None else None
         ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
         st = lib.q4_gemv(x.data_ptr(), xt, M, K, packed.data_ptr(), scales.data_ptr(), N,
@@ -100,7 +111,6 @@ def gemv(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, out: torch
 
 
 def gemv_multi_workspace_size(M: int, K: int, Ns) -> int:
-    import ctypes
     arr = (ctypes.c_int64 * len(Ns))(*Ns)
     return int(_lib.load().q4_gemv_multi_workspace_size(M, K, ctypes.cast(arr, ctypes.c_void_p), len(Ns)))
 
@@ -112,7 +122,6 @@ def gemv_multi(x: torch.Tensor, weights, outs=None, workspace: torch.Tensor | No
     ``weights_static=True`` declares that no kernel still running on the stream writes
     these weights, so they may be streamed before the preceding kernel finishes.
     """
-    import ctypes
     if x.dtype == torch.float32:
         xt = _lib.Q4_F32
     elif x.dtype == torch.bfloat16:
@@ -135,10 +144,11 @@ def gemv_multi(x: torch.Tensor, weights, outs=None, workspace: torch.Tensor | No
             raise ValueError("shape mismatch between x, packed, scales and out")
         arr[i] = _lib.Weight(packed.data_ptr(), scales.data_ptr(), N, y.data_ptr())
     lib = _lib.load()
-    with torch.cuda.device(x.device):
-        need = gemv_multi_workspace_size(M, K, [p.shape[0] for p, _ in weights])
-        if need and workspace is None:
-            workspace = torch.zeros(need, dtype=torch.uint8, device=x.device)
+    with _on(x.device):
+        if workspace is None:
+            need = gemv_multi_workspace_size(M, K, [p.shape[0] for p, _ in weights])
+            if need:
+                workspace = torch.zeros(need, dtype=torch.uint8, device=x.device)
         ws_ptr = workspace.data_ptr() if workspace is not None else None
         ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
         st = lib.q4_gemv_multi(x.data_ptr(), xt, M, K, ctypes.cast(arr, ctypes.c_void_p), len(weights),
@@ -162,7 +172,7 @@ def gemm(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, out: torch
         _need(out, "out", torch.bfloat16, 2)
         if tuple(out.shape) != (M, N):
             raise ValueError("out has the wrong shape")
-    with torch.cuda.device(x.device):
+    with _on(x.device):
         st = _lib.load().q4_gemm(x.data_ptr(), M, K, packed.data_ptr(), scales.data_ptr(), N, out.data_ptr(),
                                  _stream())
     _lib.check(st, "q4_gemm")

@@ -415,12 +415,7 @@ template <int MA, int BN>
 bool setup_kernel(size_t* smem)
 {
     *smem = GemmCfg<MA, BN>::kSmem;
-    if (cudaFuncSetAttribute(gemm_tc_kernel<MA, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)*smem) !=
-        cudaSuccess) {
-        cudaGetLastError();
-        return false;
-    }
-    return true;
+    return blocks_per_sm(reinterpret_cast<const void*>(&gemm_tc_kernel<MA, BN>), kThreads, *smem) >= 1;
 }
 
 }  // namespace

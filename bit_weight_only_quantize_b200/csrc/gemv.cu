@@ -310,13 +310,7 @@ bool plan_gemv_generic(int64_t M, int64_t N, int64_t K, q4_dtype xt, const Devic
     p->chunk = chunk;
     p->xcap = xcap;
     p->smem_bytes = mt * held * 128;
-    int per_sm = 2;
-    const void* fn = pick_ffma(mt, xt == Q4_BF16);
-    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, p->smem_bytes) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kThreads, p->smem_bytes) != cudaSuccess) {
-        cudaGetLastError();
-        return false;
-    }
+    const int per_sm = blocks_per_sm(pick_ffma(mt, xt == Q4_BF16), kThreads, (size_t)p->smem_bytes);
     if (per_sm < 1) return false;
     const long long resident = (long long)dev.sm_count * per_sm;
     long long gx = (resident + splits - 1) / splits;

@@ -648,16 +648,8 @@ bool plan_gemv_tma(int64_t M, const int64_t* Ns, int count, int64_t K, q4_dtype 
     const int warps = P * teams;
     const size_t smem = smem_bytes(mode, warps, nb, M);
     if (smem > budget) return false;
-    const void* fn = kernel_for(mode);
-    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) {
-        cudaGetLastError();
-        return false;
-    }
-    int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, warps * 32, smem) != cudaSuccess || per_sm < 1) {
-        cudaGetLastError();
-        return false;
-    }
+    const int per_sm = blocks_per_sm(kernel_for(mode), warps * 32, smem);
+    if (per_sm < 1) return false;
     const long long blocks_needed = ((long long)row_blocks + teams - 1) / teams;
     long long gx = (long long)dev.sm_count * per_sm / splits;
     if (gx > blocks_needed) gx = blocks_needed;

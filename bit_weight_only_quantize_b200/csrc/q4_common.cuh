@@ -57,6 +57,13 @@ q4_status launch_gemv_tma(const void* x, q4_dtype xt, int64_t M, int64_t K, cons
 q4_status launch_gemm(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed, const uint16_t* scales,
                       int64_t N, uint16_t* y, cudaStream_t stream, const DeviceInfo& dev);
 
+// Resident blocks per SM of kernel `fn` launched with `threads` threads and `smem` bytes
+// of dynamic shared memory, after opting the kernel into that much shared memory on the
+// current device.  Both the opt-in and the occupancy answer are cached per (device,
+// kernel, threads, smem), so a call that repeats a shape makes no CUDA API calls.
+// Returns 0 when the configuration cannot run.
+int blocks_per_sm(const void* fn, int threads, size_t smem);
+
 // Programmatic dependent launch is on unless the environment sets Q4_NO_PDL=1
 // (read once per process; useful under tools that do not follow such launches).
 bool pdl_enabled();

@@ -41,7 +41,63 @@ void lookup_err(int dev)
     g_err_addr[dev] = static_cast<unsigned*>(p);
 }
 
+// Occupancy answers already obtained (a handful of kernels x shapes per process).
+struct OccEntry {
+    int device;
+    const void* fn;
+    int threads;
+    size_t smem;
+    int blocks;
+};
+constexpr int kOccSlots = 256;
+OccEntry g_occ[kOccSlots];
+int g_occ_used = 0;
+std::mutex g_occ_mutex;
+
+// Largest dynamic shared memory each kernel has been opted into, per device.
+struct OptIn {
+    int device;
+    const void* fn;
+    size_t smem;
+};
+OptIn g_optin[kOccSlots];
+int g_optin_used = 0;
+
 }  // namespace
+
+int blocks_per_sm(const void* fn, int threads, size_t smem)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    std::lock_guard<std::mutex> lock(g_occ_mutex);
+    for (int i = 0; i < g_occ_used; ++i)
+        if (g_occ[i].device == dev && g_occ[i].fn == fn && g_occ[i].threads == threads && g_occ[i].smem == smem)
+            return g_occ[i].blocks;
+    int o = 0;
+    while (o < g_optin_used && !(g_optin[o].device == dev && g_optin[o].fn == fn)) ++o;
+    if (o == g_optin_used || g_optin[o].smem < smem) {
+        if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) {
+            cudaGetLastError();
+            return 0;
+        }
+        if (o == g_optin_used) {
+            if (g_optin_used == kOccSlots) return 0;
+            g_optin[g_optin_used++] = {dev, fn, smem};
+        } else {
+            g_optin[o].smem = smem;
+        }
+    }
+    int blocks = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, fn, threads, smem) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    if (g_occ_used < kOccSlots) g_occ[g_occ_used++] = {dev, fn, threads, smem, blocks};
+    return blocks;
+}
 
 bool encode_tma_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner, uint64_t outer,
                    uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle)
