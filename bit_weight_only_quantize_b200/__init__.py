@@ -33,13 +33,18 @@ def _on(device: torch.device):
     return torch.cuda.device(device)
 
 
-def _need(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int) -> None:
+def _need(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int, device: torch.device | None = None) -> None:
+    """Type, dtype, device, rank and contiguity of one argument (``device``: the device
+    every tensor of the call must share; None: any CUDA device)."""
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
-    if not t.is_cuda:
-        raise ValueError(f"{name} must be a CUDA tensor")
-    if t.dtype != dtype:
+    if t.dtype is not dtype:
         raise TypeError(f"{name} must have dtype {dtype}, got {t.dtype}")
+    if device is None:
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+    elif t.device != device:
+        raise ValueError(f"{name} must be on {device}, got {t.device}")
     if t.dim() != ndim:
         raise ValueError(f"{name} must have {ndim} dimensions")
     if not t.is_contiguous():
@@ -58,7 +63,7 @@ def quantize(W: torch.Tensor, flags: torch.Tensor | None = None):
     scales = torch.empty((N, max(K // 32, 0)), dtype=torch.int16, device=W.device)
     fptr = None
     if flags is not None:
-        _need(flags, "flags", torch.int32, 1)
+        _need(flags, "flags", torch.int32, 1, W.device)
         fptr = flags.data_ptr()
     with _on(W.device):
         st = _lib.load().q4_quantize(W.data_ptr(), N, K, packed.data_ptr(), scales.data_ptr(), fptr, _stream())
@@ -84,8 +89,8 @@ def gemv(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, out: torch
     else:
         raise TypeError("x must be float32 or bfloat16")
     _need(x, "x", x.dtype, 2)
-    _need(packed, "packed", torch.uint8, 2)
-    _need(scales, "scales", torch.int16, 2)
+    _need(packed, "packed", torch.uint8, 2, x.device)
+    _need(scales, "scales", torch.int16, 2, x.device)
     M, K = x.shape
     N = packed.shape[0]
     if packed.shape[1] * 2 != K or tuple(scales.shape) != (N, K // 32):
@@ -93,9 +98,11 @@ def gemv(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, out: torch
     if out is None:
         out = torch.empty((M, N), dtype=torch.float32, device=x.device)
     else:
-        _need(out, "out", torch.float32, 2)
+        _need(out, "out", torch.float32, 2, x.device)
         if tuple(out.shape) != (M, N):
             raise ValueError("out has the wrong shape")
+    if workspace is not None:
+        _need(workspace, "workspace", torch.uint8, 1, x.device)
     lib = _lib.load()
     with _on(x.device):
         if workspace is None:
@@ -136,13 +143,15 @@ def gemv_multi(x: torch.Tensor, weights, outs=None, workspace: torch.Tensor | No
         outs = [torch.empty((M, p.shape[0]), dtype=torch.float32, device=x.device) for p, _ in weights]
     arr = (_lib.Weight * len(weights))()
     for i, ((packed, scales), y) in enumerate(zip(weights, outs)):
-        _need(packed, "packed", torch.uint8, 2)
-        _need(scales, "scales", torch.int16, 2)
-        _need(y, "out", torch.float32, 2)
+        _need(packed, "packed", torch.uint8, 2, x.device)
+        _need(scales, "scales", torch.int16, 2, x.device)
+        _need(y, "out", torch.float32, 2, x.device)
         N = packed.shape[0]
         if packed.shape[1] * 2 != K or tuple(scales.shape) != (N, K // 32) or tuple(y.shape) != (M, N):
             raise ValueError("shape mismatch between x, packed, scales and out")
         arr[i] = _lib.Weight(packed.data_ptr(), scales.data_ptr(), N, y.data_ptr())
+    if workspace is not None:
+        _need(workspace, "workspace", torch.uint8, 1, x.device)
     lib = _lib.load()
     with _on(x.device):
         if workspace is None:
@@ -160,8 +169,8 @@ def gemv_multi(x: torch.Tensor, weights, outs=None, workspace: torch.Tensor | No
 def gemm(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
     """y[M,N] (bf16) = x[M,K] (bf16) . dequant(W)^T on the tensor cores (prefill)."""
     _need(x, "x", torch.bfloat16, 2)
-    _need(packed, "packed", torch.uint8, 2)
-    _need(scales, "scales", torch.int16, 2)
+    _need(packed, "packed", torch.uint8, 2, x.device)
+    _need(scales, "scales", torch.int16, 2, x.device)
     M, K = x.shape
     N = packed.shape[0]
     if packed.shape[1] * 2 != K or tuple(scales.shape) != (N, K // 32):
@@ -169,7 +178,7 @@ def gemm(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, out: torch
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
     else:
-        _need(out, "out", torch.bfloat16, 2)
+        _need(out, "out", torch.bfloat16, 2, x.device)
         if tuple(out.shape) != (M, N):
             raise ValueError("out has the wrong shape")
     with _on(x.device):
