@@ -299,11 +299,14 @@ def measure_e2e(torch, q4, step, steps, device, dist=None, world=1):
     y_host = torch.empty(step.y_all.shape, dtype=step.y_all.dtype).pin_memory()
     x_dev = torch.empty_like(step.x)
     stream = torch.cuda.current_stream(device)
-    weights = [[(step.pk[j][c], step.sc[j][c]) for j in range(len(step.mats))] for c in range(step.copies)]
+    # one prepared call per weight copy: the weights are checked once, each step checks x
+    calls = [q4.GemvMulti([(step.pk[j][c], step.sc[j][c]) for j in range(len(step.mats))], 1, step.x.shape[1],
+                          step.x.dtype, outs=step.y, workspace=step.ws, weights_static=True)
+             for c in range(step.copies)]
 
     def one(i):
         x_dev.copy_(x_host, non_blocking=True)
-        q4.gemv_multi(x_dev, weights[i % step.copies], step.y, workspace=step.ws, weights_static=True)
+        calls[i % step.copies](x_dev)
         y_host.copy_(step.y_all, non_blocking=True)
         stream.synchronize()
 
@@ -325,7 +328,8 @@ def measure_e2e(torch, q4, step, steps, device, dist=None, world=1):
             "h2d_bytes_per_step": x_host.numel() * 2,
             "d2h_bytes_per_step": y_host.numel() * 4,
             "steps": n, "ms_per_step": ms,
-            "api": "bit_weight_only_quantize_b200.gemv_multi, pinned host x in, host y out, sync per step"}
+            "api": "bit_weight_only_quantize_b200.GemvMulti (prepared gemv_multi), pinned host x in, host y out, "
+                   "sync per step"}
 
 
 def time_launches(torch, fn, n, device, stream):

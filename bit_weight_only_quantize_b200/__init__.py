@@ -17,8 +17,8 @@ from . import _lib
 from ._lib import Q4Error, FLAG_NONFINITE, FLAG_SCALE_OVERFLOW, GEMV_MAX_M  # noqa: F401
 
 __all__ = [
-    "quantize", "gemv", "gemv_multi", "gemm", "gemv_workspace_size", "gemv_multi_workspace_size", "Q4Error", "FLAG_NONFINITE", "FLAG_SCALE_OVERFLOW",
-    "GEMV_MAX_M",
+    "quantize", "gemv", "gemv_multi", "GemvMulti", "gemm", "gemv_workspace_size", "gemv_multi_workspace_size",
+    "Q4Error", "FLAG_NONFINITE", "FLAG_SCALE_OVERFLOW", "GEMV_MAX_M",
 ]
 
 
@@ -164,6 +164,68 @@ def gemv_multi(x: torch.Tensor, weights, outs=None, workspace: torch.Tensor | No
                                _lib.WEIGHTS_STATIC if weights_static else 0, ws_ptr, ws_bytes, _stream())
     _lib.check(st, "q4_gemv_multi")
     return outs
+
+
+class GemvMulti:
+    """A prepared ``gemv_multi`` for a decode loop: the weights, outputs and workspace are
+    checked once, and each call checks only x before the launch.
+
+    The tensors are held by reference; their storage must not be replaced (``set_``,
+    ``resize_``) while the object is in use.
+    """
+
+    def __init__(self, weights, M: int, K: int, x_dtype: torch.dtype, outs=None,
+                 workspace: torch.Tensor | None = None, weights_static: bool = False):
+        if x_dtype is torch.float32:
+            self._xt = _lib.Q4_F32
+        elif x_dtype is torch.bfloat16:
+            self._xt = _lib.Q4_BF16
+        else:
+            raise TypeError("x must be float32 or bfloat16")
+        if not 1 <= len(weights) <= _lib.MULTI_MAX:
+            raise ValueError(f"between 1 and {_lib.MULTI_MAX} weight matrices")
+        dev = weights[0][0].device
+        if outs is None:
+            outs = [torch.empty((M, p.shape[0]), dtype=torch.float32, device=dev) for p, _ in weights]
+        self._arr = (_lib.Weight * len(weights))()
+        for i, ((packed, scales), y) in enumerate(zip(weights, outs)):
+            _need(packed, "packed", torch.uint8, 2, dev)
+            _need(scales, "scales", torch.int16, 2, dev)
+            _need(y, "out", torch.float32, 2, dev)
+            N = packed.shape[0]
+            if packed.shape[1] * 2 != K or tuple(scales.shape) != (N, K // 32) or tuple(y.shape) != (M, N):
+                raise ValueError("shape mismatch between x, packed, scales and out")
+            self._arr[i] = _lib.Weight(packed.data_ptr(), scales.data_ptr(), N, y.data_ptr())
+        with _on(dev):
+            if workspace is None:
+                need = gemv_multi_workspace_size(M, K, [p.shape[0] for p, _ in weights])
+                if need:
+                    workspace = torch.zeros(need, dtype=torch.uint8, device=dev)
+        if workspace is not None:
+            _need(workspace, "workspace", torch.uint8, 1, dev)
+        self._keep = (weights, workspace)
+        self._vp = ctypes.cast(self._arr, ctypes.c_void_p)
+        self._ws = workspace.data_ptr() if workspace is not None else None
+        self._wsb = workspace.numel() if workspace is not None else 0
+        self._count = len(weights)
+        self._flags = _lib.WEIGHTS_STATIC if weights_static else 0
+        self._shape = (M, K)
+        self._dtype = x_dtype
+        self.device = dev
+        self.outs = outs
+        self._lib = _lib.load()
+
+    def __call__(self, x: torch.Tensor):
+        """Launch on the current stream; returns the output list given at construction."""
+        if not isinstance(x, torch.Tensor) or x.dtype is not self._dtype:
+            raise TypeError(f"x must be a {self._dtype} tensor")
+        if x.device != self.device or x.shape != self._shape or not x.is_contiguous():
+            raise ValueError(f"x must be a contiguous {self._shape} tensor on {self.device}")
+        with _on(self.device):
+            st = self._lib.q4_gemv_multi(x.data_ptr(), self._xt, self._shape[0], self._shape[1], self._vp,
+                                         self._count, self._flags, self._ws, self._wsb, _stream())
+        _lib.check(st, "q4_gemv_multi")
+        return self.outs
 
 
 def gemm(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:

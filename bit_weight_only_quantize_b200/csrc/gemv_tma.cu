@@ -424,7 +424,7 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
                                 smem_addr(cb) + ((li & 1) * 8 + lr) * 128 + (((li >> 1) ^ lr) << 4);
                             // All MMAs of a batch of groups are issued before any result is
                             // read, so the tensor-core latency overlaps across groups.
-                            constexpr int GB = NT == 1 ? 8 : 4;            // groups per batch
+                            constexpr int GB = 2;            // groups per batch
 #pragma unroll
                             for (int c0 = 0; c0 < 8; c0 += GB) {
                                 float d[GB][NT][4];

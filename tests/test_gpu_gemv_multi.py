@@ -90,3 +90,25 @@ def test_graph_chain_with_static_weights():
     for i, x in enumerate(xs):
         for (packed, scales), y in zip(mats, outs[i]):
             assert rel_inf(y.cpu().numpy(), oracle.matmul(x, packed, scales, threads=8)) <= 1e-5
+
+
+@pytest.mark.parametrize("M,x_dtype", [(1, "bf16"), (1, "f32"), (3, "bf16")])
+def test_prepared_call_matches_gemv_multi(M, x_dtype):
+    """GemvMulti checks the weights once and launches the same kernel: identical bits."""
+    import bit_weight_only_quantize_b200 as q4
+    Ns, K = [2048, 4096, 1024], 2560
+    dm = _dev(_prep(Ns, K, seed=21))
+    plan = q4.GemvMulti(dm, M, K, torch.float32 if x_dtype == "f32" else torch.bfloat16, weights_static=True)
+    for seed in (1, 2):
+        x = synth_inputs.activations(M, K, x_dtype, seed=seed)
+        xd = to_dev_x(x)
+        ys = [y.clone() for y in plan(xd)]
+        ref = q4.gemv_multi(xd, dm)
+        torch.cuda.synchronize()
+        for y, r, (p, s) in zip(ys, ref, _prep(Ns, K, seed=21)):
+            assert torch.equal(y, r)
+            assert rel_inf(y.cpu().numpy(), oracle.matmul(x, p, s, threads=8)) <= (2e-3 if x_dtype == "f32" else 1e-2)
+    with pytest.raises(ValueError):
+        plan(to_dev_x(synth_inputs.activations(M + 1, K, x_dtype, seed=3)))      # wrong shape
+    with pytest.raises(TypeError):
+        plan(torch.zeros((M, K), dtype=torch.float16, device="cuda"))            # wrong dtype
