@@ -65,6 +65,8 @@ def _load():
         lib.oracle_q4_matmul_rows.restype = i32
         lib.oracle_q4_matmul.argtypes = [vp, i32, i64, i64, vp, vp, i64, vp, i32]
         lib.oracle_q4_matmul.restype = i32
+        lib.oracle_q4_gate_up_rows.argtypes = [vp, i32, i64, i64, vp, vp, vp, vp, vp, i64, vp, i32]
+        lib.oracle_q4_gate_up_rows.restype = i32
         lib.oracle_max_threads.argtypes = []
         lib.oracle_max_threads.restype = i32
         _lib = lib
@@ -149,6 +151,39 @@ def matmul(x: np.ndarray, packed: np.ndarray, scales: np.ndarray, rows=None, thr
                                        _ptr(r), r.size, _ptr(y), threads)
     if rc != 0:
         raise MemoryError("oracle matmul: allocation failed")
+    return y
+
+
+def gate_up(x: np.ndarray, gate, up, rows=None, threads: int = 1) -> np.ndarray:
+    """y = silu(x . dequant(Wg)^T) * (x . dequant(Wu)^T) in binary64, silu(g) = g/(1+e^-g).
+
+    The fused gate+up of the QORA-LLM-0.8B model card (section "AVX-512 SIMD
+    Acceleration"); the activation is read as SiLU (see ``q4_oracle.c``).
+    gate, up: (packed, scales) pairs with equal shapes.  x and rows as for ``matmul``.
+    """
+    if x.dtype == np.uint16:
+        is_bf16 = 1
+    elif x.dtype == np.float32:
+        is_bf16 = 0
+    else:
+        raise TypeError("x must be float32 or uint16 (bfloat16 bits)")
+    x = np.ascontiguousarray(x)
+    if x.ndim == 1:
+        x = x[None, :]
+    gp, gs = (np.ascontiguousarray(gate[0], dtype=np.uint8), np.ascontiguousarray(gate[1], dtype=np.uint16))
+    upk, us = (np.ascontiguousarray(up[0], dtype=np.uint8), np.ascontiguousarray(up[1], dtype=np.uint16))
+    M, K = x.shape
+    N = gp.shape[0]
+    if gp.shape != upk.shape or gs.shape != us.shape or gp.shape[1] * 2 != K or gs.shape != (N, K // 32):
+        raise ValueError("shape mismatch between x, gate and up")
+    r = np.arange(N, dtype=np.int64) if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    if r.size and (r.min() < 0 or r.max() >= N):
+        raise IndexError("row index out of range")
+    y = np.empty((M, r.size), dtype=np.float64)
+    rc = _load().oracle_q4_gate_up_rows(_ptr(x), is_bf16, M, K, _ptr(gp), _ptr(gs), _ptr(upk), _ptr(us), _ptr(r),
+                                        r.size, _ptr(y), threads)
+    if rc != 0:
+        raise MemoryError("oracle gate_up: allocation failed")
     return y
 
 

@@ -250,6 +250,32 @@ int oracle_q4_matmul(const void* x, int x_is_bf16, int64_t M, int64_t K,
     return oracle_q4_matmul_rows(x, x_is_bf16, M, K, packed, scales, NULL, N, y, nthreads);
 }
 
+/* Fused gate+up of the MLP (QORA-LLM-0.8B model card, section "AVX-512 SIMD
+ * Acceleration": "Fused gate+up", the gate and up projections decoded in one pass).
+ * The activation is not named there; the model card's only activation is SiLU, so
+ * the gated product is taken as SwiGLU's:
+ *     y[m, j] = silu(g[m, j]) * u[m, j],   silu(g) = g / (1 + exp(-g)),
+ * with g = x . dequant(Wg)^T and u = x . dequant(Wu)^T from oracle_q4_matmul_rows,
+ * everything in binary64.  rows, nrows, y and nthreads as for oracle_q4_matmul_rows.
+ * Returns -1 on allocation failure, else 0. */
+int oracle_q4_gate_up_rows(const void* x, int x_is_bf16, int64_t M, int64_t K,
+                           const uint8_t* gate_packed, const uint16_t* gate_scales,
+                           const uint8_t* up_packed, const uint16_t* up_scales,
+                           const int64_t* rows, int64_t nrows, double* y, int nthreads)
+{
+    const size_t count = (size_t)(M * nrows > 0 ? M * nrows : 1);
+    double* g = (double*)malloc(count * sizeof(double));
+    double* u = (double*)malloc(count * sizeof(double));
+    int rc = (g && u) ? 0 : -1;
+    if (rc == 0) rc = oracle_q4_matmul_rows(x, x_is_bf16, M, K, gate_packed, gate_scales, rows, nrows, g, nthreads);
+    if (rc == 0) rc = oracle_q4_matmul_rows(x, x_is_bf16, M, K, up_packed, up_scales, rows, nrows, u, nthreads);
+    if (rc == 0)
+        for (int64_t i = 0; i < M * nrows; ++i) y[i] = g[i] / (1.0 + exp(-g[i])) * u[i];
+    free(g);
+    free(u);
+    return rc;
+}
+
 int oracle_max_threads(void)
 {
 #ifdef _OPENMP
