@@ -419,6 +419,29 @@ def measure_rows(torch, q4, lib, device, peaks, l2):
         out[f"gemv_m{sw.M}"] = {"workload": f"M={sw.M} K=2560 N=4096 bf16 x", "ms": ms, "GB/s": b / ms / 1e6,
                                 "frac_hbm": b / ms / 1e6 / hbm, "bytes": b, "launches": copies * 4}
         del pks, scs
+    # Fused MLP gate+up decode (M=1, K=2560, N=4096 per matrix, bf16 x): two weight
+    # matrices, one launch, y = silu(gate) * up; rotating copies for a cold L2.
+    gu = synth_inputs.DECODE_PROJ[1]
+    _, gpk, gsc = make_quantized(torch, q4, gu, 0, device)
+    _, upk, usc = make_quantized(torch, q4, gu, 1, device)
+    setb = 2 * (gpk.numel() + gsc.numel() * 2)
+    copies = max(2, -(-3 * l2 // setb) + 1)
+    mats = [(gpk, gsc, upk, usc)] + [(gpk.clone(), gsc.clone(), upk.clone(), usc.clone()) for _ in range(copies - 1)]
+    xg = torch.from_numpy(synth_inputs.activations(1, gu.K, "bf16", 0).view(np.int16)).view(torch.bfloat16).to(device)
+    yg = torch.empty((1, gu.N), dtype=torch.float32, device=device)
+
+    def gate_up(i):
+        m = mats[i % copies]
+        st = lib.q4_gemv_gate_up(xg.data_ptr(), 1, 1, gu.K, m[0].data_ptr(), m[1].data_ptr(), m[2].data_ptr(),
+                                 m[3].data_ptr(), gu.N, yg.data_ptr(), 1, stream.cuda_stream)
+        assert st == 0
+    log("rows: gate+up")
+    ms = time_launches(torch, gate_up, copies * 4, device, stream)
+    b = 2 * (gu.N * gu.K // 2 + gu.N * (gu.K // 32) * 2) + gu.K * 2 + gu.N * 4
+    out["gate_up_gemv"] = {"workload": "fused gate+up M=1 K=2560 N=4096 x2, bf16 x, y = silu(g)*u", "ms": ms,
+                           "GB/s": b / ms / 1e6, "frac_hbm": b / ms / 1e6 / hbm, "bytes": b,
+                           "launches": copies * 4}
+    del mats
     # Prefill q4_gemm (bf16 x, bf16 y, f32 accumulate); inputs rotated to exceed 3x L2.
     for gw in synth_inputs.PREFILL:
         _, packed, scales = make_quantized(torch, q4, gw, 0, device)

@@ -17,7 +17,7 @@ from . import _lib
 from ._lib import Q4Error, FLAG_NONFINITE, FLAG_SCALE_OVERFLOW, GEMV_MAX_M  # noqa: F401
 
 __all__ = [
-    "quantize", "gemv", "gemv_multi", "GemvMulti", "gemm", "gemv_workspace_size", "gemv_multi_workspace_size",
+    "quantize", "gemv", "gemv_multi", "GemvMulti", "gemv_gate_up", "gemm", "gemv_workspace_size", "gemv_multi_workspace_size",
     "Q4Error", "FLAG_NONFINITE", "FLAG_SCALE_OVERFLOW", "GEMV_MAX_M",
 ]
 
@@ -164,6 +164,41 @@ def gemv_multi(x: torch.Tensor, weights, outs=None, workspace: torch.Tensor | No
                                _lib.WEIGHTS_STATIC if weights_static else 0, ws_ptr, ws_bytes, _stream())
     _lib.check(st, "q4_gemv_multi")
     return outs
+
+
+def gemv_gate_up(x: torch.Tensor, gate, up, out: torch.Tensor | None = None, weights_static: bool = False):
+    """y[M,N] (f32) = silu(x . dequant(Wg)^T) * (x . dequant(Wu)^T) in one launch.
+
+    gate, up: (packed, scales) of equal shapes.  K must be a multiple of 256; x is f32
+    (M == 1) or bf16 (M <= 16).  SiLU(g) = g / (1 + exp(-g)).
+    """
+    if x.dtype is torch.float32:
+        xt = _lib.Q4_F32
+    elif x.dtype is torch.bfloat16:
+        xt = _lib.Q4_BF16
+    else:
+        raise TypeError("x must be float32 or bfloat16")
+    _need(x, "x", x.dtype, 2)
+    (gp, gs), (upk, us) = gate, up
+    for t, name, dt in ((gp, "gate packed", torch.uint8), (gs, "gate scales", torch.int16),
+                        (upk, "up packed", torch.uint8), (us, "up scales", torch.int16)):
+        _need(t, name, dt, 2, x.device)
+    M, K = x.shape
+    N = gp.shape[0]
+    if gp.shape[1] * 2 != K or tuple(gs.shape) != (N, K // 32) or gp.shape != upk.shape or gs.shape != us.shape:
+        raise ValueError("shape mismatch between x, gate and up")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float32, device=x.device)
+    else:
+        _need(out, "out", torch.float32, 2, x.device)
+        if tuple(out.shape) != (M, N):
+            raise ValueError("out has the wrong shape")
+    with _on(x.device):
+        st = _lib.load().q4_gemv_gate_up(x.data_ptr(), xt, M, K, gp.data_ptr(), gs.data_ptr(), upk.data_ptr(),
+                                         us.data_ptr(), N, out.data_ptr(),
+                                         _lib.WEIGHTS_STATIC if weights_static else 0, _stream())
+    _lib.check(st, "q4_gemv_gate_up")
+    return out
 
 
 class GemvMulti:

@@ -203,6 +203,34 @@ q4_status q4_gemv_multi(const void* x, q4_dtype x_dtype, int64_t M, int64_t K, c
     return gemv_common(x, x_dtype, M, K, mats, count, flags, workspace, workspace_bytes, stream);
 }
 
+q4_status q4_gemv_gate_up(const void* x, q4_dtype x_dtype, int64_t M, int64_t K, const uint8_t* gate_packed,
+                          const uint16_t* gate_scales, const uint8_t* up_packed, const uint16_t* up_scales,
+                          int64_t N, float* y, uint32_t flags, void* stream)
+{
+    if (x_dtype != Q4_F32 && x_dtype != Q4_BF16) return Q4_ERR_DTYPE;
+    if (M < 0 || M > Q4_GEMV_MAX_M) return Q4_ERR_SHAPE;
+    q4_status st = check_nk(N, K);
+    if (st != Q4_OK) return st;
+    if (flags & ~Q4_WEIGHTS_STATIC) return Q4_ERR_INVALID_ARG;
+    if (M == 0 || N == 0) return Q4_OK;
+    if (!x || !gate_packed || !gate_scales || !up_packed || !up_scales || !y) return Q4_ERR_INVALID_ARG;
+    if (misaligned(x, 16) || misaligned(gate_packed, 16) || misaligned(up_packed, 16) ||
+        misaligned(gate_scales, 16) || misaligned(up_scales, 16) || misaligned(y, 4))
+        return Q4_ERR_ALIGN;
+    if (K % 256 != 0 || (M > 1 && x_dtype != Q4_BF16)) return Q4_ERR_SHAPE;
+    q4::DeviceInfo dev;
+    if ((st = q4::current_device(&dev)) != Q4_OK) return st;
+    const q4_weight mats[2] = {{gate_packed, gate_scales, N, y}, {up_packed, up_scales, N, y}};
+    const int64_t Ns[2] = {N, N};
+    q4::GemvPlan plan;
+    if (!q4::plan_gemv_tma(M, Ns, 2, K, x_dtype, dev, &plan, true)) {
+        cudaGetLastError();
+        return Q4_ERR_SHAPE;                      // x of this K does not fit beside the rings
+    }
+    return q4::launch_gemv_tma(x, x_dtype, M, K, mats, 2, (flags & Q4_WEIGHTS_STATIC) ? 1 : 0, nullptr, plan,
+                               static_cast<cudaStream_t>(stream), true);
+}
+
 q4_status q4_gemm(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed, const uint16_t* scales,
                   int64_t N, uint16_t* y, void* stream)
 {

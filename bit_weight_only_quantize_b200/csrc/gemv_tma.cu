@@ -82,6 +82,7 @@ struct TmaGemvArgs {
     int P;                            // warps per team
     int teams;                        // teams per block
     int prefetch;                     // weights may be read before the dependency wait
+    int fuse;                         // gate+up: matrices 0 and 1 (equal N), y = silu(y0) * y1 into y[0]
 };
 
 __device__ __forceinline__ void team_sync(int team, int P)
@@ -251,9 +252,17 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
     const int ngp = nb * 8;                                               // groups, padded
     const int nu = (nb + kBoxesPerStage - 1) / kBoxesPerStage;            // stage units of this split
     const int u0 = wt * nu / P, nbw = (wt + 1) * nu / P - u0;             // this warp's units
+    // A team walks row blocks first_rb, first_rb + rb_stride, ...  With fuse it walks the
+    // row-block pairs of the gate and up matrices instead, visiting gate block p and then
+    // up block p (= p + the gate's block count) of each pair in turn.
     const int first_rb = blockIdx.x * a.teams + team;
     const int rb_stride = gridDim.x * a.teams;
-    const int nrb = (active && first_rb < a.row_blocks) ? (a.row_blocks - first_rb + rb_stride - 1) / rb_stride : 0;
+    const int walk = a.fuse ? a.rb_begin[1] : a.row_blocks;
+    const int nwalk = (active && first_rb < walk) ? (walk - first_rb + rb_stride - 1) / rb_stride : 0;
+    const int nrb = a.fuse ? 2 * nwalk : nwalk;                           // row-block visits
+    auto rb_of = [&](int i) {
+        return a.fuse ? first_rb + (i >> 1) * rb_stride + (i & 1) * a.rb_begin[1] : first_rb + i * rb_stride;
+    };
     const int njobs = nrb * nbw;
     uint64_t* my_bars = bars + warp * kStages;
     const size_t K = (size_t)a.G * 32;
@@ -280,10 +289,11 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
     // kBoxesPerStage consecutive code boxes plus one scale box spanning all of them.  Jobs
     // are issued in order, so a cursor (unit, row block and its matrix) replaces the
     // division and the matrix lookup.
-    int iss_u = 0, iss_rb = first_rb, iss_mi = 0, iss_lrow = 0;
+    int iss_u = 0, iss_vis = 0, iss_mi = 0, iss_lrow = 0;
     auto locate = [&]() {
-        iss_mi = matrix_of(a, iss_rb);
-        iss_lrow = (iss_rb - a.rb_begin[iss_mi]) * kRows;
+        const int rb = rb_of(iss_vis);
+        iss_mi = matrix_of(a, rb);
+        iss_lrow = (rb - a.rb_begin[iss_mi]) * kRows;
     };
     if (lane == 0 && njobs > 0) locate();
     auto issue = [&](int j) {
@@ -298,7 +308,7 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
         tma_load_2d(scl + (warp * kStages + s) * kStageScales, &maps.scales[iss_mi], g0 + 8 * bf, iss_lrow, bar);
         if (++iss_u == nbw) {
             iss_u = 0;
-            iss_rb += rb_stride;
+            ++iss_vis;
             if (j + 1 < njobs) locate();
         }
     };
@@ -376,8 +386,9 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
 
     bool ok = true;
     int consumed = 0;
+    float gsave[kRows * Q4_GEMV_MAX_M / 32];       // fuse: the gate totals of the current pair
     for (int rbi = 0; rbi < nrb; ++rbi) {
-        const int rb = first_rb + rbi * rb_stride;
+        const int rb = rb_of(rbi);
         float yacc = 0.f;     // kF32M1: row (lane & 15), half (lane >> 4)
         float acc[NT][4];     // MMA modes: rows g, g+8; x rows n*8 + 2t, +1
 #pragma unroll
@@ -503,7 +514,24 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
             const int nrow = a.N[mi];
             const int lrow0 = (rb - a.rb_begin[mi]) * kRows;
             const size_t vrows = (size_t)a.row_blocks * kRows;            // padded rows over all matrices
-            for (int e = lane; e < kRows * a.M; e += 32) {           // x row major: coalesced y
+            if (a.fuse) {                       // splits == 1: gate totals wait in registers
+#pragma unroll
+                for (int it = 0; it < kRows * Q4_GEMV_MAX_M / 32; ++it) {
+                    const int e = lane + 32 * it;
+                    if (e < kRows * a.M) {
+                        const int m = e / kRows, rr = e - m * kRows;
+                        float total = 0.f;
+                        for (int w = 0; w < P; ++w) total += red[(team * P + w) * kRows * MP + rr * MP + m];
+                        if (mi == 0) {
+                            gsave[it] = total;
+                        } else if (lrow0 + rr < nrow) {
+                            const float g = gsave[it];
+                            a.y[0][(size_t)m * nrow + lrow0 + rr] = g / (1.0f + expf(-g)) * total;
+                        }
+                    }
+                }
+            }
+            for (int e = lane; e < (a.fuse ? 0 : kRows * a.M); e += 32) {   // x row major: coalesced y
                 const int m = e / kRows, rr = e - m * kRows;
                 float total = 0.f;
                 for (int w = 0; w < P; ++w) total += red[(team * P + w) * kRows * MP + rr * MP + m];
@@ -586,14 +614,17 @@ bool tma_gemv_eligible(int64_t M, int64_t K, q4_dtype xt, const void* packed, co
 }
 
 bool plan_gemv_tma(int64_t M, const int64_t* Ns, int count, int64_t K, q4_dtype xt, const DeviceInfo& dev,
-                   GemvPlan* p)
+                   GemvPlan* p, bool fuse)
 {
+    if (fuse && (count != 2 || Ns[0] != Ns[1])) return false;
     const int mode = mode_for(M, xt);
     const int G = (int)(K / 32);
     long long rbl = 0;
     for (int i = 0; i < count; ++i) rbl += (Ns[i] + kRows - 1) / kRows;
     if (rbl < 1 || rbl > INT32_MAX / kRows) return false;
     const int row_blocks = (int)rbl;
+    const int walk = fuse ? row_blocks / 2 : row_blocks;      // row blocks (gate+up: pairs) teams walk
+    const int visits = fuse ? 2 : 1;                          // row blocks per walked item
     const int boxes = (G + 7) / 8;
     const int units = (boxes + kBoxesPerStage - 1) / kBoxesPerStage;
     const size_t pw = per_warp_bytes(mode);
@@ -615,7 +646,8 @@ bool plan_gemv_tma(int64_t M, const int64_t* Ns, int count, int64_t K, q4_dtype 
     // per block are capped so that small problems spread over all SMs.
     int splits = 0, P = 0, teams = 0;
     double best = 0.0;
-    const int max_splits = row_blocks <= kCounterSlots ? units : splits_min;
+    if (fuse && splits_min > 1) return false;                 // the fused epilogue needs whole sums
+    const int max_splits = (row_blocks <= kCounterSlots && !fuse) ? units : splits_min;
     for (int sp = splits_min; sp <= max_splits; ++sp) {
         const int nbs = split_boxes(sp);
         if ((boxes + nbs - 1) / nbs != sp) continue;                  // same cut as fewer splits
@@ -628,10 +660,10 @@ bool plan_gemv_tma(int64_t M, const int64_t* Ns, int count, int64_t K, q4_dtype 
         for (int pp = 1; pp <= nus && pp <= wbs; ++pp) {
             const int pwu = (nus + pp - 1) / pp;                          // units per warp per row block
             long long tm = wbs / pp;
-            const long long spread = ((long long)row_blocks + sms - 1) / sms;
+            const long long spread = ((long long)walk + sms - 1) / sms;
             if (tm > spread) tm = spread;
-            const long long gxs = std::min(((long long)row_blocks + tm - 1) / tm, sms);
-            const long long rounds = ((long long)row_blocks + gxs * tm - 1) / (gxs * tm);
+            const long long gxs = std::min(((long long)walk + tm - 1) / tm, sms);
+            const long long rounds = visits * (((long long)walk + gxs * tm - 1) / (gxs * tm));
             const double share = std::max((double)(tm * pp), kMinWarpShare) / 16.0;
             const double cost = (double)rounds * (pwu + kEpilogueCost) * share + (sp > 1 ? kSplitCost : 0.0);
             if (splits == 0 || cost < best - 1e-9) {
@@ -650,7 +682,7 @@ bool plan_gemv_tma(int64_t M, const int64_t* Ns, int count, int64_t K, q4_dtype 
     if (smem > budget) return false;
     const int per_sm = blocks_per_sm(kernel_for(mode), warps * 32, smem);
     if (per_sm < 1) return false;
-    const long long blocks_needed = ((long long)row_blocks + teams - 1) / teams;
+    const long long blocks_needed = ((long long)walk + teams - 1) / teams;
     long long gx = (long long)dev.sm_count * per_sm / splits;
     if (gx > blocks_needed) gx = blocks_needed;
     if (gx < 1) gx = 1;
@@ -668,7 +700,7 @@ bool plan_gemv_tma(int64_t M, const int64_t* Ns, int count, int64_t K, q4_dtype 
 }
 
 q4_status launch_gemv_tma(const void* x, q4_dtype xt, int64_t M, int64_t K, const q4_weight* mats, int count,
-                          int prefetch, void* workspace, const GemvPlan& plan, cudaStream_t stream)
+                          int prefetch, void* workspace, const GemvPlan& plan, cudaStream_t stream, bool fuse)
 {
     TmaMaps maps;
     TmaGemvArgs a;
@@ -712,6 +744,7 @@ q4_status launch_gemv_tma(const void* x, q4_dtype xt, int64_t M, int64_t K, cons
     a.P = plan.chunk;
     a.teams = plan.xcap;
     a.prefetch = prefetch;
+    a.fuse = fuse ? 1 : 0;
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)plan.grid_x, (unsigned)plan.splits);

@@ -49,10 +49,13 @@ q4_status launch_gemv(const void* x, q4_dtype xt, int64_t M, int64_t K, const q4
                       uint32_t flags, void* workspace, const GemvPlan& plan, cudaStream_t stream);
 
 bool tma_gemv_eligible(int64_t M, int64_t K, q4_dtype xt, const void* packed, const void* scales);
+// fuse: mats are gate and up of equal N; the kernel writes silu(x.gate^T) * (x.up^T) into
+// mats[0].y and never splits K.
 bool plan_gemv_tma(int64_t M, const int64_t* Ns, int count, int64_t K, q4_dtype xt, const DeviceInfo& dev,
-                   GemvPlan* plan);
+                   GemvPlan* plan, bool fuse = false);
 q4_status launch_gemv_tma(const void* x, q4_dtype xt, int64_t M, int64_t K, const q4_weight* mats, int count,
-                          int prefetch, void* workspace, const GemvPlan& plan, cudaStream_t stream);
+                          int prefetch, void* workspace, const GemvPlan& plan, cudaStream_t stream,
+                          bool fuse = false);
 
 q4_status launch_gemm(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed, const uint16_t* scales,
                       int64_t N, uint16_t* y, cudaStream_t stream, const DeviceInfo& dev);

@@ -169,6 +169,27 @@ Q4_API q4_status q4_gemv_multi(const void* x, q4_dtype x_dtype, int64_t M, int64
                                void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * q4_gemv_gate_up: the fused gate+up of an MLP decode step (QORA-LLM-0.8B model card,
+ * section "AVX-512 SIMD Acceleration": "Fused gate+up", both projections decoded in one
+ * pass over x).  The page names no activation; the model card's one activation is SiLU,
+ * so the gated product is SwiGLU's:
+ *     y[m, n] = silu(g[m, n]) * u[m, n],   silu(g) = g / (1 + exp(-g)),
+ *     g = x . dequant(Wg)^T,  u = x . dequant(Wu)^T   (f32 accumulation, as q4_gemv),
+ * g and u never leave the chip: one launch, one f32 output.
+ *   x        device, f32 (M == 1) or bfloat16 (M = 1..16) [M,K], 16-byte aligned.
+ *   K        a multiple of 256 (the kernel streams 256-wide boxes; other K: Q4_ERR_SHAPE).
+ *   gate_*, up_*  Q4 encodings of Wg[N,K] and Wu[N,K]: packed 16-byte aligned, scales
+ *            16-byte aligned (Q4_ERR_ALIGN otherwise).
+ *   y        device, f32 [M,N], 4-byte aligned (output, overwritten).
+ *   flags    0 or Q4_WEIGHTS_STATIC, as for q4_gemv_multi.
+ * No workspace (K is never split).  M == 0 or N == 0 is a no-op.
+ */
+Q4_API q4_status q4_gemv_gate_up(const void* x, q4_dtype x_dtype, int64_t M, int64_t K,
+                                 const uint8_t* gate_packed, const uint16_t* gate_scales,
+                                 const uint8_t* up_packed, const uint16_t* up_scales, int64_t N,
+                                 float* y, uint32_t flags, void* stream);
+
+/*
  * q4_gemm: y = bf16( x . dequant(W)^T ) for prefill (any M >= 0; tuned for M >= 512).
  * The pages batch the prefill projections across tokens into GEMMs (QORA-4B thread,
  * section "GPU 预填充优化"; QORA-LLM-0.8B model card, section "Performance").

@@ -123,3 +123,20 @@ def test_binding_raises_without_gpu_tensors():
     import bit_weight_only_quantize_b200 as q4
     with pytest.raises(ValueError):
         q4.quantize(torch.zeros(4, 64))
+
+
+def test_gate_up_validation(lib):
+    S = None
+    f = lib.q4_gemv_gate_up
+    assert f(A16, 7, 1, 256, A16, A16, A16, A16, 8, A16, 0, S) == 4            # dtype
+    assert f(A16, 1, 17, 256, A16, A16, A16, A16, 8, A16, 0, S) == 2           # M > 16
+    assert f(A16, 1, 1, 40, A16, A16, A16, A16, 8, A16, 0, S) == 2             # K % 32
+    assert f(A16, 1, 1, 256, A16, A16, A16, A16, 8, A16, 4, S) == 1            # unknown flag
+    assert f(A16, 1, 1, 256, None, A16, A16, A16, 8, A16, 0, S) == 1
+    assert f(A16, 1, 1, 256, A16, A16, A16, A16, 8, None, 0, S) == 1
+    assert f(A16, 1, 1, 256, A16, A16, A8, A16, 8, A16, 0, S) == 3             # up packed alignment
+    assert f(A16, 1, 1, 256, A16, A8, A16, A16, 8, A16, 0, S) == 3             # gate scales: 16 bytes
+    assert f(A16, 1, 1, 96, A16, A16, A16, A16, 8, A16, 0, S) == 2             # K % 256
+    assert f(A16, 0, 2, 256, A16, A16, A16, A16, 8, A16, 0, S) == 2            # f32 x with M > 1
+    assert f(None, 1, 0, 256, None, None, None, None, 8, None, 0, S) == 0      # M == 0: no-op
+    assert f(None, 1, 3, 256, None, None, None, None, 0, None, 0, S) == 0      # N == 0: no-op
