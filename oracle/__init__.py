@@ -187,5 +187,19 @@ def gate_up(x: np.ndarray, gate, up, rows=None, threads: int = 1) -> np.ndarray:
     return y
 
 
+def argmax(x: np.ndarray, packed: np.ndarray, scales: np.ndarray, threads: int = 1):
+    """Greedy decoding over an LM head: for each x row, the index and value of the
+    largest logit of y = x . dequant(W)^T (binary64), the lowest index on ties.
+
+    The QORA-4B thread (section "量化与内存管理") lists the LM head among the parallel
+    workloads; greedy decoding (temperature 0) is the deterministic mode of the
+    QORA-LLM-0.8B model card (section "CLI Flags", ``--greedy``).  The index is numpy's
+    argmax (first occurrence of the maximum) over the binary64 logits.
+    """
+    y = matmul(x, packed, scales, threads=threads)
+    idx = np.argmax(y, axis=1).astype(np.int64)
+    return idx, y[np.arange(y.shape[0]), idx]
+
+
 def max_threads() -> int:
     return int(_load().oracle_max_threads())
