@@ -378,6 +378,23 @@ def measure_rows(torch, q4, lib, device, peaks, l2):
     out["lm_head_gemv"] = {"workload": "M=1 K=2560 N=248320 bf16 x", "ms": ms, "GB/s": b / ms / 1e6,
                            "frac_hbm": b / ms / 1e6 / hbm, "bytes": b, "launches": 20}
 
+    # Greedy LM-head step: the same GEMV with the argmax fused, logits kept on chip.
+    am_ws = torch.zeros(int(lib.q4_gemv_argmax_workspace_size()), dtype=torch.uint8, device=device)
+    am_idx = torch.empty((1,), dtype=torch.int64, device=device)
+    am_val = torch.empty((1,), dtype=torch.float32, device=device)
+
+    def lm_argmax(i):
+        st = lib.q4_gemv_argmax(x.data_ptr(), 1, 1, w.K, packed.data_ptr(), scales.data_ptr(), w.N, None,
+                                am_idx.data_ptr(), am_val.data_ptr(), 1, am_ws.data_ptr(), am_ws.numel(),
+                                stream.cuda_stream)
+        assert st == 0
+    log("rows: lm head argmax")
+    ms = time_launches(torch, lm_argmax, 20, device, stream)
+    b = w.N * w.K // 2 + w.N * (w.K // 32) * 2 + w.K * 2 + 12
+    out["lm_head_argmax"] = {"workload": "greedy step: M=1 K=2560 N=248320 bf16 x, argmax fused, no logits out",
+                             "ms": ms, "GB/s": b / ms / 1e6, "frac_hbm": b / ms / 1e6 / hbm, "bytes": b,
+                             "launches": 20}
+
     # Quantise the LM-head weights: reads 4 B and writes 0.5625 B per weight.
     Wd = torch.from_numpy(W).to(device)
     del W

@@ -17,7 +17,7 @@ from . import _lib
 from ._lib import Q4Error, FLAG_NONFINITE, FLAG_SCALE_OVERFLOW, GEMV_MAX_M  # noqa: F401
 
 __all__ = [
-    "quantize", "gemv", "gemv_multi", "GemvMulti", "gemv_gate_up", "gemm", "gemv_workspace_size", "gemv_multi_workspace_size",
+    "quantize", "gemv", "gemv_multi", "GemvMulti", "gemv_gate_up", "gemv_argmax", "gemm", "gemv_workspace_size", "gemv_multi_workspace_size",
     "Q4Error", "FLAG_NONFINITE", "FLAG_SCALE_OVERFLOW", "GEMV_MAX_M",
 ]
 
@@ -199,6 +199,45 @@ def gemv_gate_up(x: torch.Tensor, gate, up, out: torch.Tensor | None = None, wei
                                          _lib.WEIGHTS_STATIC if weights_static else 0, _stream())
     _lib.check(st, "q4_gemv_gate_up")
     return out
+
+
+def gemv_argmax(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, logits: bool = False,
+                workspace: torch.Tensor | None = None, weights_static: bool = False):
+    """Greedy LM-head step in one launch: (index int64 [M], value f32 [M], y or None) with
+    index[m] the row of the largest logit of x[m] . dequant(W)^T (lowest row on ties).
+
+    ``logits=True`` also returns the f32 logits [M,N].  ``workspace`` (uint8, zero before
+    its first use, left zero by every call) is allocated here when not given; calls in
+    flight at the same time on different streams need their own.
+    """
+    if x.dtype is torch.float32:
+        xt = _lib.Q4_F32
+    elif x.dtype is torch.bfloat16:
+        xt = _lib.Q4_BF16
+    else:
+        raise TypeError("x must be float32 or bfloat16")
+    _need(x, "x", x.dtype, 2)
+    _need(packed, "packed", torch.uint8, 2, x.device)
+    _need(scales, "scales", torch.int16, 2, x.device)
+    M, K = x.shape
+    N = packed.shape[0]
+    if packed.shape[1] * 2 != K or tuple(scales.shape) != (N, K // 32):
+        raise ValueError("shape mismatch between x, packed and scales")
+    lib = _lib.load()
+    index = torch.empty((M,), dtype=torch.int64, device=x.device)
+    value = torch.empty((M,), dtype=torch.float32, device=x.device)
+    y = torch.empty((M, N), dtype=torch.float32, device=x.device) if logits else None
+    if workspace is None:
+        workspace = torch.zeros(int(lib.q4_gemv_argmax_workspace_size()), dtype=torch.uint8, device=x.device)
+    else:
+        _need(workspace, "workspace", torch.uint8, 1, x.device)
+    with _on(x.device):
+        st = lib.q4_gemv_argmax(x.data_ptr(), xt, M, K, packed.data_ptr(), scales.data_ptr(), N,
+                                y.data_ptr() if y is not None else None, index.data_ptr(), value.data_ptr(),
+                                _lib.WEIGHTS_STATIC if weights_static else 0, workspace.data_ptr(),
+                                workspace.numel(), _stream())
+    _lib.check(st, "q4_gemv_argmax")
+    return index, value, y
 
 
 class GemvMulti:

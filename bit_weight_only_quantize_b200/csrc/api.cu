@@ -231,6 +231,41 @@ q4_status q4_gemv_gate_up(const void* x, q4_dtype x_dtype, int64_t M, int64_t K,
                                static_cast<cudaStream_t>(stream), true);
 }
 
+size_t q4_gemv_argmax_workspace_size(void) { return 256; }   // Q4_GEMV_MAX_M keys, then the counter
+
+q4_status q4_gemv_argmax(const void* x, q4_dtype x_dtype, int64_t M, int64_t K, const uint8_t* packed,
+                         const uint16_t* scales, int64_t N, float* y, int64_t* index, float* value,
+                         uint32_t flags, void* workspace, size_t workspace_bytes, void* stream)
+{
+    if (x_dtype != Q4_F32 && x_dtype != Q4_BF16) return Q4_ERR_DTYPE;
+    if (M < 0 || M > Q4_GEMV_MAX_M) return Q4_ERR_SHAPE;
+    q4_status st = check_nk(N, K);
+    if (st != Q4_OK) return st;
+    if (flags & ~Q4_WEIGHTS_STATIC) return Q4_ERR_INVALID_ARG;
+    if (M == 0 || N == 0) return Q4_OK;
+    if (!x || !packed || !scales || !index) return Q4_ERR_INVALID_ARG;
+    if (!workspace || workspace_bytes < q4_gemv_argmax_workspace_size()) return Q4_ERR_WORKSPACE;
+    if (misaligned(x, 16) || misaligned(packed, 16) || misaligned(scales, 16) || (y && misaligned(y, 4)) ||
+        misaligned(index, 8) || (value && misaligned(value, 4)) || misaligned(workspace, 16))
+        return Q4_ERR_ALIGN;
+    if (K % 256 != 0 || (M > 1 && x_dtype != Q4_BF16)) return Q4_ERR_SHAPE;
+    q4::DeviceInfo dev;
+    if ((st = q4::current_device(&dev)) != Q4_OK) return st;
+    const q4_weight w = {packed, scales, N, y};
+    q4::GemvPlan plan;
+    if (!q4::plan_gemv_tma(M, &N, 1, K, x_dtype, dev, &plan, false, true)) {
+        cudaGetLastError();
+        return Q4_ERR_SHAPE;
+    }
+    q4::ArgmaxOut am;
+    am.key = static_cast<unsigned long long*>(workspace);
+    am.done = reinterpret_cast<unsigned*>(static_cast<char*>(workspace) + Q4_GEMV_MAX_M * 8);
+    am.index = reinterpret_cast<long long*>(index);
+    am.value = value;
+    return q4::launch_gemv_tma(x, x_dtype, M, K, &w, 1, (flags & Q4_WEIGHTS_STATIC) ? 1 : 0, nullptr, plan,
+                               static_cast<cudaStream_t>(stream), false, &am);
+}
+
 q4_status q4_gemm(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed, const uint16_t* scales,
                   int64_t N, uint16_t* y, void* stream)
 {

@@ -83,7 +83,30 @@ struct TmaGemvArgs {
     int teams;                        // teams per block
     int prefetch;                     // weights may be read before the dependency wait
     int fuse;                         // gate+up: matrices 0 and 1 (equal N), y = silu(y0) * y1 into y[0]
+    // greedy argmax over the rows of matrix 0 (splits == 1): per x row, the largest logit
+    // and its row; keys and the block counter live in a workspace that is zero at rest
+    int argmax;
+    unsigned long long* am_key;       // [M] (value order, then lowest row)
+    unsigned* am_done;                // blocks finished
+    long long* am_index;              // [M] output
+    float* am_value;                  // [M] output, may be null
 };
+
+// Orderable 64-bit key of (logit v, row r): larger v wins, then the lower row; every NaN
+// counts as the largest value (a NaN logit is reported, as numpy's argmax does).
+__device__ __forceinline__ unsigned long long argmax_key(float v, int r)
+{
+    uint32_t b = __float_as_uint(v);
+    if ((b & 0x7FFFFFFFu) > 0x7F800000u) b = 0x7FC00000u;
+    const uint32_t ord = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+    return ((unsigned long long)ord << 32) | (0xFFFFFFFFu - (uint32_t)r);
+}
+
+__device__ __forceinline__ float argmax_value(unsigned long long key)
+{
+    const uint32_t ord = (uint32_t)(key >> 32);
+    return __uint_as_float((ord & 0x80000000u) ? (ord & 0x7FFFFFFFu) : ~ord);
+}
 
 __device__ __forceinline__ void team_sync(int team, int P)
 {
@@ -531,13 +554,25 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
                     }
                 }
             }
-            for (int e = lane; e < (a.fuse ? 0 : kRows * a.M); e += 32) {   // x row major: coalesced y
+            for (int e0 = 0; e0 < (a.fuse ? 0 : kRows * a.M); e0 += 32) {   // x row major: coalesced y
+                const int e = e0 + lane;
                 const int m = e / kRows, rr = e - m * kRows;
+                const bool live = e < kRows * a.M && lrow0 + rr < nrow;
                 float total = 0.f;
-                for (int w = 0; w < P; ++w) total += red[(team * P + w) * kRows * MP + rr * MP + m];
-                if (lrow0 + rr < nrow) {
-                    if (a.splits == 1) a.y[mi][(size_t)m * nrow + lrow0 + rr] = total;
-                    else a.partial[((size_t)split * a.M + m) * vrows + (size_t)rb * kRows + rr] = total;
+                if (e < kRows * a.M)
+                    for (int w = 0; w < P; ++w) total += red[(team * P + w) * kRows * MP + rr * MP + m];
+                if (live) {
+                    if (a.splits > 1) a.partial[((size_t)split * a.M + m) * vrows + (size_t)rb * kRows + rr] = total;
+                    else if (a.y[mi]) a.y[mi][(size_t)m * nrow + lrow0 + rr] = total;
+                }
+                if (a.argmax) {                // the 16 lanes of one x row agree on its best row
+                    unsigned long long key = live ? argmax_key(total, lrow0 + rr) : 0ull;
+#pragma unroll
+                    for (int o = 1; o < kRows; o <<= 1) {
+                        const unsigned long long k2 = __shfl_xor_sync(0xffffffffu, key, o);
+                        key = k2 > key ? k2 : key;
+                    }
+                    if (rr == 0 && m < a.M && key) atomicMax(&a.am_key[m], key);
                 }
             }
             if (a.splits > 1) {
@@ -567,6 +602,24 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
         if (lane == 0) atomicOr(a.err, kErrWaitTimeout);
         for (int j = consumed; j < issued; ++j)    // copies still in flight into this warp's ring
             if (!mbar_wait_bounded(&my_bars[j % kStages], (uint32_t)(j / kStages) & 1u, kWaitLimit)) break;
+    }
+
+    if (a.argmax) {                                // the last block to finish reports and resets
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            __threadfence();
+            s_last[0] = atomicAdd(a.am_done, 1u) == gridDim.x - 1;
+        }
+        __syncthreads();
+        if (s_last[0]) {
+            __threadfence();
+            if ((int)threadIdx.x < a.M) {
+                const unsigned long long key = atomicExch(&a.am_key[threadIdx.x], 0ull);
+                a.am_index[threadIdx.x] = key ? (long long)(0xFFFFFFFFu - (uint32_t)key) : -1;
+                if (a.am_value) a.am_value[threadIdx.x] = key ? argmax_value(key) : __int_as_float(0x7FC00000);
+            }
+            if (threadIdx.x == 0) *a.am_done = 0u;
+        }
     }
 }
 
@@ -614,7 +667,7 @@ bool tma_gemv_eligible(int64_t M, int64_t K, q4_dtype xt, const void* packed, co
 }
 
 bool plan_gemv_tma(int64_t M, const int64_t* Ns, int count, int64_t K, q4_dtype xt, const DeviceInfo& dev,
-                   GemvPlan* p, bool fuse)
+                   GemvPlan* p, bool fuse, bool whole_k)
 {
     if (fuse && (count != 2 || Ns[0] != Ns[1])) return false;
     const int mode = mode_for(M, xt);
@@ -646,8 +699,8 @@ bool plan_gemv_tma(int64_t M, const int64_t* Ns, int count, int64_t K, q4_dtype 
     // per block are capped so that small problems spread over all SMs.
     int splits = 0, P = 0, teams = 0;
     double best = 0.0;
-    if (fuse && splits_min > 1) return false;                 // the fused epilogue needs whole sums
-    const int max_splits = (row_blocks <= kCounterSlots && !fuse) ? units : splits_min;
+    if ((fuse || whole_k) && splits_min > 1) return false;   // fused epilogues need whole sums
+    const int max_splits = (row_blocks <= kCounterSlots && !fuse && !whole_k) ? units : splits_min;
     for (int sp = splits_min; sp <= max_splits; ++sp) {
         const int nbs = split_boxes(sp);
         if ((boxes + nbs - 1) / nbs != sp) continue;                  // same cut as fewer splits
@@ -700,7 +753,8 @@ bool plan_gemv_tma(int64_t M, const int64_t* Ns, int count, int64_t K, q4_dtype 
 }
 
 q4_status launch_gemv_tma(const void* x, q4_dtype xt, int64_t M, int64_t K, const q4_weight* mats, int count,
-                          int prefetch, void* workspace, const GemvPlan& plan, cudaStream_t stream, bool fuse)
+                          int prefetch, void* workspace, const GemvPlan& plan, cudaStream_t stream, bool fuse,
+                          const ArgmaxOut* am)
 {
     TmaMaps maps;
     TmaGemvArgs a;
@@ -745,6 +799,11 @@ q4_status launch_gemv_tma(const void* x, q4_dtype xt, int64_t M, int64_t K, cons
     a.teams = plan.xcap;
     a.prefetch = prefetch;
     a.fuse = fuse ? 1 : 0;
+    a.argmax = am ? 1 : 0;
+    a.am_key = am ? am->key : nullptr;
+    a.am_done = am ? am->done : nullptr;
+    a.am_index = am ? am->index : nullptr;
+    a.am_value = am ? am->value : nullptr;
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)plan.grid_x, (unsigned)plan.splits);

@@ -49,13 +49,22 @@ q4_status launch_gemv(const void* x, q4_dtype xt, int64_t M, int64_t K, const q4
                       uint32_t flags, void* workspace, const GemvPlan& plan, cudaStream_t stream);
 
 bool tma_gemv_eligible(int64_t M, int64_t K, q4_dtype xt, const void* packed, const void* scales);
+// Greedy argmax outputs of a TMA GEMV launch over one matrix (see q4_gemv_argmax).
+struct ArgmaxOut {
+    unsigned long long* key;   // [M] workspace, zero at rest
+    unsigned* done;            // workspace, zero at rest
+    long long* index;          // [M]
+    float* value;              // [M] or null
+};
+
 // fuse: mats are gate and up of equal N; the kernel writes silu(x.gate^T) * (x.up^T) into
-// mats[0].y and never splits K.
+// mats[0].y.  whole_k: K is never split (fused epilogues that need whole sums).
 bool plan_gemv_tma(int64_t M, const int64_t* Ns, int count, int64_t K, q4_dtype xt, const DeviceInfo& dev,
-                   GemvPlan* plan, bool fuse = false);
+                   GemvPlan* plan, bool fuse = false, bool whole_k = false);
+// am: non-null for a greedy argmax launch (count == 1; mats[0].y may be null).
 q4_status launch_gemv_tma(const void* x, q4_dtype xt, int64_t M, int64_t K, const q4_weight* mats, int count,
                           int prefetch, void* workspace, const GemvPlan& plan, cudaStream_t stream,
-                          bool fuse = false);
+                          bool fuse = false, const ArgmaxOut* am = nullptr);
 
 q4_status launch_gemm(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed, const uint16_t* scales,
                       int64_t N, uint16_t* y, cudaStream_t stream, const DeviceInfo& dev);

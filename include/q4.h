@@ -190,6 +190,29 @@ Q4_API q4_status q4_gemv_gate_up(const void* x, q4_dtype x_dtype, int64_t M, int
                                  float* y, uint32_t flags, void* stream);
 
 /*
+ * q4_gemv_argmax: greedy decoding over an LM head in one launch: for each x row m,
+ *     index[m] = the row n with the largest y[m, n] = x . dequant(W)^T (f32, as q4_gemv),
+ *     the lowest such n on ties; a NaN logit counts as the largest value;
+ *     value[m] = y[m, index[m]].
+ * The logits need not leave the chip (QORA-4B thread, section "量化与内存管理": the LM head
+ * is one of the parallel workloads; QORA-LLM-0.8B model card, section "CLI Flags":
+ * --greedy, temperature 0).  Shapes, dtypes and alignment as for q4_gemv_gate_up
+ * (K % 256 == 0; M == 1 with f32 x or M = 1..16 with bf16 x; scales 16-byte aligned).
+ *   y        device f32 [M,N] or NULL: when given, the logits are written too.
+ *   index    device int64 [M], 8-byte aligned (output).
+ *   value    device f32 [M] or NULL (output).
+ *   workspace  device, q4_gemv_argmax_workspace_size() bytes, 16-byte aligned, all zero
+ *            before the first call; every call leaves it zero again, so one workspace
+ *            serves every call on a stream (calls in flight at the same time on
+ *            different streams need their own).
+ * K is never split.  M == 0 or N == 0 is a no-op.
+ */
+Q4_API size_t q4_gemv_argmax_workspace_size(void);
+Q4_API q4_status q4_gemv_argmax(const void* x, q4_dtype x_dtype, int64_t M, int64_t K, const uint8_t* packed,
+                                const uint16_t* scales, int64_t N, float* y, int64_t* index, float* value,
+                                uint32_t flags, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * q4_gemm: y = bf16( x . dequant(W)^T ) for prefill (any M >= 0; tuned for M >= 512).
  * The pages batch the prefill projections across tokens into GEMMs (QORA-4B thread,
  * section "GPU 预填充优化"; QORA-LLM-0.8B model card, section "Performance").

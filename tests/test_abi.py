@@ -140,3 +140,19 @@ def test_gate_up_validation(lib):
     assert f(A16, 0, 2, 256, A16, A16, A16, A16, 8, A16, 0, S) == 2            # f32 x with M > 1
     assert f(None, 1, 0, 256, None, None, None, None, 8, None, 0, S) == 0      # M == 0: no-op
     assert f(None, 1, 3, 256, None, None, None, None, 0, None, 0, S) == 0      # N == 0: no-op
+
+
+def test_argmax_validation(lib):
+    S = None
+    f = lib.q4_gemv_argmax
+    assert lib.q4_gemv_argmax_workspace_size() >= 16 * 8 + 4
+    W = 256
+    assert f(A16, 7, 1, 256, A16, A16, 8, None, A16, None, 0, A16, W, S) == 4      # dtype
+    assert f(A16, 1, 17, 256, A16, A16, 8, None, A16, None, 0, A16, W, S) == 2     # M > 16
+    assert f(A16, 1, 1, 256, A16, A16, 8, None, None, None, 0, A16, W, S) == 1     # index required
+    assert f(A16, 1, 1, 256, A16, A16, 8, None, A16, None, 0, None, 0, S) == 5     # workspace required
+    assert f(A16, 1, 1, 256, A16, A16, 8, None, A16, None, 0, A16, 64, S) == 5     # workspace too small
+    assert f(A16, 1, 1, 256, A16, A16, 8, None, A16 + 4, None, 0, A16, W, S) == 3  # index alignment
+    assert f(A16, 1, 1, 256, A16, A8, 8, None, A16, None, 0, A16, W, S) == 3       # scales: 16 bytes
+    assert f(A16, 1, 1, 96, A16, A16, 8, None, A16, None, 0, A16, W, S) == 2       # K % 256
+    assert f(None, 1, 0, 256, None, None, 8, None, None, None, 0, None, 0, S) == 0  # M == 0: no-op
