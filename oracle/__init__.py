@@ -67,6 +67,8 @@ def _load():
         lib.oracle_q4_matmul.restype = i32
         lib.oracle_q4_gate_up_rows.argtypes = [vp, i32, i64, i64, vp, vp, vp, vp, vp, i64, vp, i32]
         lib.oracle_q4_gate_up_rows.restype = i32
+        lib.oracle_f16_matmul.argtypes = [vp, i32, i64, i64, vp, i64, vp, i32]
+        lib.oracle_f16_matmul.restype = i32
         lib.oracle_max_threads.argtypes = []
         lib.oracle_max_threads.restype = i32
         _lib = lib
@@ -199,6 +201,29 @@ def argmax(x: np.ndarray, packed: np.ndarray, scales: np.ndarray, threads: int =
     y = matmul(x, packed, scales, threads=threads)
     idx = np.argmax(y, axis=1).astype(np.int64)
     return idx, y[np.arange(y.shape[0]), idx]
+
+
+def f16_matmul(x: np.ndarray, w16: np.ndarray, threads: int = 1) -> np.ndarray:
+    """y = x . W^T in binary64 for binary16 weights W (the F16 GEMV of the QORA-LLM-0.8B
+    model card, section "AVX-512 SIMD Acceleration").  w16: uint16 binary16 bits [N, K];
+    x as for ``matmul``."""
+    if x.dtype == np.uint16:
+        is_bf16 = 1
+    elif x.dtype == np.float32:
+        is_bf16 = 0
+    else:
+        raise TypeError("x must be float32 or uint16 (bfloat16 bits)")
+    x = np.ascontiguousarray(x)
+    if x.ndim == 1:
+        x = x[None, :]
+    w16 = np.ascontiguousarray(w16, dtype=np.uint16)
+    M, K = x.shape
+    N = w16.shape[0]
+    if w16.ndim != 2 or w16.shape[1] != K:
+        raise ValueError("shape mismatch between x and w16")
+    y = np.empty((M, N), dtype=np.float64)
+    _load().oracle_f16_matmul(_ptr(x), is_bf16, M, K, _ptr(w16), N, _ptr(y), threads)
+    return y
 
 
 def max_threads() -> int:

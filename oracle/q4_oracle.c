@@ -276,6 +276,32 @@ int oracle_q4_gate_up_rows(const void* x, int x_is_bf16, int64_t M, int64_t K,
     return rc;
 }
 
+/* F16-weight GEMV, the pages' second weight format (QORA-LLM-0.8B model card, section
+ * "AVX-512 SIMD Acceleration": "F16 GEMV", binary16 weights widened to f32 and
+ * multiply-added; section "File Structure": Q4/F16 GEMV kernels):
+ *     y[m, n] = sum_k x[m, k] * w[n, k],   w binary16 bits [N, K] row-major,
+ * every term and the running sum in binary64, k ascending (binary16 widens exactly).
+ * x, M, K, y and nthreads as for oracle_q4_matmul. */
+int oracle_f16_matmul(const void* x, int x_is_bf16, int64_t M, int64_t K, const uint16_t* w, int64_t N,
+                      double* y, int nthreads)
+{
+#ifdef _OPENMP
+    if (nthreads < 1) nthreads = 1;
+    #pragma omp parallel for schedule(dynamic, 16) num_threads(nthreads)
+#else
+    (void)nthreads;
+#endif
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t m = 0; m < M; ++m) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k)
+                acc += x_value(x, x_is_bf16, m * K + k) * (double)oracle_f16_to_f32(w[n * K + k]);
+            y[m * N + n] = acc;
+        }
+    }
+    return 0;
+}
+
 int oracle_max_threads(void)
 {
 #ifdef _OPENMP
