@@ -459,6 +459,27 @@ def measure_rows(torch, q4, lib, device, peaks, l2):
                            "GB/s": b / ms / 1e6, "frac_hbm": b / ms / 1e6 / hbm, "bytes": b,
                            "launches": copies * 4}
     del mats
+    # F16-weight GEMV (2 bytes per weight), bf16 x: the decode projection shape with
+    # rotating copies, and the LM-head shape (1.27 GB, already far above L2).
+    for name, N, K in (("f16_gemv_2560x4096", 4096, 2560), ("f16_gemv_lm_head", 248320, 2560)):
+        w16 = torch.from_numpy(synth_inputs.weights("normal", N, K, 0).astype(np.float16)).to(device)
+        setb = w16.numel() * 2
+        copies = max(1, -(-3 * l2 // setb) + 1) if setb < 3 * l2 else 1
+        ws16 = [w16] + [w16.clone() for _ in range(copies - 1)]
+        xf = torch.from_numpy(synth_inputs.activations(1, K, "bf16", 0).view(np.int16)).view(torch.bfloat16).to(device)
+        yf = torch.empty((1, N), dtype=torch.float32, device=device)
+
+        def f16(i, ws16=ws16, xf=xf, yf=yf, N=N, K=K, copies=copies):
+            st = lib.q4_f16_gemv(xf.data_ptr(), 1, 1, K, ws16[i % copies].data_ptr(), N, yf.data_ptr(), 1,
+                                 stream.cuda_stream)
+            assert st == 0
+        log(f"rows: {name}")
+        n_l = max(copies * 4, 10)
+        ms = time_launches(torch, f16, n_l, device, stream)
+        b = N * K * 2 + K * 2 + N * 4
+        out[name] = {"workload": f"F16 weights M=1 K={K} N={N} bf16 x", "ms": ms, "GB/s": b / ms / 1e6,
+                     "frac_hbm": b / ms / 1e6 / hbm, "bytes": b, "launches": n_l}
+        del ws16, w16
     # Prefill q4_gemm (bf16 x, bf16 y, f32 accumulate); inputs rotated to exceed 3x L2.
     for gw in synth_inputs.PREFILL:
         _, packed, scales = make_quantized(torch, q4, gw, 0, device)

@@ -17,7 +17,7 @@ from . import _lib
 from ._lib import Q4Error, FLAG_NONFINITE, FLAG_SCALE_OVERFLOW, GEMV_MAX_M  # noqa: F401
 
 __all__ = [
-    "quantize", "gemv", "gemv_multi", "GemvMulti", "gemv_gate_up", "gemv_argmax", "gemm", "gemv_workspace_size", "gemv_multi_workspace_size",
+    "quantize", "gemv", "gemv_multi", "GemvMulti", "gemv_gate_up", "gemv_argmax", "f16_gemv", "gemm", "gemv_workspace_size", "gemv_multi_workspace_size",
     "Q4Error", "FLAG_NONFINITE", "FLAG_SCALE_OVERFLOW", "GEMV_MAX_M",
 ]
 
@@ -238,6 +238,34 @@ def gemv_argmax(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, log
                                 workspace.numel(), _stream())
     _lib.check(st, "q4_gemv_argmax")
     return index, value, y
+
+
+def f16_gemv(x: torch.Tensor, w: torch.Tensor, out: torch.Tensor | None = None, weights_static: bool = False):
+    """y[M,N] (f32) = x[M,K] . W^T for binary16 weights W [N,K] (torch.float16), on the
+    tensor cores; x is f32 (M == 1) or bf16 (M <= 16), K a multiple of 8."""
+    if x.dtype is torch.float32:
+        xt = _lib.Q4_F32
+    elif x.dtype is torch.bfloat16:
+        xt = _lib.Q4_BF16
+    else:
+        raise TypeError("x must be float32 or bfloat16")
+    _need(x, "x", x.dtype, 2)
+    _need(w, "w", torch.float16, 2, x.device)
+    M, K = x.shape
+    N = w.shape[0]
+    if w.shape[1] != K:
+        raise ValueError("shape mismatch between x and w")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float32, device=x.device)
+    else:
+        _need(out, "out", torch.float32, 2, x.device)
+        if tuple(out.shape) != (M, N):
+            raise ValueError("out has the wrong shape")
+    with _on(x.device):
+        st = _lib.load().q4_f16_gemv(x.data_ptr(), xt, M, K, w.data_ptr(), N, out.data_ptr(),
+                                     _lib.WEIGHTS_STATIC if weights_static else 0, _stream())
+    _lib.check(st, "q4_f16_gemv")
+    return out
 
 
 class GemvMulti:

@@ -46,6 +46,7 @@ SIGNATURES = {
     "q4_gemv_multi_workspace_size": (_sz, [_i64, _i64, _vp, _i32]),
     "q4_gemv_multi": (_i32, [_vp, _i32, _i64, _i64, _vp, _i32, ctypes.c_uint32, _vp, _sz, _vp]),
     "q4_gemv_gate_up": (_i32, [_vp, _i32, _i64, _i64, _vp, _vp, _vp, _vp, _i64, _vp, ctypes.c_uint32, _vp]),
+    "q4_f16_gemv": (_i32, [_vp, _i32, _i64, _i64, _vp, _i64, _vp, ctypes.c_uint32, _vp]),
     "q4_gemv_argmax_workspace_size": (_sz, []),
     "q4_gemv_argmax": (_i32, [_vp, _i32, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _vp, ctypes.c_uint32, _vp, _sz,
                               _vp]),

@@ -266,6 +266,23 @@ q4_status q4_gemv_argmax(const void* x, q4_dtype x_dtype, int64_t M, int64_t K, 
                                static_cast<cudaStream_t>(stream), false, &am);
 }
 
+q4_status q4_f16_gemv(const void* x, q4_dtype x_dtype, int64_t M, int64_t K, const uint16_t* w, int64_t N, float* y,
+                      uint32_t flags, void* stream)
+{
+    if (x_dtype != Q4_F32 && x_dtype != Q4_BF16) return Q4_ERR_DTYPE;
+    if (M < 0 || M > Q4_GEMV_MAX_M || (M > 1 && x_dtype != Q4_BF16)) return Q4_ERR_SHAPE;
+    if (K < 8 || K % 8 != 0 || K > INT32_MAX || N < 0 || N > INT32_MAX) return Q4_ERR_SHAPE;
+    if (flags & ~Q4_WEIGHTS_STATIC) return Q4_ERR_INVALID_ARG;
+    if (M == 0 || N == 0) return Q4_OK;
+    if (!x || !w || !y) return Q4_ERR_INVALID_ARG;
+    if (misaligned(x, 16) || misaligned(w, 16) || misaligned(y, 4)) return Q4_ERR_ALIGN;
+    q4::DeviceInfo dev;
+    q4_status st = q4::current_device(&dev);
+    if (st != Q4_OK) return st;
+    return q4::launch_f16_gemv(x, x_dtype, M, K, w, N, y, (flags & Q4_WEIGHTS_STATIC) ? 1 : 0,
+                               static_cast<cudaStream_t>(stream), dev);
+}
+
 q4_status q4_gemm(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed, const uint16_t* scales,
                   int64_t N, uint16_t* y, void* stream)
 {

@@ -66,6 +66,9 @@ q4_status launch_gemv_tma(const void* x, q4_dtype xt, int64_t M, int64_t K, cons
                           int prefetch, void* workspace, const GemvPlan& plan, cudaStream_t stream,
                           bool fuse = false, const ArgmaxOut* am = nullptr);
 
+q4_status launch_f16_gemv(const void* x, q4_dtype xt, int64_t M, int64_t K, const uint16_t* w, int64_t N, float* y,
+                          int prefetch, cudaStream_t stream, const DeviceInfo& dev);
+
 q4_status launch_gemm(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed, const uint16_t* scales,
                       int64_t N, uint16_t* y, cudaStream_t stream, const DeviceInfo& dev);
 

@@ -213,6 +213,25 @@ Q4_API q4_status q4_gemv_argmax(const void* x, q4_dtype x_dtype, int64_t M, int6
                                 uint32_t flags, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * q4_f16_gemv: y[M,N] = x[M,K] . W^T for binary16 weights W (2 bytes per weight), the
+ * pages' second weight format (QORA-LLM-0.8B model card, section "AVX-512 SIMD
+ * Acceleration": "F16 GEMV").  Same roles as q4_gemv, without quantisation:
+ *   x        device, f32 (M == 1) or bfloat16 (M = 1..16) [M,K], 16-byte aligned.
+ *   K        a positive multiple of 8 (16-byte weight rows); any such K.
+ *   w        device, binary16 bits [N,K] row-major, 16-byte aligned.
+ *   y        device, f32 [M,N], 4-byte aligned (output, overwritten).
+ *   flags    0 or Q4_WEIGHTS_STATIC, as for q4_gemv_multi.
+ * Arithmetic: the products run on the tensor cores with binary16 operands and f32
+ * accumulation.  bf16 x row m is scaled by a power of two 2^-e_m that puts max |x| in
+ * [2^14, 2^15) and converted to binary16, exact for every value above max |x| * 2^-24;
+ * f32 x is split into two binary16 parts (22 significant bits); y is scaled back by
+ * 2^e_m.  No workspace.  M == 0 or N == 0 is a no-op; a K whose x does not fit in
+ * shared memory returns Q4_ERR_SHAPE.
+ */
+Q4_API q4_status q4_f16_gemv(const void* x, q4_dtype x_dtype, int64_t M, int64_t K, const uint16_t* w, int64_t N,
+                             float* y, uint32_t flags, void* stream);
+
+/*
  * q4_gemm: y = bf16( x . dequant(W)^T ) for prefill (any M >= 0; tuned for M >= 512).
  * The pages batch the prefill projections across tokens into GEMMs (QORA-4B thread,
  * section "GPU 预填充优化"; QORA-LLM-0.8B model card, section "Performance").

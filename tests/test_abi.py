@@ -156,3 +156,17 @@ def test_argmax_validation(lib):
     assert f(A16, 1, 1, 256, A16, A8, 8, None, A16, None, 0, A16, W, S) == 3       # scales: 16 bytes
     assert f(A16, 1, 1, 96, A16, A16, 8, None, A16, None, 0, A16, W, S) == 2       # K % 256
     assert f(None, 1, 0, 256, None, None, 8, None, None, None, 0, None, 0, S) == 0  # M == 0: no-op
+
+
+def test_f16_gemv_validation(lib):
+    S = None
+    f = lib.q4_f16_gemv
+    assert f(A16, 7, 1, 64, A16, 8, A16, 0, S) == 4                 # dtype
+    assert f(A16, 0, 2, 64, A16, 8, A16, 0, S) == 2                 # f32 x with M > 1
+    assert f(A16, 1, 17, 64, A16, 8, A16, 0, S) == 2                # M > 16
+    assert f(A16, 1, 1, 12, A16, 8, A16, 0, S) == 2                 # K % 8
+    assert f(A16, 1, 1, 64, A16, 8, A16, 2, S) == 1                 # unknown flag
+    assert f(A16, 1, 1, 64, None, 8, A16, 0, S) == 1
+    assert f(A16, 1, 1, 64, A8, 8, A16, 0, S) == 3                  # w alignment
+    assert f(A16, 1, 1, 64, A16, 8, A16 + 2, 0, S) == 3             # y alignment
+    assert f(None, 1, 0, 64, None, 8, None, 0, S) == 0              # M == 0: no-op
