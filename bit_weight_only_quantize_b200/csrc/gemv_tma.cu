@@ -82,10 +82,9 @@ struct TmaGemvArgs {
     int P;                            // warps per team
     int teams;                        // teams per block
     int prefetch;                     // weights may be read before the dependency wait
-    int fuse;                         // gate+up: matrices 0 and 1 (equal N), y = silu(y0) * y1 into y[0]
-    // greedy argmax over the rows of matrix 0 (splits == 1): per x row, the largest logit
-    // and its row; keys and the block counter live in a workspace that is zero at rest
-    int argmax;
+    // kEpiArgmax (greedy argmax over the rows of matrix 0, splits == 1): per x row, the
+    // largest logit and its row; keys and the block counter live in a workspace that is
+    // zero at rest.  (kEpiFuse: matrices 0 and 1 are gate and up, y = silu(y0) * y1 into y[0].)
     unsigned long long* am_key;       // [M] (value order, then lowest row)
     unsigned* am_done;                // blocks finished
     long long* am_index;              // [M] output
@@ -247,12 +246,18 @@ struct ModeCfg {
     static constexpr int kMinBlocks = 1;
 };
 
-template <int MODE>
+// Row-block epilogues: plain stores, fused gate+up, greedy argmax (compile-time, so the
+// plain GEMV carries none of the others' code or registers).
+enum Epi { kEpiPlain = 0, kEpiFuse = 1, kEpiArgmax = 2 };
+
+template <int MODE, int EPI>
 __global__ void __launch_bounds__(kMaxWarps * 32, ModeCfg<MODE>::kMinBlocks)
 gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
 {
     constexpr int MP = ModeCfg<MODE>::MP;
     constexpr int NT = ModeCfg<MODE>::NT;
+    constexpr bool kFuse = EPI == kEpiFuse;
+    constexpr bool kArgmax = EPI == kEpiArgmax;
     extern __shared__ unsigned char smem_raw[];
     __shared__ int s_last[kMaxWarps];
     const int W = blockDim.x >> 5;
@@ -280,11 +285,11 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
     // up block p (= p + the gate's block count) of each pair in turn.
     const int first_rb = blockIdx.x * a.teams + team;
     const int rb_stride = gridDim.x * a.teams;
-    const int walk = a.fuse ? a.rb_begin[1] : a.row_blocks;
+    const int walk = kFuse ? a.rb_begin[1] : a.row_blocks;
     const int nwalk = (active && first_rb < walk) ? (walk - first_rb + rb_stride - 1) / rb_stride : 0;
-    const int nrb = a.fuse ? 2 * nwalk : nwalk;                           // row-block visits
+    const int nrb = kFuse ? 2 * nwalk : nwalk;                           // row-block visits
     auto rb_of = [&](int i) {
-        return a.fuse ? first_rb + (i >> 1) * rb_stride + (i & 1) * a.rb_begin[1] : first_rb + i * rb_stride;
+        return kFuse ? first_rb + (i >> 1) * rb_stride + (i & 1) * a.rb_begin[1] : first_rb + i * rb_stride;
     };
     const int njobs = nrb * nbw;
     uint64_t* my_bars = bars + warp * kStages;
@@ -409,7 +414,7 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
 
     bool ok = true;
     int consumed = 0;
-    float gsave[kRows * Q4_GEMV_MAX_M / 32];       // fuse: the gate totals of the current pair
+    float gsave[kFuse ? kRows * Q4_GEMV_MAX_M / 32 : 1];   // fuse: the gate totals of the current pair
     for (int rbi = 0; rbi < nrb; ++rbi) {
         const int rb = rb_of(rbi);
         float yacc = 0.f;     // kF32M1: row (lane & 15), half (lane >> 4)
@@ -537,7 +542,7 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
             const int nrow = a.N[mi];
             const int lrow0 = (rb - a.rb_begin[mi]) * kRows;
             const size_t vrows = (size_t)a.row_blocks * kRows;            // padded rows over all matrices
-            if (a.fuse) {                       // splits == 1: gate totals wait in registers
+            if constexpr (kFuse) {                       // splits == 1: gate totals wait in registers
 #pragma unroll
                 for (int it = 0; it < kRows * Q4_GEMV_MAX_M / 32; ++it) {
                     const int e = lane + 32 * it;
@@ -554,7 +559,7 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
                     }
                 }
             }
-            for (int e0 = 0; e0 < (a.fuse ? 0 : kRows * a.M); e0 += 32) {   // x row major: coalesced y
+            for (int e0 = 0; e0 < (kFuse ? 0 : kRows * a.M); e0 += 32) {   // x row major: coalesced y
                 const int e = e0 + lane;
                 const int m = e / kRows, rr = e - m * kRows;
                 const bool live = e < kRows * a.M && lrow0 + rr < nrow;
@@ -565,7 +570,7 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
                     if (a.splits > 1) a.partial[((size_t)split * a.M + m) * vrows + (size_t)rb * kRows + rr] = total;
                     else if (a.y[mi]) a.y[mi][(size_t)m * nrow + lrow0 + rr] = total;
                 }
-                if (a.argmax) {                // the 16 lanes of one x row agree on its best row
+                if constexpr (kArgmax) {                // the 16 lanes of one x row agree on its best row
                     unsigned long long key = live ? argmax_key(total, lrow0 + rr) : 0ull;
 #pragma unroll
                     for (int o = 1; o < kRows; o <<= 1) {
@@ -604,7 +609,7 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
             if (!mbar_wait_bounded(&my_bars[j % kStages], (uint32_t)(j / kStages) & 1u, kWaitLimit)) break;
     }
 
-    if (a.argmax) {                                // the last block to finish reports and resets
+    if constexpr (kArgmax) {                                // the last block to finish reports and resets
         __syncthreads();
         if (threadIdx.x == 0) {
             __threadfence();
@@ -647,14 +652,21 @@ int mode_for(int64_t M, q4_dtype xt)
     return M == 1 ? kMma1 : M <= 8 ? kMma8 : kMma16;
 }
 
-const void* kernel_for(int mode)
+template <int EPI>
+const void* kernel_for_epi(int mode)
 {
     switch (mode) {
-    case kF32M1: return reinterpret_cast<const void*>(&gemv_tma_kernel<kF32M1>);
-    case kMma8: return reinterpret_cast<const void*>(&gemv_tma_kernel<kMma8>);
-    case kMma1: return reinterpret_cast<const void*>(&gemv_tma_kernel<kMma1>);
-    default: return reinterpret_cast<const void*>(&gemv_tma_kernel<kMma16>);
+    case kF32M1: return reinterpret_cast<const void*>(&gemv_tma_kernel<kF32M1, EPI>);
+    case kMma8: return reinterpret_cast<const void*>(&gemv_tma_kernel<kMma8, EPI>);
+    case kMma1: return reinterpret_cast<const void*>(&gemv_tma_kernel<kMma1, EPI>);
+    default: return reinterpret_cast<const void*>(&gemv_tma_kernel<kMma16, EPI>);
     }
+}
+
+const void* kernel_for(int mode, int epi)
+{
+    return epi == kEpiFuse ? kernel_for_epi<kEpiFuse>(mode)
+                           : epi == kEpiArgmax ? kernel_for_epi<kEpiArgmax>(mode) : kernel_for_epi<kEpiPlain>(mode);
 }
 
 }  // namespace
@@ -733,7 +745,8 @@ bool plan_gemv_tma(int64_t M, const int64_t* Ns, int count, int64_t K, q4_dtype 
     const int warps = P * teams;
     const size_t smem = smem_bytes(mode, warps, nb, M);
     if (smem > budget) return false;
-    const int per_sm = blocks_per_sm(kernel_for(mode), warps * 32, smem);
+    const int per_sm = blocks_per_sm(kernel_for(mode, fuse ? kEpiFuse : whole_k ? kEpiArgmax : kEpiPlain), warps * 32,
+                                     smem);
     if (per_sm < 1) return false;
     const long long blocks_needed = ((long long)walk + teams - 1) / teams;
     long long gx = (long long)dev.sm_count * per_sm / splits;
@@ -798,8 +811,6 @@ q4_status launch_gemv_tma(const void* x, q4_dtype xt, int64_t M, int64_t K, cons
     a.P = plan.chunk;
     a.teams = plan.xcap;
     a.prefetch = prefetch;
-    a.fuse = fuse ? 1 : 0;
-    a.argmax = am ? 1 : 0;
     a.am_key = am ? am->key : nullptr;
     a.am_done = am ? am->done : nullptr;
     a.am_index = am ? am->index : nullptr;
@@ -816,7 +827,8 @@ q4_status launch_gemv_tma(const void* x, q4_dtype xt, int64_t M, int64_t K, cons
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     void* args[] = {&maps, &a};
-    const cudaError_t e = cudaLaunchKernelExC(&cfg, kernel_for(mode_for(M, xt)), args);
+    const int epi = fuse ? kEpiFuse : am ? kEpiArgmax : kEpiPlain;
+    const cudaError_t e = cudaLaunchKernelExC(&cfg, kernel_for(mode_for(M, xt), epi), args);
     return e == cudaSuccess ? Q4_OK : Q4_ERR_CUDA;
 }
 
