@@ -240,6 +240,20 @@ def timed_graph(torch, launch, steps, period, stream):
     return run, graphs
 
 
+def max_over_ranks(torch, ms, dist, device):
+    """The slowest rank's time (every rank gets it); ms itself without a process group."""
+    if dist is None:
+        return ms
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_gbs(world, bytes_per_step, steps, ms):
+    """Whole-job GB/s: every rank moved bytes_per_step per step, in the slowest rank's time."""
+    return world * bytes_per_step * steps / (ms * 1e-3) / 1e9
+
+
 def measure_main(torch, q4, lib, args, world, rank, device, peaks, dist):
     props = torch.cuda.get_device_properties(device)
     l2 = int(getattr(props, "L2_cache_size", 126 * 2 ** 20))
@@ -280,11 +294,7 @@ def measure_main(torch, q4, lib, args, world, rank, device, peaks, dist):
     if dist is not None:
         dist.barrier()
     ms = e0.elapsed_time(e1)
-    ms_max = ms
-    if dist is not None:
-        t = torch.tensor([ms], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_max = float(t.item())
+    ms_max = max_over_ranks(torch, ms, dist, device)
     log(f"timed {ms:.3f} ms; checking outputs")
     err = step.check()
     del graphs
@@ -319,12 +329,8 @@ def measure_e2e(torch, q4, step, steps, device, dist=None, world=1):
         one(i)
     e1.record(stream)
     torch.cuda.synchronize(device)
-    ms = e0.elapsed_time(e1) / n
-    if dist is not None:
-        t = torch.tensor([ms], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    return {"value": world * STEP_BYTES / (ms * 1e-3) / 1e9, "unit": UNIT,
+    ms = max_over_ranks(torch, e0.elapsed_time(e1) / n, dist, device)
+    return {"value": job_gbs(world, STEP_BYTES, 1, ms), "unit": UNIT,
             "h2d_bytes_per_step": x_host.numel() * 2,
             "d2h_bytes_per_step": y_host.numel() * 4,
             "steps": n, "ms_per_step": ms,
@@ -675,7 +681,7 @@ def main():
 
     step, ms, clocks, err = measure_main(torch, q4, lib, args, world, rank, device, peaks, dist)
     ms_step = ms / args.steps
-    value = world * STEP_BYTES * args.steps / (ms * 1e-3) / 1e9
+    value = job_gbs(world, STEP_BYTES, args.steps, ms)
     per_gpu = STEP_BYTES / (ms_step * 1e-3) / 1e9
     launches = args.steps
     traffic = recorded_traffic("gemv_tma_kernel", "decode_proj", "gemv_tma.cu")
