@@ -203,6 +203,44 @@ def argmax(x: np.ndarray, packed: np.ndarray, scales: np.ndarray, threads: int =
     return idx, y[np.arange(y.shape[0]), idx]
 
 
+def select_topk(values: np.ndarray, indices: np.ndarray, k: int):
+    """The k best (value, index) candidates of each row of ``values`` [M, C] (binary64 or
+    float32) with row numbers ``indices`` [M, C] (int64): larger value first, the lower
+    index among equal values, and a NaN above every number (as numpy's argmax reports a
+    NaN).  Returns (index [M, k] int64, value [M, k] float64); when a row has fewer than k
+    candidates the tail holds index -1 and value NaN.
+
+    This is the ranking the top-k sampler of the QORA-LLM-0.8B model card (section
+    "Sampling Defaults", top_k 20) starts from, written as a plain sort; merging the
+    per-shard lists of an N-sharded LM head is the same selection over their union.
+    """
+    values = np.asarray(values, dtype=np.float64)
+    indices = np.asarray(indices, dtype=np.int64)
+    if values.shape != indices.shape or values.ndim != 2:
+        raise ValueError("values and indices must both be [M, C]")
+    if k < 1:
+        raise ValueError("k must be at least 1")
+    M, C = values.shape
+    out_i = np.full((M, k), -1, dtype=np.int64)
+    out_v = np.full((M, k), np.nan, dtype=np.float64)
+    for m in range(M):
+        nan = np.isnan(values[m])
+        # lexsort sorts by its last key first: NaN first, then larger value, then lower index
+        order = np.lexsort((indices[m], -np.where(nan, 0.0, values[m]), ~nan))
+        take = order[:min(k, C)]
+        out_i[m, :take.size] = indices[m, take]
+        out_v[m, :take.size] = values[m, take]
+    return out_i, out_v
+
+
+def topk(x: np.ndarray, packed: np.ndarray, scales: np.ndarray, k: int, threads: int = 1, row_base: int = 0):
+    """The k largest logits of y = x . dequant(W)^T (binary64) per x row and their rows
+    (``row_base`` added, for a shard of a larger LM head), ordered as ``select_topk``."""
+    y = matmul(x, packed, scales, threads=threads)
+    rows = np.broadcast_to(np.arange(y.shape[1], dtype=np.int64) + row_base, y.shape)
+    return select_topk(y, rows, k)
+
+
 def f16_matmul(x: np.ndarray, w16: np.ndarray, threads: int = 1) -> np.ndarray:
     """y = x . W^T in binary64 for binary16 weights W (the F16 GEMV of the QORA-LLM-0.8B
     model card, section "AVX-512 SIMD Acceleration").  w16: uint16 binary16 bits [N, K];
