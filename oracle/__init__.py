@@ -207,8 +207,9 @@ def select_topk(values: np.ndarray, indices: np.ndarray, k: int):
     """The k best (value, index) candidates of each row of ``values`` [M, C] (binary64 or
     float32) with row numbers ``indices`` [M, C] (int64): larger value first, the lower
     index among equal values, and a NaN above every number (as numpy's argmax reports a
-    NaN).  Returns (index [M, k] int64, value [M, k] float64); when a row has fewer than k
-    candidates the tail holds index -1 and value NaN.
+    NaN).  A candidate with a negative index is padding (the tail of a short list) and
+    takes no place.  Returns (index [M, k] int64, value [M, k] float64); when a row has
+    fewer than k candidates the tail holds index -1 and value NaN.
 
     This is the ranking the top-k sampler of the QORA-LLM-0.8B model card (section
     "Sampling Defaults", top_k 20) starts from, written as a plain sort; merging the
@@ -224,12 +225,14 @@ def select_topk(values: np.ndarray, indices: np.ndarray, k: int):
     out_i = np.full((M, k), -1, dtype=np.int64)
     out_v = np.full((M, k), np.nan, dtype=np.float64)
     for m in range(M):
-        nan = np.isnan(values[m])
+        real = np.nonzero(indices[m] >= 0)[0]
+        v, r = values[m, real], indices[m, real]
+        nan = np.isnan(v)
         # lexsort sorts by its last key first: NaN first, then larger value, then lower index
-        order = np.lexsort((indices[m], -np.where(nan, 0.0, values[m]), ~nan))
-        take = order[:min(k, C)]
-        out_i[m, :take.size] = indices[m, take]
-        out_v[m, :take.size] = values[m, take]
+        order = np.lexsort((r, -np.where(nan, 0.0, v), ~nan))
+        take = order[:k]
+        out_i[m, :take.size] = r[take]
+        out_v[m, :take.size] = v[take]
     return out_i, out_v
 
 

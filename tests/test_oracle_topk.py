@@ -22,7 +22,7 @@ def _q(W):
 def _brute(values, rows, k):
     out = []
     for vr, ir in zip(values.tolist(), rows.tolist()):
-        best = sorted(zip(vr, ir), key=lambda t: (0 if math.isnan(t[0]) else 1,
+        best = sorted([(v, i) for v, i in zip(vr, ir) if i >= 0], key=lambda t: (0 if math.isnan(t[0]) else 1,
                                                   0.0 if math.isnan(t[0]) else -t[0], t[1]))[:k]
         best += [(math.nan, -1)] * (k - len(best))
         out.append(best)
@@ -92,6 +92,11 @@ def test_nan_ranks_first_and_merge_of_shards():
     idx, val = oracle.select_topk(vals, rows, 4)
     assert idx[0].tolist() == [11, 15, 12, 14]
     _same(idx, val, _brute(vals, rows, 4))
+    # padding (negative index, NaN value) takes no place, even though a NaN ranks first
+    pad = np.array([[np.nan, 2.0, np.nan, 5.0]]), np.array([[-1, 40, -1, 41]])
+    idx, val = oracle.select_topk(*pad, 3)
+    assert idx[0].tolist() == [41, 40, -1] and np.isnan(val[0, 2])
+    _same(idx, val, _brute(*pad, 3))
     # selection over the union of two shards' lists equals selection over all logits
     rng = np.random.default_rng(9)
     y = rng.standard_normal((3, 200))
