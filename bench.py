@@ -401,6 +401,25 @@ def measure_rows(torch, q4, lib, device, peaks, l2):
                              "ms": ms, "GB/s": b / ms / 1e6, "frac_hbm": b / ms / 1e6 / hbm, "bytes": b,
                              "launches": 20}
 
+    # Top-k(20) LM-head step: the list a top-k sampler draws from, logits kept on chip.
+    TK = 20
+    tk_ws = torch.zeros(max(16, q4.gemv_topk_workspace_size(1, w.N, w.K, TK)), dtype=torch.uint8, device=device)
+    tk_idx = torch.empty((1, TK), dtype=torch.int64, device=device)
+    tk_val = torch.empty((1, TK), dtype=torch.float32, device=device)
+
+    def lm_topk(i):
+        st = lib.q4_gemv_topk(x.data_ptr(), 1, 1, w.K, packed.data_ptr(), scales.data_ptr(), w.N, TK, 0, None,
+                              tk_idx.data_ptr(), tk_val.data_ptr(), 1, tk_ws.data_ptr(), tk_ws.numel(),
+                              stream.cuda_stream)
+        assert st == 0
+    log("rows: lm head top-k")
+    ms = time_launches(torch, lm_topk, 20, device, stream)
+    b = w.N * w.K // 2 + w.N * (w.K // 32) * 2 + w.K * 2 + TK * 12
+    out["lm_head_topk20"] = {"workload": "top-k step: M=1 K=2560 N=248320 bf16 x, top-20 fused, no logits out",
+                             "ms": ms, "GB/s": b / ms / 1e6, "frac_hbm": b / ms / 1e6 / hbm, "bytes": b,
+                             "launches": 20,
+                             "matches_argmax": bool(torch.equal(tk_idx[:, 0], am_idx) and torch.equal(tk_val[:, 0], am_val))}
+
     # Quantise the LM-head weights: reads 4 B and writes 0.5625 B per weight.
     Wd = torch.from_numpy(W).to(device)
     del W
@@ -626,6 +645,17 @@ def run_profile_case(args):
             torch.cuda.synchronize(device)
             print(json.dumps({"profile_case": case, "launches": args.warmup + args.steps}))
             return
+        if case == "lm_head_topk":
+            w = synth_inputs.LM_HEAD
+            _, packed, scales = make_quantized(torch, q4, w, 0, device)
+            x = torch.from_numpy(synth_inputs.activations(1, w.K, "bf16", 0).view(np.int16)).view(
+                torch.bfloat16).to(device)
+            ws = torch.zeros(max(16, q4.gemv_topk_workspace_size(1, w.N, w.K, 20)), dtype=torch.uint8, device=device)
+            for _ in range(args.warmup + args.steps):
+                q4.gemv_topk(x, packed, scales, 20, workspace=ws, weights_static=True)
+            torch.cuda.synchronize(device)
+            print(json.dumps({"profile_case": case, "launches": args.warmup + args.steps}))
+            return
         w = {"decode": synth_inputs.DECODE_PROJ[1], "lm_head": synth_inputs.LM_HEAD,
              "gemv_m4": synth_inputs.SMALL_BATCH[1], "decode_small": synth_inputs.DECODE_PROJ[2]}[case]
         _, packed, scales = make_quantized(torch, q4, w, 0, device)
@@ -650,8 +680,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--rows", choices=["all", "main"], default="all")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    ap.add_argument("--profile", choices=["none", "decode", "decode_small", "decode_multi", "lm_head", "gemv_m4", "quantize", "gemm",
-                             "gemm_m2048"],
+    ap.add_argument("--profile", choices=["none", "decode", "decode_small", "decode_multi", "lm_head", "lm_head_topk", "gemv_m4",
+                             "quantize", "gemm", "gemm_m2048"],
                     default="none", help="run a few untimed launches of one row (for ncu) and exit")
     args = ap.parse_args()
     if args.profile != "none":

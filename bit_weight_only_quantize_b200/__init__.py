@@ -17,7 +17,8 @@ from . import _lib
 from ._lib import Q4Error, FLAG_NONFINITE, FLAG_SCALE_OVERFLOW, GEMV_MAX_M  # noqa: F401
 
 __all__ = [
-    "quantize", "gemv", "gemv_multi", "GemvMulti", "gemv_gate_up", "gemv_argmax", "f16_gemv", "gemm", "gemv_workspace_size", "gemv_multi_workspace_size",
+    "quantize", "gemv", "gemv_multi", "GemvMulti", "gemv_gate_up", "gemv_argmax", "gemv_topk",
+    "gemv_topk_workspace_size", "topk_merge", "f16_gemv", "gemm", "gemv_workspace_size", "gemv_multi_workspace_size",
     "Q4Error", "FLAG_NONFINITE", "FLAG_SCALE_OVERFLOW", "GEMV_MAX_M",
 ]
 
@@ -238,6 +239,76 @@ def gemv_argmax(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, log
                                 workspace.numel(), _stream())
     _lib.check(st, "q4_gemv_argmax")
     return index, value, y
+
+
+def gemv_topk(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, k: int, row_base: int = 0,
+              logits: bool = False, workspace: torch.Tensor | None = None, weights_static: bool = False):
+    """The k largest logits of an LM head per x row in one launch: (index int64 [M,k],
+    value f32 [M,k], y or None), larger first, the lower row on ties, rows reported as
+    ``row_base`` + row; past N rows the lists hold -1 / NaN.
+
+    ``logits=True`` also returns the f32 logits [M,N].  ``workspace`` (uint8, its first
+    16 bytes zero before its first use and left zero by every call, at least
+    ``gemv_topk_workspace_size`` bytes) is allocated here when not given.
+    """
+    if x.dtype is torch.float32:
+        xt = _lib.Q4_F32
+    elif x.dtype is torch.bfloat16:
+        xt = _lib.Q4_BF16
+    else:
+        raise TypeError("x must be float32 or bfloat16")
+    _need(x, "x", x.dtype, 2)
+    _need(packed, "packed", torch.uint8, 2, x.device)
+    _need(scales, "scales", torch.int16, 2, x.device)
+    M, K = x.shape
+    N = packed.shape[0]
+    if packed.shape[1] * 2 != K or tuple(scales.shape) != (N, K // 32):
+        raise ValueError("shape mismatch between x, packed and scales")
+    lib = _lib.load()
+    index = torch.empty((M, k), dtype=torch.int64, device=x.device)
+    value = torch.empty((M, k), dtype=torch.float32, device=x.device)
+    y = torch.empty((M, N), dtype=torch.float32, device=x.device) if logits else None
+    with _on(x.device):
+        if workspace is None:
+            size = int(lib.q4_gemv_topk_workspace_size(M, N, K, k, xt)) if M and N else 16
+            workspace = torch.zeros(max(size, 16), dtype=torch.uint8, device=x.device)
+        else:
+            _need(workspace, "workspace", torch.uint8, 1, x.device)
+        st = lib.q4_gemv_topk(x.data_ptr(), xt, M, K, packed.data_ptr(), scales.data_ptr(), N, k, row_base,
+                              y.data_ptr() if y is not None else None, index.data_ptr(), value.data_ptr(),
+                              _lib.WEIGHTS_STATIC if weights_static else 0, workspace.data_ptr(),
+                              workspace.numel(), _stream())
+    _lib.check(st, "q4_gemv_topk")
+    if N == 0:                         # no rows: the lists are all padding
+        index.fill_(-1)
+        value.fill_(float("nan"))
+    return index, value, y
+
+
+def topk_merge(values: torch.Tensor, indices: torch.Tensor, k: int):
+    """The k best entries per x row over S top-k lists (values f32 [S,M,k], indices int64
+    [S,M,k], as gathered from the shards of an LM head), ordered as ``gemv_topk`` orders
+    them: (index int64 [M,k], value f32 [M,k])."""
+    _need(values, "values", torch.float32, 3)
+    _need(indices, "indices", torch.int64, 3, values.device)
+    if tuple(values.shape) != tuple(indices.shape):
+        raise ValueError("values and indices must have the same shape")
+    S, M, kin = values.shape
+    if kin != k:
+        raise ValueError("the lists must hold k entries each")
+    index = torch.empty((M, k), dtype=torch.int64, device=values.device)
+    value = torch.empty((M, k), dtype=torch.float32, device=values.device)
+    with _on(values.device):
+        st = _lib.load().q4_topk_merge(values.data_ptr(), indices.data_ptr(), S, M, k, index.data_ptr(),
+                                       value.data_ptr(), _stream())
+    _lib.check(st, "q4_topk_merge")
+    return index, value
+
+
+def gemv_topk_workspace_size(M: int, N: int, K: int, k: int, x_dtype: torch.dtype = torch.bfloat16) -> int:
+    """Bytes of workspace ``gemv_topk`` needs on the current device (0: shape not served)."""
+    xt = _lib.Q4_F32 if x_dtype is torch.float32 else _lib.Q4_BF16
+    return int(_lib.load().q4_gemv_topk_workspace_size(M, N, K, k, xt))
 
 
 def f16_gemv(x: torch.Tensor, w: torch.Tensor, out: torch.Tensor | None = None, weights_static: bool = False):

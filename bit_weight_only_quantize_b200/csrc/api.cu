@@ -223,12 +223,12 @@ q4_status q4_gemv_gate_up(const void* x, q4_dtype x_dtype, int64_t M, int64_t K,
     const q4_weight mats[2] = {{gate_packed, gate_scales, N, y}, {up_packed, up_scales, N, y}};
     const int64_t Ns[2] = {N, N};
     q4::GemvPlan plan;
-    if (!q4::plan_gemv_tma(M, Ns, 2, K, x_dtype, dev, &plan, true)) {
+    if (!q4::plan_gemv_tma(M, Ns, 2, K, x_dtype, dev, &plan, q4::kGemvFuse)) {
         cudaGetLastError();
         return Q4_ERR_SHAPE;                      // x of this K does not fit beside the rings
     }
     return q4::launch_gemv_tma(x, x_dtype, M, K, mats, 2, (flags & Q4_WEIGHTS_STATIC) ? 1 : 0, nullptr, plan,
-                               static_cast<cudaStream_t>(stream), true);
+                               static_cast<cudaStream_t>(stream), q4::kGemvFuse);
 }
 
 size_t q4_gemv_argmax_workspace_size(void) { return 256; }   // Q4_GEMV_MAX_M keys, then the counter
@@ -253,7 +253,7 @@ q4_status q4_gemv_argmax(const void* x, q4_dtype x_dtype, int64_t M, int64_t K, 
     if ((st = q4::current_device(&dev)) != Q4_OK) return st;
     const q4_weight w = {packed, scales, N, y};
     q4::GemvPlan plan;
-    if (!q4::plan_gemv_tma(M, &N, 1, K, x_dtype, dev, &plan, false, true)) {
+    if (!q4::plan_gemv_tma(M, &N, 1, K, x_dtype, dev, &plan, q4::kGemvArgmax)) {
         cudaGetLastError();
         return Q4_ERR_SHAPE;
     }
@@ -262,8 +262,86 @@ q4_status q4_gemv_argmax(const void* x, q4_dtype x_dtype, int64_t M, int64_t K, 
     am.done = reinterpret_cast<unsigned*>(static_cast<char*>(workspace) + Q4_GEMV_MAX_M * 8);
     am.index = reinterpret_cast<long long*>(index);
     am.value = value;
+    am.cand = nullptr;
+    am.k = 1;
+    am.row_base = 0u;
     return q4::launch_gemv_tma(x, x_dtype, M, K, &w, 1, (flags & Q4_WEIGHTS_STATIC) ? 1 : 0, nullptr, plan,
-                               static_cast<cudaStream_t>(stream), false, &am);
+                               static_cast<cudaStream_t>(stream), q4::kGemvArgmax, &am);
+}
+
+// Top-k workspace: the block counter, then the blocks' lists [M][grid_x][k].
+static constexpr size_t kTopkListsOffset = 256;
+
+static bool topk_shape(int64_t M, int64_t N, int64_t K, int64_t k, q4_dtype x_dtype)
+{
+    return M >= 1 && M <= Q4_GEMV_MAX_M && k >= 1 && k <= Q4_TOPK_MAX && N >= 1 && check_nk(N, K) == Q4_OK &&
+           K % 256 == 0 && (x_dtype == Q4_BF16 || (x_dtype == Q4_F32 && M == 1));
+}
+
+static bool topk_plan(int64_t M, int64_t N, int64_t K, q4_dtype x_dtype, q4::DeviceInfo* dev, q4::GemvPlan* plan)
+{
+    if (q4::current_device(dev) != Q4_OK) return false;
+    if (!q4::plan_gemv_tma(M, &N, 1, K, x_dtype, *dev, plan, q4::kGemvTopk)) {
+        cudaGetLastError();
+        return false;
+    }
+    return true;
+}
+
+size_t q4_gemv_topk_workspace_size(int64_t M, int64_t N, int64_t K, int64_t k, q4_dtype x_dtype)
+{
+    q4::DeviceInfo dev;
+    q4::GemvPlan plan;
+    if (!topk_shape(M, N, K, k, x_dtype) || !topk_plan(M, N, K, x_dtype, &dev, &plan)) return 0;
+    return kTopkListsOffset + (size_t)M * (size_t)plan.grid_x * (size_t)k * sizeof(unsigned long long);
+}
+
+q4_status q4_gemv_topk(const void* x, q4_dtype x_dtype, int64_t M, int64_t K, const uint8_t* packed,
+                       const uint16_t* scales, int64_t N, int64_t k, int64_t row_base, float* y, int64_t* index,
+                       float* value, uint32_t flags, void* workspace, size_t workspace_bytes, void* stream)
+{
+    if (x_dtype != Q4_F32 && x_dtype != Q4_BF16) return Q4_ERR_DTYPE;
+    if (M < 0 || M > Q4_GEMV_MAX_M) return Q4_ERR_SHAPE;
+    q4_status st = check_nk(N, K);
+    if (st != Q4_OK) return st;
+    if (k < 1 || k > Q4_TOPK_MAX || row_base < 0 || row_base > INT32_MAX - N) return Q4_ERR_SHAPE;
+    if (flags & ~Q4_WEIGHTS_STATIC) return Q4_ERR_INVALID_ARG;
+    if (M == 0 || N == 0) return Q4_OK;
+    if (!x || !packed || !scales || !index) return Q4_ERR_INVALID_ARG;
+    if (!workspace) return Q4_ERR_WORKSPACE;
+    if (misaligned(x, 16) || misaligned(packed, 16) || misaligned(scales, 16) || (y && misaligned(y, 4)) ||
+        misaligned(index, 8) || (value && misaligned(value, 4)) || misaligned(workspace, 16))
+        return Q4_ERR_ALIGN;
+    if (!topk_shape(M, N, K, k, x_dtype)) return Q4_ERR_SHAPE;
+    q4::DeviceInfo dev;
+    q4::GemvPlan plan;
+    if (!topk_plan(M, N, K, x_dtype, &dev, &plan)) return Q4_ERR_SHAPE;
+    if (workspace_bytes < kTopkListsOffset + (size_t)M * (size_t)plan.grid_x * (size_t)k * 8) return Q4_ERR_WORKSPACE;
+    const q4_weight w = {packed, scales, N, y};
+    q4::ArgmaxOut am;
+    am.key = nullptr;
+    am.done = static_cast<unsigned*>(workspace);
+    am.index = reinterpret_cast<long long*>(index);
+    am.value = value;
+    am.cand = reinterpret_cast<unsigned long long*>(static_cast<char*>(workspace) + kTopkListsOffset);
+    am.k = (int)k;
+    am.row_base = (unsigned)row_base;
+    return q4::launch_gemv_tma(x, x_dtype, M, K, &w, 1, (flags & Q4_WEIGHTS_STATIC) ? 1 : 0, nullptr, plan,
+                               static_cast<cudaStream_t>(stream), q4::kGemvTopk, &am);
+}
+
+q4_status q4_topk_merge(const float* values, const int64_t* indices, int64_t S, int64_t M, int64_t k,
+                        int64_t* index, float* value, void* stream)
+{
+    if (S < 1 || S > (1 << 20) || M < 0 || M > INT32_MAX / 4 || k < 1 || k > Q4_TOPK_MAX) return Q4_ERR_SHAPE;
+    if (M == 0) return Q4_OK;
+    if (!values || !indices || !index) return Q4_ERR_INVALID_ARG;
+    if (misaligned(values, 4) || misaligned(indices, 8) || misaligned(index, 8) || (value && misaligned(value, 4)))
+        return Q4_ERR_ALIGN;
+    q4::DeviceInfo dev;
+    const q4_status st = q4::current_device(&dev);
+    if (st != Q4_OK) return st;
+    return q4::launch_topk_merge(values, indices, S, M, k, index, value, static_cast<cudaStream_t>(stream));
 }
 
 q4_status q4_f16_gemv(const void* x, q4_dtype x_dtype, int64_t M, int64_t K, const uint16_t* w, int64_t N, float* y,

@@ -34,6 +34,7 @@
 #include <algorithm>
 
 #include "tma.cuh"
+#include "topk.cuh"
 
 namespace q4 {
 namespace {
@@ -85,27 +86,17 @@ struct TmaGemvArgs {
     // kEpiArgmax (greedy argmax over the rows of matrix 0, splits == 1): per x row, the
     // largest logit and its row; keys and the block counter live in a workspace that is
     // zero at rest.  (kEpiFuse: matrices 0 and 1 are gate and up, y = silu(y0) * y1 into y[0].)
+    // kEpiTopk (the k largest logits of matrix 0, splits == 1): each team keeps a sorted
+    // list per x row, each block merges its teams' lists into tk_cand [M][gridDim.x][k],
+    // and the last block merges those.  Rows are reported as row_base + row.
     unsigned long long* am_key;       // [M] (value order, then lowest row)
     unsigned* am_done;                // blocks finished
-    long long* am_index;              // [M] output
-    float* am_value;                  // [M] output, may be null
+    long long* am_index;              // [M] output ([M][k] for top-k)
+    float* am_value;                  // [M] output ([M][k]), may be null
+    unsigned long long* tk_cand;      // top-k: per-block lists
+    int tk_k;                         // top-k: list length, 1..32
+    unsigned row_base;                // argmax / top-k: added to every reported row
 };
-
-// Orderable 64-bit key of (logit v, row r): larger v wins, then the lower row; every NaN
-// counts as the largest value (a NaN logit is reported, as numpy's argmax does).
-__device__ __forceinline__ unsigned long long argmax_key(float v, int r)
-{
-    uint32_t b = __float_as_uint(v);
-    if ((b & 0x7FFFFFFFu) > 0x7F800000u) b = 0x7FC00000u;
-    const uint32_t ord = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-    return ((unsigned long long)ord << 32) | (0xFFFFFFFFu - (uint32_t)r);
-}
-
-__device__ __forceinline__ float argmax_value(unsigned long long key)
-{
-    const uint32_t ord = (uint32_t)(key >> 32);
-    return __uint_as_float((ord & 0x80000000u) ? (ord & 0x7FFFFFFFu) : ~ord);
-}
 
 __device__ __forceinline__ void team_sync(int team, int P)
 {
@@ -248,7 +239,7 @@ struct ModeCfg {
 
 // Row-block epilogues: plain stores, fused gate+up, greedy argmax (compile-time, so the
 // plain GEMV carries none of the others' code or registers).
-enum Epi { kEpiPlain = 0, kEpiFuse = 1, kEpiArgmax = 2 };
+enum Epi { kEpiPlain = kGemvPlain, kEpiFuse = kGemvFuse, kEpiArgmax = kGemvArgmax, kEpiTopk = kGemvTopk };
 
 template <int MODE, int EPI>
 __global__ void __launch_bounds__(kMaxWarps * 32, ModeCfg<MODE>::kMinBlocks)
@@ -258,6 +249,8 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
     constexpr int NT = ModeCfg<MODE>::NT;
     constexpr bool kFuse = EPI == kEpiFuse;
     constexpr bool kArgmax = EPI == kEpiArgmax;
+    constexpr bool kTopk = EPI == kEpiTopk;
+    constexpr int kTkM = (MODE == kF32M1 || MODE == kMma1) ? 1 : MP;     // x rows a top-k list set covers
     extern __shared__ unsigned char smem_raw[];
     __shared__ int s_last[kMaxWarps];
     const int W = blockDim.x >> 5;
@@ -415,6 +408,9 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
     bool ok = true;
     int consumed = 0;
     float gsave[kFuse ? kRows * Q4_GEMV_MAX_M / 32 : 1];   // fuse: the gate totals of the current pair
+    unsigned long long tk[kTopk ? kTkM + 1 : 1];           // top-k: the team's list per x row
+#pragma unroll
+    for (int i = 0; i < (kTopk ? kTkM + 1 : 1); ++i) tk[i] = 0ull;
     for (int rbi = 0; rbi < nrb; ++rbi) {
         const int rb = rb_of(rbi);
         float yacc = 0.f;     // kF32M1: row (lane & 15), half (lane >> 4)
@@ -559,7 +555,9 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
                     }
                 }
             }
-            for (int e0 = 0; e0 < (kFuse ? 0 : kRows * a.M); e0 += 32) {   // x row major: coalesced y
+            // Lanes cover 32 (x row, row) pairs from e0 on, x row major (coalesced y); the
+            // key of each live total orders it for argmax and top-k (0 when not live).
+            auto rows_out = [&](int e0) {
                 const int e = e0 + lane;
                 const int m = e / kRows, rr = e - m * kRows;
                 const bool live = e < kRows * a.M && lrow0 + rr < nrow;
@@ -570,14 +568,29 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
                     if (a.splits > 1) a.partial[((size_t)split * a.M + m) * vrows + (size_t)rb * kRows + rr] = total;
                     else if (a.y[mi]) a.y[mi][(size_t)m * nrow + lrow0 + rr] = total;
                 }
-                if constexpr (kArgmax) {                // the 16 lanes of one x row agree on its best row
-                    unsigned long long key = live ? argmax_key(total, lrow0 + rr) : 0ull;
+                return live ? argmax_key(total, a.row_base + (uint32_t)(lrow0 + rr)) : 0ull;
+            };
+            if constexpr (kTopk) {                      // lanes 0-15: x row 2h, lanes 16-31: x row 2h + 1
 #pragma unroll
-                    for (int o = 1; o < kRows; o <<= 1) {
-                        const unsigned long long k2 = __shfl_xor_sync(0xffffffffu, key, o);
-                        key = k2 > key ? k2 : key;
+                for (int h = 0; h < (kTkM + 1) / 2; ++h) {
+                    if (h * 32 < kRows * a.M) {
+                        const unsigned long long key = rows_out(h * 32);
+                        topk_insert(tk[2 * h], key, lane < 16, a.tk_k, lane);
+                        if (2 * h + 1 < kTkM) topk_insert(tk[2 * h + 1], key, lane >= 16, a.tk_k, lane);
                     }
-                    if (rr == 0 && m < a.M && key) atomicMax(&a.am_key[m], key);
+                }
+            } else {
+                for (int e0 = 0; e0 < (kFuse ? 0 : kRows * a.M); e0 += 32) {
+                    unsigned long long key = rows_out(e0);
+                    if constexpr (kArgmax) {            // the 16 lanes of one x row agree on its best row
+                        const int m = (e0 + lane) / kRows;
+#pragma unroll
+                        for (int o = 1; o < kRows; o <<= 1) {
+                            const unsigned long long k2 = __shfl_xor_sync(0xffffffffu, key, o);
+                            key = k2 > key ? k2 : key;
+                        }
+                        if ((lane & (kRows - 1)) == 0 && m < a.M && key) atomicMax(&a.am_key[m], key);
+                    }
                 }
             }
             if (a.splits > 1) {
@@ -626,6 +639,70 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
             if (threadIdx.x == 0) *a.am_done = 0u;
         }
     }
+
+    if constexpr (kTopk) {
+        // Every team is past its last row block, so the code rings are free: each team
+        // leader parks its lists in its own warp's ring, then warp m merges the teams'
+        // lists of x row m into this block's list.
+        const int kk = a.tk_k;
+        constexpr int kRingWords = kStages * kStageCodes / 8;          // u64 per warp ring
+        unsigned long long* lists = reinterpret_cast<unsigned long long*>(codes);
+        __syncthreads();
+        if (active && wt == 0) {
+#pragma unroll
+            for (int mm = 0; mm < kTkM; ++mm)
+                if (mm < a.M && lane < kk) lists[(size_t)warp * kRingWords + mm * kk + lane] = tk[mm];
+            if (lane == 0) s_last[team] = ok;
+        }
+        __syncthreads();
+        for (int m = warp; m < a.M; m += W) {
+            unsigned long long list = 0ull;
+            for (int t = 0; t < a.teams; ++t) {
+                if (!s_last[t]) continue;                               // a team that gave up
+                const unsigned long long c = lane < kk ? lists[(size_t)t * P * kRingWords + m * kk + lane] : 0ull;
+                topk_insert(list, c, true, kk, lane);
+            }
+            if (lane < kk) a.tk_cand[((size_t)m * gridDim.x + blockIdx.x) * kk + lane] = list;
+            __threadfence();
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            __threadfence();
+            s_last[0] = atomicAdd(a.am_done, 1u) == gridDim.x - 1;
+        }
+        __syncthreads();
+        if (s_last[0]) {
+            // The last block: S warps per x row each merge a slice of the blocks' lists,
+            // then warp m merges the S slice lists of x row m and writes the result.
+            __threadfence();
+            const int S = max(1, W / a.M);
+            const int len = gridDim.x * kk;                              // candidates per x row
+            for (int job = warp; job < a.M * S; job += W) {
+                const int m = job / S, sl = job - m * S;
+                const int lo = sl * len / S, hi = (sl + 1) * len / S;
+                const unsigned long long* src = a.tk_cand + (size_t)m * len;
+                unsigned long long list = 0ull;
+                for (int i0 = lo; i0 < hi; i0 += 32) {
+                    const unsigned long long c = i0 + lane < hi ? __ldcg(src + i0 + lane) : 0ull;
+                    topk_insert(list, c, true, kk, lane);
+                }
+                if (lane < kk) lists[(size_t)job * kk + lane] = list;
+            }
+            __syncthreads();
+            for (int m = warp; m < a.M; m += W) {
+                unsigned long long list = 0ull;
+                for (int i0 = 0; i0 < S * kk; i0 += 32) {
+                    const int i = i0 + lane;
+                    topk_insert(list, i < S * kk ? lists[(size_t)m * S * kk + i] : 0ull, true, kk, lane);
+                }
+                if (lane < kk) {
+                    a.am_index[(size_t)m * kk + lane] = list ? (long long)(0xFFFFFFFFu - (uint32_t)list) : -1;
+                    if (a.am_value) a.am_value[(size_t)m * kk + lane] = list ? argmax_value(list) : __int_as_float(0x7FC00000);
+                }
+            }
+            if (threadIdx.x == 0) *a.am_done = 0u;
+        }
+    }
 }
 
 size_t per_warp_bytes(int mode)
@@ -665,8 +742,12 @@ const void* kernel_for_epi(int mode)
 
 const void* kernel_for(int mode, int epi)
 {
-    return epi == kEpiFuse ? kernel_for_epi<kEpiFuse>(mode)
-                           : epi == kEpiArgmax ? kernel_for_epi<kEpiArgmax>(mode) : kernel_for_epi<kEpiPlain>(mode);
+    switch (epi) {
+    case kEpiFuse: return kernel_for_epi<kEpiFuse>(mode);
+    case kEpiArgmax: return kernel_for_epi<kEpiArgmax>(mode);
+    case kEpiTopk: return kernel_for_epi<kEpiTopk>(mode);
+    default: return kernel_for_epi<kEpiPlain>(mode);
+    }
 }
 
 }  // namespace
@@ -679,8 +760,9 @@ bool tma_gemv_eligible(int64_t M, int64_t K, q4_dtype xt, const void* packed, co
 }
 
 bool plan_gemv_tma(int64_t M, const int64_t* Ns, int count, int64_t K, q4_dtype xt, const DeviceInfo& dev,
-                   GemvPlan* p, bool fuse, bool whole_k)
+                   GemvPlan* p, int epi)
 {
+    const bool fuse = epi == kEpiFuse, whole_k = epi != kEpiPlain;
     if (fuse && (count != 2 || Ns[0] != Ns[1])) return false;
     const int mode = mode_for(M, xt);
     const int G = (int)(K / 32);
@@ -724,18 +806,21 @@ bool plan_gemv_tma(int64_t M, const int64_t* Ns, int count, int64_t K, q4_dtype 
         const long long sms = dev.sm_count / sp > 0 ? dev.sm_count / sp : 1;   // blocks of one split
         for (int pp = 1; pp <= nus && pp <= wbs; ++pp) {
             const int pwu = (nus + pp - 1) / pp;                          // units per warp per row block
-            long long tm = wbs / pp;
             const long long spread = ((long long)walk + sms - 1) / sms;
-            if (tm > spread) tm = spread;
-            const long long gxs = std::min(((long long)walk + tm - 1) / tm, sms);
-            const long long rounds = visits * (((long long)walk + gxs * tm - 1) / (gxs * tm));
-            const double share = std::max((double)(tm * pp), kMinWarpShare) / 16.0;
-            const double cost = (double)rounds * (pwu + kEpilogueCost) * share + (sp > 1 ? kSplitCost : 0.0);
-            if (splits == 0 || cost < best - 1e-9) {
-                splits = sp;
-                P = pp;
-                teams = (int)tm;
-                best = cost;
+            // Fewer teams than fit can finish sooner: the last round of row blocks is then
+            // full (e.g. 15 teams of one warp cover 15,520 row blocks in 7 rounds on 148
+            // SMs, 16 teams need 7 rounds of 16 warps each).
+            for (long long tm = std::min<long long>(wbs / pp, spread); tm >= 1; --tm) {
+                const long long gxs = std::min(((long long)walk + tm - 1) / tm, sms);
+                const long long rounds = visits * (((long long)walk + gxs * tm - 1) / (gxs * tm));
+                const double share = std::max((double)(tm * pp), kMinWarpShare) / 16.0;
+                const double cost = (double)rounds * (pwu + kEpilogueCost) * share + (sp > 1 ? kSplitCost : 0.0);
+                if (splits == 0 || cost < best - 1e-9) {
+                    splits = sp;
+                    P = pp;
+                    teams = (int)tm;
+                    best = cost;
+                }
             }
         }
     }
@@ -745,8 +830,7 @@ bool plan_gemv_tma(int64_t M, const int64_t* Ns, int count, int64_t K, q4_dtype 
     const int warps = P * teams;
     const size_t smem = smem_bytes(mode, warps, nb, M);
     if (smem > budget) return false;
-    const int per_sm = blocks_per_sm(kernel_for(mode, fuse ? kEpiFuse : whole_k ? kEpiArgmax : kEpiPlain), warps * 32,
-                                     smem);
+    const int per_sm = blocks_per_sm(kernel_for(mode, epi), warps * 32, smem);
     if (per_sm < 1) return false;
     const long long blocks_needed = ((long long)walk + teams - 1) / teams;
     long long gx = (long long)dev.sm_count * per_sm / splits;
@@ -766,7 +850,7 @@ bool plan_gemv_tma(int64_t M, const int64_t* Ns, int count, int64_t K, q4_dtype 
 }
 
 q4_status launch_gemv_tma(const void* x, q4_dtype xt, int64_t M, int64_t K, const q4_weight* mats, int count,
-                          int prefetch, void* workspace, const GemvPlan& plan, cudaStream_t stream, bool fuse,
+                          int prefetch, void* workspace, const GemvPlan& plan, cudaStream_t stream, int epi,
                           const ArgmaxOut* am)
 {
     TmaMaps maps;
@@ -815,6 +899,9 @@ q4_status launch_gemv_tma(const void* x, q4_dtype xt, int64_t M, int64_t K, cons
     a.am_done = am ? am->done : nullptr;
     a.am_index = am ? am->index : nullptr;
     a.am_value = am ? am->value : nullptr;
+    a.tk_cand = am ? am->cand : nullptr;
+    a.tk_k = am ? am->k : 1;
+    a.row_base = am ? am->row_base : 0u;
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)plan.grid_x, (unsigned)plan.splits);
@@ -827,7 +914,6 @@ q4_status launch_gemv_tma(const void* x, q4_dtype xt, int64_t M, int64_t K, cons
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     void* args[] = {&maps, &a};
-    const int epi = fuse ? kEpiFuse : am ? kEpiArgmax : kEpiPlain;
     const cudaError_t e = cudaLaunchKernelExC(&cfg, kernel_for(mode_for(M, xt), epi), args);
     return e == cudaSuccess ? Q4_OK : Q4_ERR_CUDA;
 }

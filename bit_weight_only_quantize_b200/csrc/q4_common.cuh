@@ -49,22 +49,32 @@ q4_status launch_gemv(const void* x, q4_dtype xt, int64_t M, int64_t K, const q4
                       uint32_t flags, void* workspace, const GemvPlan& plan, cudaStream_t stream);
 
 bool tma_gemv_eligible(int64_t M, int64_t K, q4_dtype xt, const void* packed, const void* scales);
-// Greedy argmax outputs of a TMA GEMV launch over one matrix (see q4_gemv_argmax).
+// Row-block epilogues of the TMA GEMV.  Fuse: mats are gate and up of equal N and the
+// kernel writes silu(x.gate^T) * (x.up^T) into mats[0].y.  Argmax / top-k: one matrix
+// (mats[0].y may be null), greedy argmax or the k largest logits per x row.  Every
+// epilogue but the plain one needs whole sums, so K is never split for them.
+enum GemvEpilogue { kGemvPlain = 0, kGemvFuse = 1, kGemvArgmax = 2, kGemvTopk = 3 };
+
+// Argmax / top-k outputs of a TMA GEMV launch (see q4_gemv_argmax, q4_gemv_topk).
 struct ArgmaxOut {
-    unsigned long long* key;   // [M] workspace, zero at rest
-    unsigned* done;            // workspace, zero at rest
-    long long* index;          // [M]
-    float* value;              // [M] or null
+    unsigned long long* key;   // argmax: [M] workspace, zero at rest
+    unsigned* done;            // workspace block counter, zero at rest
+    long long* index;          // [M] (top-k: [M][k])
+    float* value;              // [M] (top-k: [M][k]) or null
+    unsigned long long* cand;  // top-k: [M][grid_x][k] workspace
+    int k;                     // top-k list length (1..32)
+    unsigned row_base;         // added to every reported row
 };
 
-// fuse: mats are gate and up of equal N; the kernel writes silu(x.gate^T) * (x.up^T) into
-// mats[0].y.  whole_k: K is never split (fused epilogues that need whole sums).
 bool plan_gemv_tma(int64_t M, const int64_t* Ns, int count, int64_t K, q4_dtype xt, const DeviceInfo& dev,
-                   GemvPlan* plan, bool fuse = false, bool whole_k = false);
-// am: non-null for a greedy argmax launch (count == 1; mats[0].y may be null).
+                   GemvPlan* plan, int epi = kGemvPlain);
+// am: non-null for an argmax or top-k launch.
 q4_status launch_gemv_tma(const void* x, q4_dtype xt, int64_t M, int64_t K, const q4_weight* mats, int count,
                           int prefetch, void* workspace, const GemvPlan& plan, cudaStream_t stream,
-                          bool fuse = false, const ArgmaxOut* am = nullptr);
+                          int epi = kGemvPlain, const ArgmaxOut* am = nullptr);
+
+q4_status launch_topk_merge(const float* values, const int64_t* indices, int64_t S, int64_t M, int64_t k,
+                            int64_t* out_index, float* out_value, cudaStream_t stream);
 
 q4_status launch_f16_gemv(const void* x, q4_dtype xt, int64_t M, int64_t K, const uint16_t* w, int64_t N, float* y,
                           int prefetch, cudaStream_t stream, const DeviceInfo& dev);

@@ -213,6 +213,53 @@ Q4_API q4_status q4_gemv_argmax(const void* x, q4_dtype x_dtype, int64_t M, int6
                                 uint32_t flags, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * q4_gemv_topk: the k largest logits of an LM head per x row in one launch: for each x
+ * row m, index[m][0..k-1] are the rows n of the k largest y[m, n] = x . dequant(W)^T (f32,
+ * as q4_gemv), larger value first, the lower n among equal values, a NaN logit above
+ * every number; value[m][i] = y[m, index[m][i]].  Rows are reported as row_base + n, so
+ * that an LM head split by rows across devices reports global rows.  When N < k the
+ * tail of each list holds index -1 and value NaN.
+ * The list is what a top-k sampler draws from (QORA-LLM-0.8B model card, section
+ * "Sampling Defaults": top_k 20); the logits need not leave the chip.  Shapes, dtypes and
+ * alignment as for q4_gemv_argmax.
+ *   k        1 .. Q4_TOPK_MAX.
+ *   row_base >= 0, with row_base + N <= 2^31 - 1 (Q4_ERR_SHAPE otherwise).
+ *   y        device f32 [M,N] or NULL: when given, the logits are written too.
+ *   index    device int64 [M,k], 8-byte aligned (output).
+ *   value    device f32 [M,k] or NULL (output).
+ *   workspace  device, at least q4_gemv_topk_workspace_size(M, N, K, k, x_dtype) bytes
+ *            (0 when the shape is not served or no device is current), 16-byte aligned;
+ *            its first 16 bytes must be zero before the first call and every call leaves
+ *            them zero again (one workspace per stream, as for q4_gemv_argmax).
+ * K is never split.  M == 0 or N == 0 is a no-op (nothing is written).
+ */
+#define Q4_TOPK_MAX 32
+Q4_API size_t q4_gemv_topk_workspace_size(int64_t M, int64_t N, int64_t K, int64_t k, q4_dtype x_dtype);
+Q4_API q4_status q4_gemv_topk(const void* x, q4_dtype x_dtype, int64_t M, int64_t K, const uint8_t* packed,
+                              const uint16_t* scales, int64_t N, int64_t k, int64_t row_base, float* y,
+                              int64_t* index, float* value, uint32_t flags, void* workspace,
+                              size_t workspace_bytes, void* stream);
+
+/*
+ * q4_topk_merge: the k best entries per x row over S top-k lists, ordered as q4_gemv_topk
+ * orders them (larger value first, the lower row among equal values, a NaN above every
+ * number).  With an LM head split by rows across S devices, each device runs
+ * q4_gemv_topk on its rows with row_base = its first row, the [M,k] lists are gathered
+ * (S * M * k entries, the only exchange), and this call selects the global top k
+ * (QORA-LLM-0.8B model card, section "Sampling Defaults": top_k 20; QORA-4B thread,
+ * section "量化与内存管理": the LM head among the parallel workloads).
+ *   values   device f32 [S,M,k], 4-byte aligned; indices device int64 [S,M,k], 8-byte
+ *            aligned: list s of x row m at [s,m,:].  An index outside [0, 2^31 - 1)
+ *            (such as the -1 of a short list) marks padding and is skipped.  Rows must be
+ *            distinct across the lists of one x row (disjoint shards).
+ *   S        1 .. 2^20 lists;  M >= 0 x rows (0: no-op);  k 1 .. Q4_TOPK_MAX.
+ *   index    device int64 [M,k], 8-byte aligned (output); value f32 [M,k] or NULL.
+ * When fewer than k entries exist the tail holds index -1 and value NaN.
+ */
+Q4_API q4_status q4_topk_merge(const float* values, const int64_t* indices, int64_t S, int64_t M, int64_t k,
+                               int64_t* index, float* value, void* stream);
+
+/*
  * q4_f16_gemv: y[M,N] = x[M,K] . W^T for binary16 weights W (2 bytes per weight), the
  * pages' second weight format (QORA-LLM-0.8B model card, section "AVX-512 SIMD
  * Acceleration": "F16 GEMV").  Same roles as q4_gemv, without quantisation:

@@ -158,6 +158,50 @@ def test_argmax_validation(lib):
     assert f(None, 1, 0, 256, None, None, 8, None, None, None, 0, None, 0, S) == 0  # M == 0: no-op
 
 
+def test_topk_validation(lib):
+    S = None
+    f = lib.q4_gemv_topk
+    W = 1 << 20
+    ok = dict(x=A16, t=1, M=1, K=256, p=A16, s=A16, N=8, k=20, rb=0, y=None, i=A16, v=None, fl=0, ws=A16, wb=W)
+
+    def call(**kw):
+        a = {**ok, **kw}
+        return f(a["x"], a["t"], a["M"], a["K"], a["p"], a["s"], a["N"], a["k"], a["rb"], a["y"], a["i"], a["v"],
+                 a["fl"], a["ws"], a["wb"], S)
+    assert call(t=7) == 4                                   # dtype
+    assert call(M=17) == 2                                  # M > 16
+    assert call(k=0) == 2 and call(k=33) == 2               # k in 1..32
+    assert call(rb=-1) == 2                                 # row_base >= 0
+    assert call(rb=(1 << 31) - 8) == 2                      # row_base + N past 2^31 - 1
+    assert call(fl=2) == 1                                  # unknown flag
+    assert call(i=None) == 1                                # index required
+    assert call(ws=None, wb=0) == 5                         # workspace required
+    assert call(i=A16 + 4) == 3                             # index alignment
+    assert call(s=A8) == 3                                  # scales: 16 bytes
+    assert call(v=A16 + 2) == 3                             # value alignment
+    assert call(K=96) == 2                                  # K % 256
+    assert call(t=0, M=2) == 2                              # f32 x only with M == 1
+    assert call(x=None, M=0, p=None, s=None, i=None, ws=None, wb=0) == 0   # M == 0: no-op
+    assert call(x=None, N=0, p=None, s=None, i=None, ws=None, wb=0) == 0   # N == 0: no-op
+    assert lib.q4_gemv_topk_workspace_size(1, 8, 96, 20, 1) == 0          # K % 256: not served
+    assert lib.q4_gemv_topk_workspace_size(1, 8, 256, 33, 1) == 0         # k > 32
+
+
+def test_topk_merge_validation(lib):
+    f = lib.q4_topk_merge
+    assert f(A16, A16, 0, 1, 20, A16, None, None) == 2              # S >= 1
+    assert f(A16, A16, 1 << 21, 1, 20, A16, None, None) == 2        # S <= 2^20
+    assert f(A16, A16, 2, 1, 0, A16, None, None) == 2               # k >= 1
+    assert f(A16, A16, 2, 1, 33, A16, None, None) == 2              # k <= 32
+    assert f(A16, A16, 2, -1, 20, A16, None, None) == 2             # M >= 0
+    assert f(None, A16, 2, 1, 20, A16, None, None) == 1             # values required
+    assert f(A16, A16, 2, 1, 20, None, None, None) == 1             # index required
+    assert f(A16 + 2, A16, 2, 1, 20, A16, None, None) == 3          # values alignment
+    assert f(A16, A16 + 4, 2, 1, 20, A16, None, None) == 3          # indices alignment
+    assert f(A16, A16, 2, 1, 20, A16, A16 + 2, None) == 3           # value alignment
+    assert f(None, None, 2, 0, 20, None, None, None) == 0           # M == 0: no-op
+
+
 def test_f16_gemv_validation(lib):
     S = None
     f = lib.q4_f16_gemv
