@@ -307,17 +307,18 @@ def measure_e2e(torch, q4, step, steps, device, dist=None, world=1):
     n = max(1, min(steps, 2000))
     x_host = torch.from_numpy(step.x_np.view(np.int16)).view(torch.bfloat16).pin_memory()
     y_host = torch.empty(step.y_all.shape, dtype=step.y_all.dtype).pin_memory()
-    x_dev = torch.empty_like(step.x)
     stream = torch.cuda.current_stream(device)
     # one prepared call per weight copy: the weights are checked once, each step checks x
     calls = [q4.GemvMulti([(step.pk[j][c], step.sc[j][c]) for j in range(len(step.mats))], 1, step.x.shape[1],
                           step.x.dtype, outs=step.y, workspace=step.ws, weights_static=True)
              for c in range(step.copies)]
 
+    # each step: one graph (pinned x -> device, the GEMVs, all outputs -> pinned host), then
+    # the host waits for it
+    host_steps = [c.host_step(x_host, y_host, y_dev=step.y_all) for c in calls]
+
     def one(i):
-        x_dev.copy_(x_host, non_blocking=True)
-        calls[i % step.copies](x_dev)
-        y_host.copy_(step.y_all, non_blocking=True)
+        host_steps[i % step.copies]()
         stream.synchronize()
 
     for i in range(3):
@@ -334,8 +335,8 @@ def measure_e2e(torch, q4, step, steps, device, dist=None, world=1):
             "h2d_bytes_per_step": x_host.numel() * 2,
             "d2h_bytes_per_step": y_host.numel() * 4,
             "steps": n, "ms_per_step": ms,
-            "api": "bit_weight_only_quantize_b200.GemvMulti (prepared gemv_multi), pinned host x in, host y out, "
-                   "sync per step"}
+            "api": "bit_weight_only_quantize_b200.GemvMulti.host_step (graph: pinned host x in, gemv_multi, "
+                   "host y out), sync per step"}
 
 
 def time_launches(torch, fn, n, device, stream):

@@ -400,6 +400,45 @@ class GemvMulti:
         _lib.check(st, "q4_gemv_multi")
         return self.outs
 
+    def host_step(self, x_host: torch.Tensor, y_host, y_dev: torch.Tensor | None = None):
+        """One decode step fed from pinned host memory, captured as a CUDA graph: x_host ->
+        device, the GEMVs, the outputs -> pinned host memory.  ``y_host`` is a list of
+        pinned tensors, one per output, or, with ``y_dev`` (a device tensor whose storage
+        holds every output), one pinned tensor of y_dev's shape that receives it in one
+        copy.  Returns a callable that replays the step on the current stream; the caller
+        synchronizes before reading y_host.  The host tensors are held by reference."""
+        if not (x_host.is_pinned() and x_host.dtype is self._dtype and tuple(x_host.shape) == self._shape):
+            raise ValueError(f"x_host must be a pinned {self._dtype} tensor of shape {self._shape}")
+        if y_dev is not None:
+            if not (isinstance(y_host, torch.Tensor) and y_host.is_pinned() and y_host.shape == y_dev.shape
+                    and y_host.dtype is y_dev.dtype and y_dev.device == self.device):
+                raise ValueError("y_host must be a pinned tensor shaped like y_dev")
+            base, end = y_dev.data_ptr(), y_dev.data_ptr() + y_dev.numel() * y_dev.element_size()
+            if any(not base <= o.data_ptr() < end for o in self.outs):
+                raise ValueError("every output must lie in y_dev")
+            pairs = [(y_host, y_dev)]
+        else:
+            if len(y_host) != len(self.outs) or any(not (h.is_pinned() and h.shape == o.shape and h.dtype is o.dtype)
+                                                    for h, o in zip(y_host, self.outs)):
+                raise ValueError("y_host must hold one pinned tensor per output, shaped like it")
+            pairs = list(zip(y_host, self.outs))
+        x_dev = torch.empty(self._shape, dtype=self._dtype, device=self.device)
+        graph = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(device=self.device)
+        with _on(self.device), torch.cuda.stream(side):
+            self(x_dev)                                   # the launch works before it is captured
+            side.synchronize()
+            with torch.cuda.graph(graph, stream=side):
+                x_dev.copy_(x_host, non_blocking=True)
+                self(x_dev)
+                for h, d in pairs:
+                    h.copy_(d, non_blocking=True)
+        keep = (x_host, y_host, x_dev, graph)
+
+        def replay():
+            keep[3].replay()
+        return replay
+
 
 def gemm(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
     """y[M,N] (bf16) = x[M,K] (bf16) . dequant(W)^T on the tensor cores (prefill)."""

@@ -642,27 +642,34 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
 
     if constexpr (kTopk) {
         // Every team is past its last row block, so the code rings are free: each team
-        // leader parks its lists in its own warp's ring, then warp m merges the teams'
-        // lists of x row m into this block's list.
+        // leader parks its 32-key list of every x row in its own warp's ring (a team that
+        // gave up parks empty lists), then a tree of warp merges reduces the teams' lists
+        // of each x row to one, and the block writes its first k keys to the workspace.
         const int kk = a.tk_k;
         constexpr int kRingWords = kStages * kStageCodes / 8;          // u64 per warp ring
         unsigned long long* lists = reinterpret_cast<unsigned long long*>(codes);
+        const size_t team_stride = (size_t)P * kRingWords;            // list of team t: t * team_stride
         __syncthreads();
         if (active && wt == 0) {
 #pragma unroll
             for (int mm = 0; mm < kTkM; ++mm)
-                if (mm < a.M && lane < kk) lists[(size_t)warp * kRingWords + mm * kk + lane] = tk[mm];
-            if (lane == 0) s_last[team] = ok;
+                if (mm < a.M) lists[(size_t)warp * kRingWords + mm * 32 + lane] = ok ? tk[mm] : 0ull;
         }
         __syncthreads();
-        for (int m = warp; m < a.M; m += W) {
-            unsigned long long list = 0ull;
-            for (int t = 0; t < a.teams; ++t) {
-                if (!s_last[t]) continue;                               // a team that gave up
-                const unsigned long long c = lane < kk ? lists[(size_t)t * P * kRingWords + m * kk + lane] : 0ull;
-                topk_insert(list, c, true, kk, lane);
+        for (int step = 1; step < a.teams; step <<= 1) {               // merge team i + step into team i
+            const int pairs = (a.teams + 2 * step - 1) / (2 * step);
+            for (int job = warp; job < a.M * pairs; job += W) {
+                const int m = job / pairs, t = (job - m * pairs) * 2 * step;
+                if (t + step < a.teams) {
+                    unsigned long long* dst = lists + (size_t)t * team_stride + m * 32;
+                    const unsigned long long* src = lists + (size_t)(t + step) * team_stride + m * 32;
+                    dst[lane] = warp_merge_desc(dst[lane], src[lane], lane);
+                }
             }
-            if (lane < kk) a.tk_cand[((size_t)m * gridDim.x + blockIdx.x) * kk + lane] = list;
+            __syncthreads();
+        }
+        for (int m = warp; m < a.M; m += W) {
+            if (lane < kk) a.tk_cand[((size_t)m * gridDim.x + blockIdx.x) * kk + lane] = lists[m * 32 + lane];
             __threadfence();
         }
         __syncthreads();
@@ -672,32 +679,36 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
         }
         __syncthreads();
         if (s_last[0]) {
-            // The last block: S warps per x row each merge a slice of the blocks' lists,
-            // then warp m merges the S slice lists of x row m and writes the result.
+            // The last block: S warps per x row each merge the lists of every S-th block
+            // (k keys each, padded with 0 to 32 lanes), then a tree of warp merges reduces
+            // the S slice lists of each x row to the result.
             __threadfence();
             const int S = max(1, W / a.M);
-            const int len = gridDim.x * kk;                              // candidates per x row
             for (int job = warp; job < a.M * S; job += W) {
                 const int m = job / S, sl = job - m * S;
-                const int lo = sl * len / S, hi = (sl + 1) * len / S;
-                const unsigned long long* src = a.tk_cand + (size_t)m * len;
+                const unsigned long long* src = a.tk_cand + (size_t)m * gridDim.x * kk;
                 unsigned long long list = 0ull;
-                for (int i0 = lo; i0 < hi; i0 += 32) {
-                    const unsigned long long c = i0 + lane < hi ? __ldcg(src + i0 + lane) : 0ull;
-                    topk_insert(list, c, true, kk, lane);
-                }
-                if (lane < kk) lists[(size_t)job * kk + lane] = list;
+                for (int b = sl; b < (int)gridDim.x; b += S)
+                    list = warp_merge_desc(list, lane < kk ? __ldcg(src + (size_t)b * kk + lane) : 0ull, lane);
+                lists[(size_t)job * 32 + lane] = list;
             }
             __syncthreads();
-            for (int m = warp; m < a.M; m += W) {
-                unsigned long long list = 0ull;
-                for (int i0 = 0; i0 < S * kk; i0 += 32) {
-                    const int i = i0 + lane;
-                    topk_insert(list, i < S * kk ? lists[(size_t)m * S * kk + i] : 0ull, true, kk, lane);
+            for (int step = 1; step < S; step <<= 1) {
+                const int pairs = (S + 2 * step - 1) / (2 * step);
+                for (int job = warp; job < a.M * pairs; job += W) {
+                    const int m = job / pairs, i = (job - m * pairs) * 2 * step;
+                    if (i + step < S) {
+                        unsigned long long* dst = lists + ((size_t)m * S + i) * 32;
+                        dst[lane] = warp_merge_desc(dst[lane], dst[(size_t)step * 32 + lane], lane);
+                    }
                 }
+                __syncthreads();
+            }
+            for (int m = warp; m < a.M; m += W) {
+                const unsigned long long key = lists[(size_t)m * S * 32 + lane];
                 if (lane < kk) {
-                    a.am_index[(size_t)m * kk + lane] = list ? (long long)(0xFFFFFFFFu - (uint32_t)list) : -1;
-                    if (a.am_value) a.am_value[(size_t)m * kk + lane] = list ? argmax_value(list) : __int_as_float(0x7FC00000);
+                    a.am_index[(size_t)m * kk + lane] = key ? (long long)(0xFFFFFFFFu - (uint32_t)key) : -1;
+                    if (a.am_value) a.am_value[(size_t)m * kk + lane] = key ? argmax_value(key) : __int_as_float(0x7FC00000);
                 }
             }
             if (threadIdx.x == 0) *a.am_done = 0u;

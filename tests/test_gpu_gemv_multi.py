@@ -112,3 +112,39 @@ def test_prepared_call_matches_gemv_multi(M, x_dtype):
         plan(to_dev_x(synth_inputs.activations(M + 1, K, x_dtype, seed=3)))      # wrong shape
     with pytest.raises(TypeError):
         plan(torch.zeros((M, K), dtype=torch.float16, device="cuda"))            # wrong dtype
+
+
+@pytest.mark.parametrize("M,x_dtype,shared", [(1, "bf16", True), (1, "f32", False), (4, "bf16", False)])
+def test_host_step_graph_matches_oracle(M, x_dtype, shared):
+    """GemvMulti.host_step: pinned x in, the GEMVs, outputs to pinned host memory, as one
+    graph; replayed with new host inputs it gives the prepared call's bits each time."""
+    import bit_weight_only_quantize_b200 as q4
+    Ns, K = [2048, 4096, 1024], 2560
+    mats = _prep(Ns, K, seed=31)
+    dm = _dev(mats)
+    dt = torch.float32 if x_dtype == "f32" else torch.bfloat16
+    if shared:                                        # M == 1: outputs are views of one buffer
+        y_dev = torch.empty((M, sum(Ns)), dtype=torch.float32, device="cuda")
+        outs = [y_dev[:, a:a + n] for a, n in zip(np.cumsum([0] + Ns[:-1]).tolist(), Ns)]
+    else:
+        y_dev, outs = None, None
+    plan = q4.GemvMulti(dm, M, K, dt, outs=outs, weights_static=True)
+    x_host = torch.empty((M, K), dtype=dt).pin_memory()
+    if shared:
+        y_host = torch.empty_like(y_dev, device="cpu").pin_memory()
+    else:
+        y_host = [torch.empty((M, n), dtype=torch.float32).pin_memory() for n in Ns]
+    step = plan.host_step(x_host, y_host, y_dev=y_dev)
+    for seed in (4, 5):
+        x = synth_inputs.activations(M, K, x_dtype, seed=seed)
+        x_host.copy_(torch.from_numpy(x.view(np.int16)).view(torch.bfloat16) if x_dtype == "bf16"
+                     else torch.from_numpy(x))
+        step()
+        torch.cuda.synchronize()
+        got = torch.split(y_host, Ns, dim=1) if shared else y_host
+        ref = q4.gemv_multi(to_dev_x(x), dm)
+        for g, r, (p, s) in zip(got, ref, mats):
+            assert torch.equal(g, r.cpu())
+            assert rel_inf(g.numpy(), oracle.matmul(x, p, s, threads=8)) <= (2e-3 if x_dtype == "f32" else 1e-2)
+    with pytest.raises(ValueError):
+        plan.host_step(torch.empty((M, K), dtype=dt), y_host, y_dev=y_dev)        # x not pinned
