@@ -263,13 +263,16 @@ q4_status q4_gemv_argmax(const void* x, q4_dtype x_dtype, int64_t M, int64_t K, 
     am.index = reinterpret_cast<long long*>(index);
     am.value = value;
     am.cand = nullptr;
+    am.floor = nullptr;
     am.k = 1;
     am.row_base = 0u;
     return q4::launch_gemv_tma(x, x_dtype, M, K, &w, 1, (flags & Q4_WEIGHTS_STATIC) ? 1 : 0, nullptr, plan,
                                static_cast<cudaStream_t>(stream), q4::kGemvArgmax, &am);
 }
 
-// Top-k workspace: the block counter, then the blocks' lists [M][grid_x][k].
+// Top-k workspace: the block counter at 0, the published k-th key at 8 (both zero at
+// rest), then from byte 256 the blocks' lists [M][grid_x][k].
+static constexpr size_t kTopkFloorOffset = 8;
 static constexpr size_t kTopkListsOffset = 256;
 
 static bool topk_shape(int64_t M, int64_t N, int64_t K, int64_t k, q4_dtype x_dtype)
@@ -324,6 +327,7 @@ q4_status q4_gemv_topk(const void* x, q4_dtype x_dtype, int64_t M, int64_t K, co
     am.index = reinterpret_cast<long long*>(index);
     am.value = value;
     am.cand = reinterpret_cast<unsigned long long*>(static_cast<char*>(workspace) + kTopkListsOffset);
+    am.floor = reinterpret_cast<unsigned long long*>(static_cast<char*>(workspace) + kTopkFloorOffset);
     am.k = (int)k;
     am.row_base = (unsigned)row_base;
     return q4::launch_gemv_tma(x, x_dtype, M, K, &w, 1, (flags & Q4_WEIGHTS_STATIC) ? 1 : 0, nullptr, plan,

@@ -94,6 +94,7 @@ struct TmaGemvArgs {
     long long* am_index;              // [M] output ([M][k] for top-k)
     float* am_value;                  // [M] output ([M][k]), may be null
     unsigned long long* tk_cand;      // top-k: per-block lists
+    unsigned long long* tk_floor;     // top-k, M == 1: the largest k-th key any team has published
     int tk_k;                         // top-k: list length, 1..32
     unsigned row_base;                // argmax / top-k: added to every reported row
 };
@@ -411,8 +412,14 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
     unsigned long long tk[kTopk ? kTkM + 1 : 1];           // top-k: the team's list per x row
 #pragma unroll
     for (int i = 0; i < (kTopk ? kTkM + 1 : 1); ++i) tk[i] = 0ull;
+    // Top-k with one x row: every team's k-th key is at most the whole head's k-th largest,
+    // so the largest one published so far (tk_floor) is a bar no row below it can pass.
+    // A team reads it when it starts a row block and publishes its own when it rises.
+    constexpr bool kFloor = kTopk && kTkM == 1;
+    unsigned long long floor_now = 0ull, floor_pub = 0ull;
     for (int rbi = 0; rbi < nrb; ++rbi) {
         const int rb = rb_of(rbi);
+        if constexpr (kFloor) floor_now = load_key_relaxed(a.tk_floor);   // used in this block's epilogue
         float yacc = 0.f;     // kF32M1: row (lane & 15), half (lane >> 4)
         float acc[NT][4];     // MMA modes: rows g, g+8; x rows n*8 + 2t, +1
 #pragma unroll
@@ -575,7 +582,14 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
                 for (int h = 0; h < (kTkM + 1) / 2; ++h) {
                     if (h * 32 < kRows * a.M) {
                         const unsigned long long key = rows_out(h * 32);
-                        topk_insert(tk[2 * h], key, lane < 16, a.tk_k, lane);
+                        topk_insert(tk[2 * h], key, lane < 16, a.tk_k, lane, kFloor ? floor_now : 0ull);
+                        if constexpr (kFloor) {
+                            const unsigned long long kth = __shfl_sync(0xffffffffu, tk[0], a.tk_k - 1);
+                            if (kth > floor_pub && kth > floor_now) {       // the same on every lane
+                                if (lane == 0) atomicMax(a.tk_floor, kth);
+                                floor_pub = kth;
+                            }
+                        }
                         if (2 * h + 1 < kTkM) topk_insert(tk[2 * h + 1], key, lane >= 16, a.tk_k, lane);
                     }
                 }
@@ -687,9 +701,24 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
             for (int job = warp; job < a.M * S; job += W) {
                 const int m = job / S, sl = job - m * S;
                 const unsigned long long* src = a.tk_cand + (size_t)m * gridDim.x * kk;
+                // the lists of blocks sl, sl + S, ...: four loads in flight ahead of the merges
+                auto fetch = [&](int b) {
+                    return (b < (int)gridDim.x && lane < kk) ? __ldcg(src + (size_t)b * kk + lane) : 0ull;
+                };
+                unsigned long long nxt[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) nxt[q] = fetch(sl + q * S);
                 unsigned long long list = 0ull;
-                for (int b = sl; b < (int)gridDim.x; b += S)
-                    list = warp_merge_desc(list, lane < kk ? __ldcg(src + (size_t)b * kk + lane) : 0ull, lane);
+                for (int b0 = sl; b0 < (int)gridDim.x; b0 += 4 * S) {
+                    unsigned long long cur[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        cur[q] = nxt[q];
+                        nxt[q] = fetch(b0 + (4 + q) * S);
+                    }
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) list = warp_merge_desc(list, cur[q], lane);
+                }
                 lists[(size_t)job * 32 + lane] = list;
             }
             __syncthreads();
@@ -711,7 +740,10 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
                     if (a.am_value) a.am_value[(size_t)m * kk + lane] = key ? argmax_value(key) : __int_as_float(0x7FC00000);
                 }
             }
-            if (threadIdx.x == 0) *a.am_done = 0u;
+            if (threadIdx.x == 0) {
+                *a.am_done = 0u;
+                if (a.tk_floor) *a.tk_floor = 0ull;
+            }
         }
     }
 }
@@ -911,6 +943,7 @@ q4_status launch_gemv_tma(const void* x, q4_dtype xt, int64_t M, int64_t K, cons
     a.am_index = am ? am->index : nullptr;
     a.am_value = am ? am->value : nullptr;
     a.tk_cand = am ? am->cand : nullptr;
+    a.tk_floor = am ? am->floor : nullptr;
     a.tk_k = am ? am->k : 1;
     a.row_base = am ? am->row_base : 0u;
 

@@ -62,6 +62,7 @@ struct ArgmaxOut {
     long long* index;          // [M] (top-k: [M][k])
     float* value;              // [M] (top-k: [M][k]) or null
     unsigned long long* cand;  // top-k: [M][grid_x][k] workspace
+    unsigned long long* floor; // top-k: one key of workspace, zero at rest
     int k;                     // top-k list length (1..32)
     unsigned row_base;         // added to every reported row
 };

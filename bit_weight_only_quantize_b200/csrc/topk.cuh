@@ -23,6 +23,15 @@ __device__ __forceinline__ float argmax_value(unsigned long long key)
     return __uint_as_float((ord & 0x80000000u) ? (ord & 0x7FFFFFFFu) : ~ord);
 }
 
+// A relaxed load of a key other blocks raise with atomicMax (always a valid lower bound,
+// however stale).
+__device__ __forceinline__ unsigned long long load_key_relaxed(const unsigned long long* p)
+{
+    unsigned long long v;
+    asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
 __device__ __forceinline__ unsigned long long key_max(unsigned long long a, unsigned long long b)
 {
     return a > b ? a : b;
@@ -76,10 +85,11 @@ constexpr int kSortInsert = 4;
 // kk largest keys seen; a key that does not beat the kk-th entry cannot enter them and is
 // skipped.  Few candidates are inserted one at a time (the list shifts down one lane from
 // the insertion point), many are sorted and merged.
+// `floor` is a key no candidate needs to beat, as well as the list's k-th entry (0: none).
 __device__ __forceinline__ void topk_insert(unsigned long long& list, unsigned long long key, bool mine, int kk,
-                                            int lane)
+                                            int lane, unsigned long long floor = 0ull)
 {
-    const unsigned long long last = __shfl_sync(0xffffffffu, list, kk - 1);
+    const unsigned long long last = key_max(__shfl_sync(0xffffffffu, list, kk - 1), floor);
     const bool want = mine && key > last;
     unsigned mask = __ballot_sync(0xffffffffu, want);
     if (__popc(mask) > kSortInsert) {               // the same on every lane
@@ -90,7 +100,7 @@ __device__ __forceinline__ void topk_insert(unsigned long long& list, unsigned l
         const int src = __ffs(mask) - 1;
         mask &= mask - 1;
         const unsigned long long c = __shfl_sync(0xffffffffu, key, src);
-        const unsigned long long now_last = __shfl_sync(0xffffffffu, list, kk - 1);
+        const unsigned long long now_last = key_max(__shfl_sync(0xffffffffu, list, kk - 1), floor);
         if (c > now_last) {
             const int pos = __popc(__ballot_sync(0xffffffffu, list > c));   // entries above c
             const unsigned long long up = __shfl_up_sync(0xffffffffu, list, 1);
