@@ -30,7 +30,7 @@ def _rank(rank, world, port, times, out):
 @pytest.mark.parametrize("world", [2, 3])
 def test_ranks_agree_on_the_slowest_time(world):
     times = [1.5, 4.25, 2.0][:world]
-    out = mp.Manager().dict()
+    out = mp.get_context("spawn").Manager().dict()
     mp.spawn(_rank, args=(world, _free_port(), times, out), nprocs=world, join=True)
     assert [out[r] for r in range(world)] == [max(times)] * world
 

@@ -60,7 +60,7 @@ def _rank(rank, world, port, N, K, k, out):
 @pytest.mark.parametrize("world,N,k", [(2, 1000, 20), (3, 70, 32), (4, 40, 20)])
 def test_merged_shard_lists_are_the_global_topk(world, N, k):
     K = 256
-    out = mp.Manager().dict()
+    out = mp.get_context("spawn").Manager().dict()
     mp.spawn(_rank, args=(world, _free_port(), N, K, k, out), nprocs=world, join=True)
     packed, scales, _ = oracle.quantize(synth_inputs.weights("outliers", N, K, seed=3))
     x = synth_inputs.activations(2, K, "bf16", seed=4)
