@@ -375,15 +375,26 @@ def measure_rows(torch, q4, lib, device, peaks, l2):
     ws_n = q4.gemv_workspace_size(1, w.N, w.K)
     ws = torch.zeros(max(ws_n, 16), dtype=torch.uint8, device=device)
 
-    def lm(i):
+    def lm_plain(i):
         st = lib.q4_gemv(x.data_ptr(), 1, 1, w.K, packed.data_ptr(), scales.data_ptr(), w.N, y.data_ptr(),
                          ws.data_ptr(), ws.numel(), stream.cuda_stream)
         assert st == 0
     log("rows: lm head")
-    ms = time_launches(torch, lm, 20, device, stream)
     b = gemv_bytes(1, w.N, w.K)
-    out["lm_head_gemv"] = {"workload": "M=1 K=2560 N=248320 bf16 x", "ms": ms, "GB/s": b / ms / 1e6,
-                           "frac_hbm": b / ms / 1e6 / hbm, "bytes": b, "launches": 20}
+    ms = time_launches(torch, lm_plain, 20, device, stream)
+    out["lm_head_gemv_no_prefetch"] = {"workload": "M=1 K=2560 N=248320 bf16 x, q4_gemv (no static-weights flag)",
+                                       "ms": ms, "GB/s": b / ms / 1e6, "frac_hbm": b / ms / 1e6 / hbm, "bytes": b,
+                                       "launches": 20}
+    # The LM head's weights are static, as the decode step's are: with the flag a launch
+    # streams its weights before waiting for its predecessor (the argmax and top-k rows
+    # below use it too).
+    lm_call = q4.GemvMulti([(packed, scales)], 1, w.K, torch.bfloat16, outs=[y], workspace=ws, weights_static=True)
+
+    def lm(i):
+        lm_call(x)
+    ms = time_launches(torch, lm, 20, device, stream)
+    out["lm_head_gemv"] = {"workload": "M=1 K=2560 N=248320 bf16 x, static weights (q4_gemv_multi)", "ms": ms,
+                           "GB/s": b / ms / 1e6, "frac_hbm": b / ms / 1e6 / hbm, "bytes": b, "launches": 20}
 
     # Greedy LM-head step: the same GEMV with the argmax fused, logits kept on chip.
     am_ws = torch.zeros(int(lib.q4_gemv_argmax_workspace_size()), dtype=torch.uint8, device=device)
