@@ -69,6 +69,10 @@ def _load():
         lib.oracle_q4_gate_up_rows.restype = i32
         lib.oracle_f16_matmul.argtypes = [vp, i32, i64, i64, vp, i64, vp, i32]
         lib.oracle_f16_matmul.restype = i32
+        lib.oracle_q8_quantize.argtypes = [vp, i64, i64, vp, vp, vp]
+        lib.oracle_q8_quantize.restype = i32
+        lib.oracle_q8_matmul.argtypes = [vp, i32, i64, i64, vp, vp, i64, vp, i32]
+        lib.oracle_q8_matmul.restype = i32
         lib.oracle_max_threads.argtypes = []
         lib.oracle_max_threads.restype = i32
         _lib = lib
@@ -264,6 +268,50 @@ def f16_matmul(x: np.ndarray, w16: np.ndarray, threads: int = 1) -> np.ndarray:
         raise ValueError("shape mismatch between x and w16")
     y = np.empty((M, N), dtype=np.float64)
     _load().oracle_f16_matmul(_ptr(x), is_bf16, M, K, _ptr(w16), N, _ptr(y), threads)
+    return y
+
+
+def quantize8(W: np.ndarray):
+    """INT8 weights, the other half of a mixed INT8/INT4 model (QKV-Core thread, section
+    "自适应混合量化"): W f32 [N,K] -> (codes int8 [N,K], scales uint16 binary16 bits
+    [N,K/32], flags).  The encoding is written out in ``q4_oracle.c``."""
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    if W.ndim != 2 or W.shape[1] % 32 != 0:
+        raise ValueError("W must be [N, K] with K a multiple of 32")
+    N, K = W.shape
+    codes = np.empty((N, K), dtype=np.int8)
+    scales = np.empty((N, K // 32), dtype=np.uint16)
+    flags = ctypes.c_uint32(0)
+    if _load().oracle_q8_quantize(_ptr(W), N, K, _ptr(codes), _ptr(scales), ctypes.addressof(flags)) != 0:
+        raise ValueError("oracle_q8_quantize rejected the shape")
+    return codes, scales, int(flags.value)
+
+
+def dequantize8(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """Exact binary64 INT8 dequantised weights [N,K]: code * f32(scale)."""
+    s = f16_bits_to_f32(scales).astype(np.float64)
+    return codes.astype(np.float64) * np.repeat(s, 32, axis=1)
+
+
+def matmul8(x: np.ndarray, codes: np.ndarray, scales: np.ndarray, threads: int = 1) -> np.ndarray:
+    """y = x . dequant8(W)^T in binary64; x as for ``matmul``."""
+    if x.dtype == np.uint16:
+        is_bf16 = 1
+    elif x.dtype == np.float32:
+        is_bf16 = 0
+    else:
+        raise TypeError("x must be float32 or uint16 (bfloat16 bits)")
+    x = np.ascontiguousarray(x)
+    if x.ndim == 1:
+        x = x[None, :]
+    codes = np.ascontiguousarray(codes, dtype=np.int8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint16)
+    M, K = x.shape
+    N = codes.shape[0]
+    if codes.shape != (N, K) or scales.shape != (N, K // 32):
+        raise ValueError("shape mismatch between x, codes and scales")
+    y = np.empty((M, N), dtype=np.float64)
+    _load().oracle_q8_matmul(_ptr(x), is_bf16, M, K, _ptr(codes), _ptr(scales), N, _ptr(y), threads)
     return y
 
 

@@ -302,6 +302,96 @@ int oracle_f16_matmul(const void* x, int x_is_bf16, int64_t M, int64_t K, const 
     return 0;
 }
 
+/* ---- INT8 weights: the second half of a mixed INT8/INT4 model ----
+ * The QKV-Core thread (zingnex.cn, section "自适应混合量化") quantises per layer: layers
+ * that are sensitive to precision (attention) in INT8, the feed-forward layers in INT4.
+ * It gives no encoding.  The reading taken here is the Q4 format above with 8-bit codes:
+ *
+ *   s32 = amax / 127                                  (f32, round-to-nearest-even)
+ *   s   = binary16(s32)                               (round-to-nearest-even)
+ *   s == 0            -> every code 0, scale bits 0x0000
+ *   otherwise q_j     = clamp(rint(w_j / f32(s)), -128, 127)   (f32 division, ties to even)
+ *   stored byte k     = q_k as a two's-complement int8, codes [N, K] row-major
+ *   dequantised w'_j  = q_j * f32(s)
+ *
+ * The divisor is the largest positive code and the clamp is the whole code range, as
+ * 7 and [-8, 7] are for Q4: -128 is reached only when rounding the scale to binary16
+ * lowers it by more than half a code (subnormal scales).  Non-finite input and scale
+ * overflow give a zero group and the same flag bits as Q4. */
+static uint32_t quantize_group_q8(const float* w, int8_t* codes, uint16_t* scale)
+{
+    int nonfinite = 0;
+    float amax = 0.0f;
+    for (int j = 0; j < 32; ++j) {
+        if (!isfinite(w[j])) nonfinite = 1;
+        float a = fabsf(w[j]);
+        if (a > amax) amax = a;
+    }
+    uint32_t flag = 0;
+    uint16_t sbits = 0;
+    if (nonfinite) {
+        flag = ORACLE_FLAG_NONFINITE;
+    } else {
+        volatile float s32 = amax / 127.0f;   /* one IEEE f32 division */
+        sbits = oracle_f32_to_f16(s32);
+        if ((sbits & 0x7FFFu) == 0x7C00u) flag = ORACLE_FLAG_SCALE_OVERFLOW;
+    }
+    if (flag || (sbits & 0x7FFFu) == 0) {
+        for (int j = 0; j < 32; ++j) codes[j] = 0;
+        *scale = 0;
+        return flag;
+    }
+    float sf = oracle_f16_to_f32(sbits);
+    for (int j = 0; j < 32; ++j) {
+        volatile float t = w[j] / sf;         /* f32 quotient by the stored scale */
+        int q = (int)nearbyintf(t);           /* current mode: to nearest, ties to even */
+        if (q < -128) q = -128;
+        if (q > 127) q = 127;
+        codes[j] = (int8_t)q;
+    }
+    *scale = sbits;
+    return 0;
+}
+
+/* W: f32 [N,K] row-major; codes: int8 [N,K]; scales: binary16 bits [N,K/32].
+ * Returns -1 if K is not a multiple of 32, else 0.  *flags gets the OR of all groups' flags. */
+int oracle_q8_quantize(const float* W, int64_t N, int64_t K, int8_t* codes, uint16_t* scales, uint32_t* flags)
+{
+    if (K % 32 != 0 || N < 0) return -1;
+    fesetround(FE_TONEAREST);
+    uint32_t f = 0;
+    int64_t G = K / 32;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t g = 0; g < G; ++g)
+            f |= quantize_group_q8(W + n * K + g * 32, codes + n * K + g * 32, scales + n * G + g);
+    if (flags) *flags = f;
+    return 0;
+}
+
+/* y[m, n] = sum_k x[m,k] * w'[n,k] with w' = code * f32(scale), every term and the running
+ * sum in binary64, k ascending.  x, M, K, y and nthreads as for oracle_q4_matmul. */
+int oracle_q8_matmul(const void* x, int x_is_bf16, int64_t M, int64_t K, const int8_t* codes,
+                     const uint16_t* scales, int64_t N, double* y, int nthreads)
+{
+#ifdef _OPENMP
+    if (nthreads < 1) nthreads = 1;
+    #pragma omp parallel for schedule(dynamic, 16) num_threads(nthreads)
+#else
+    (void)nthreads;
+#endif
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t m = 0; m < M; ++m) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                const double s = (double)oracle_f16_to_f32(scales[n * (K / 32) + k / 32]);
+                acc += x_value(x, x_is_bf16, m * K + k) * ((double)codes[n * K + k] * s);
+            }
+            y[m * N + n] = acc;
+        }
+    }
+    return 0;
+}
+
 int oracle_max_threads(void)
 {
 #ifdef _OPENMP
