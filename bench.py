@@ -361,6 +361,32 @@ def time_launches(torch, fn, n, device, stream):
     return e0.elapsed_time(e1) / n
 
 
+def int8_row(torch, q4, lib, device, stream, hbm, l2):
+    """INT8-weight GEMV (the INT8 layers of a mixed INT8/INT4 model): the decode projection
+    shape M=1 K=2560 N=4096, bf16 x, weights quantised on the device, rotating copies."""
+    N, K = 4096, 2560
+    W = torch.from_numpy(synth_inputs.weights("outliers", N, K, 0)).to(device)
+    codes, scales = q4.int8_quantize(W)
+    del W
+    setb = codes.numel() + scales.numel() * 2
+    copies = max(2, -(-3 * l2 // setb) + 1)
+    cs = [(codes, scales)] + [(codes.clone(), scales.clone()) for _ in range(copies - 1)]
+    x8 = torch.from_numpy(synth_inputs.activations(1, K, "bf16", 0).view(np.int16)).view(torch.bfloat16).to(device)
+    y8 = torch.empty((1, N), dtype=torch.float32, device=device)
+
+    def i8(i):
+        c, s = cs[i % copies]
+        st = lib.q4_int8_gemv(x8.data_ptr(), 1, 1, K, c.data_ptr(), s.data_ptr(), N, y8.data_ptr(),
+                              stream.cuda_stream)
+        assert st == 0
+    log("rows: int8 gemv")
+    n_l = copies * 4
+    ms = time_launches(torch, i8, n_l, device, stream)
+    b = N * K + N * (K // 32) * 2 + K * 2 + N * 4
+    return {"workload": f"INT8 weights M=1 K={K} N={N} bf16 x", "ms": ms, "GB/s": b / ms / 1e6,
+            "frac_hbm": b / ms / 1e6 / hbm, "bytes": b, "launches": n_l}
+
+
 def measure_rows(torch, q4, lib, device, peaks, l2):
     """Every other hot-path row of the library at its configuration, one GPU."""
     out = {}
@@ -517,6 +543,7 @@ def measure_rows(torch, q4, lib, device, peaks, l2):
         out[name] = {"workload": f"F16 weights M=1 K={K} N={N} bf16 x", "ms": ms, "GB/s": b / ms / 1e6,
                      "frac_hbm": b / ms / 1e6 / hbm, "bytes": b, "launches": n_l}
         del ws16, w16
+    out["int8_gemv_2560x4096"] = int8_row(torch, q4, lib, device, stream, hbm, l2)
     # Prefill q4_gemm (bf16 x, bf16 y, f32 accumulate); inputs rotated to exceed 3x L2.
     for gw in synth_inputs.PREFILL:
         _, packed, scales = make_quantized(torch, q4, gw, 0, device)

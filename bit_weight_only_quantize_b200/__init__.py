@@ -18,7 +18,7 @@ from ._lib import Q4Error, FLAG_NONFINITE, FLAG_SCALE_OVERFLOW, GEMV_MAX_M  # no
 
 __all__ = [
     "quantize", "gemv", "gemv_multi", "GemvMulti", "gemv_gate_up", "gemv_argmax", "gemv_topk",
-    "gemv_topk_workspace_size", "topk_merge", "f16_gemv", "gemm", "gemv_workspace_size", "gemv_multi_workspace_size",
+    "gemv_topk_workspace_size", "topk_merge", "f16_gemv", "int8_quantize", "int8_gemv", "gemm", "gemv_workspace_size", "gemv_multi_workspace_size",
     "Q4Error", "FLAG_NONFINITE", "FLAG_SCALE_OVERFLOW", "GEMV_MAX_M",
 ]
 
@@ -70,6 +70,52 @@ def quantize(W: torch.Tensor, flags: torch.Tensor | None = None):
         st = _lib.load().q4_quantize(W.data_ptr(), N, K, packed.data_ptr(), scales.data_ptr(), fptr, _stream())
     _lib.check(st, "q4_quantize")
     return packed, scales
+
+
+def int8_quantize(W: torch.Tensor, flags: torch.Tensor | None = None):
+    """f32 W[N,K] -> (codes int8 [N,K], scales binary16 as int16 bits [N,K/32]) in the
+    library's INT8 format (the INT8 layers of a mixed INT8/INT4 model); ``flags`` as for
+    ``quantize``."""
+    _need(W, "W", torch.float32, 2)
+    N, K = W.shape
+    codes = torch.empty((N, K), dtype=torch.int8, device=W.device)
+    scales = torch.empty((N, max(K // 32, 0)), dtype=torch.int16, device=W.device)
+    fptr = None
+    if flags is not None:
+        _need(flags, "flags", torch.int32, 1, W.device)
+        fptr = flags.data_ptr()
+    with _on(W.device):
+        st = _lib.load().q4_int8_quantize(W.data_ptr(), N, K, codes.data_ptr(), scales.data_ptr(), fptr, _stream())
+    _lib.check(st, "q4_int8_quantize")
+    return codes, scales
+
+
+def int8_gemv(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, out: torch.Tensor | None = None):
+    """y[M,N] (f32) = x[M,K] . dequant8(W)^T for M <= 16; x is float32 or bfloat16."""
+    if x.dtype is torch.float32:
+        xt = _lib.Q4_F32
+    elif x.dtype is torch.bfloat16:
+        xt = _lib.Q4_BF16
+    else:
+        raise TypeError("x must be float32 or bfloat16")
+    _need(x, "x", x.dtype, 2)
+    _need(codes, "codes", torch.int8, 2, x.device)
+    _need(scales, "scales", torch.int16, 2, x.device)
+    M, K = x.shape
+    N = codes.shape[0]
+    if codes.shape[1] != K or tuple(scales.shape) != (N, K // 32):
+        raise ValueError("shape mismatch between x, codes and scales")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float32, device=x.device)
+    else:
+        _need(out, "out", torch.float32, 2, x.device)
+        if tuple(out.shape) != (M, N):
+            raise ValueError("out must be [M, N]")
+    with _on(x.device):
+        st = _lib.load().q4_int8_gemv(x.data_ptr(), xt, M, K, codes.data_ptr(), scales.data_ptr(), N, out.data_ptr(),
+                                      _stream())
+    _lib.check(st, "q4_int8_gemv")
+    return out
 
 
 def gemv_workspace_size(M: int, N: int, K: int) -> int:

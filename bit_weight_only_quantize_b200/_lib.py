@@ -50,6 +50,8 @@ SIGNATURES = {
     "q4_gemv_argmax_workspace_size": (_sz, []),
     "q4_gemv_argmax": (_i32, [_vp, _i32, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _vp, ctypes.c_uint32, _vp, _sz,
                               _vp]),
+    "q4_int8_quantize": (_i32, [_vp, _i64, _i64, _vp, _vp, _vp, _vp]),
+    "q4_int8_gemv": (_i32, [_vp, _i32, _i64, _i64, _vp, _vp, _i64, _vp, _vp]),
     "q4_topk_merge": (_i32, [_vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp]),
     "q4_gemv_topk_workspace_size": (_sz, [_i64, _i64, _i64, _i64, _i32]),
     "q4_gemv_topk": (_i32, [_vp, _i32, _i64, _i64, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp, ctypes.c_uint32,

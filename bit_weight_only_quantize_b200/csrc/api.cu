@@ -348,6 +348,36 @@ q4_status q4_topk_merge(const float* values, const int64_t* indices, int64_t S, 
     return q4::launch_topk_merge(values, indices, S, M, k, index, value, static_cast<cudaStream_t>(stream));
 }
 
+q4_status q4_int8_quantize(const float* W, int64_t N, int64_t K, int8_t* codes, uint16_t* scales,
+                           uint32_t* flags, void* stream)
+{
+    q4_status st = check_nk(N, K);
+    if (st != Q4_OK) return st;
+    if (N == 0) return Q4_OK;
+    if (!W || !codes || !scales) return Q4_ERR_INVALID_ARG;
+    if (misaligned(W, 16) || misaligned(codes, 16) || misaligned(scales, 2) || (flags && misaligned(flags, 4)))
+        return Q4_ERR_ALIGN;
+    q4::DeviceInfo dev;
+    if ((st = q4::current_device(&dev)) != Q4_OK) return st;
+    return q4::launch_int8_quantize(W, N, K, codes, scales, flags, static_cast<cudaStream_t>(stream), dev);
+}
+
+q4_status q4_int8_gemv(const void* x, q4_dtype x_dtype, int64_t M, int64_t K, const int8_t* codes,
+                       const uint16_t* scales, int64_t N, float* y, void* stream)
+{
+    if (x_dtype != Q4_F32 && x_dtype != Q4_BF16) return Q4_ERR_DTYPE;
+    if (M < 0 || M > Q4_GEMV_MAX_M) return Q4_ERR_SHAPE;
+    q4_status st = check_nk(N, K);
+    if (st != Q4_OK) return st;
+    if (M == 0 || N == 0) return Q4_OK;
+    if (!x || !codes || !scales || !y) return Q4_ERR_INVALID_ARG;
+    if (misaligned(x, 4) || misaligned(codes, 16) || misaligned(scales, 2) || misaligned(y, 4)) return Q4_ERR_ALIGN;
+    q4::DeviceInfo dev;
+    if ((st = q4::current_device(&dev)) != Q4_OK) return st;
+    if ((size_t)M * (size_t)K * sizeof(float) > (size_t)dev.max_smem_optin) return Q4_ERR_SHAPE;
+    return q4::launch_int8_gemv(x, x_dtype, M, K, codes, scales, N, y, static_cast<cudaStream_t>(stream), dev);
+}
+
 q4_status q4_f16_gemv(const void* x, q4_dtype x_dtype, int64_t M, int64_t K, const uint16_t* w, int64_t N, float* y,
                       uint32_t flags, void* stream)
 {

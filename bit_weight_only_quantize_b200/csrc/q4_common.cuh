@@ -77,6 +77,11 @@ q4_status launch_gemv_tma(const void* x, q4_dtype xt, int64_t M, int64_t K, cons
 q4_status launch_topk_merge(const float* values, const int64_t* indices, int64_t S, int64_t M, int64_t k,
                             int64_t* out_index, float* out_value, cudaStream_t stream);
 
+q4_status launch_int8_quantize(const float* W, int64_t N, int64_t K, int8_t* codes, uint16_t* scales,
+                               uint32_t* flags, cudaStream_t stream, const DeviceInfo& dev);
+q4_status launch_int8_gemv(const void* x, q4_dtype xt, int64_t M, int64_t K, const int8_t* codes,
+                           const uint16_t* scales, int64_t N, float* y, cudaStream_t stream, const DeviceInfo& dev);
+
 q4_status launch_f16_gemv(const void* x, q4_dtype xt, int64_t M, int64_t K, const uint16_t* w, int64_t N, float* y,
                           int prefetch, cudaStream_t stream, const DeviceInfo& dev);
 

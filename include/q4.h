@@ -260,6 +260,31 @@ Q4_API q4_status q4_topk_merge(const float* values, const int64_t* indices, int6
                                int64_t* index, float* value, void* stream);
 
 /*
+ * INT8 weights, for models that mix INT8 and INT4 layers (QKV-Core thread, section
+ * "自适应混合量化": precision-sensitive attention layers in INT8, feed-forward layers in
+ * INT4).  The page gives no encoding; this library's INT8 format is the Q4 one with 8-bit
+ * codes, per group of 32 consecutive k of a row:
+ *   amax = max |w| (exact);  s = binary16_rne(f32_rn(amax / 127))
+ *   s == 0 (or a non-finite group, or amax / 127 overflowing binary16): codes 0, scale 0,
+ *     and the Q4_FLAG_* bit as for q4_quantize
+ *   otherwise q = clamp(rint(w / f32(s)), -128, 127) (f32 division, ties to even),
+ *     stored as a two's-complement int8; dequantised w' = q * f32(s).
+ *
+ * q4_int8_quantize: W f32 [N,K] (device, 16-byte aligned) -> codes int8 [N,K] (device,
+ *   16-byte aligned) + scales binary16 bits [N,K/32] (2-byte aligned); flags as for
+ *   q4_quantize.  N, K as for q4_quantize.  Bit-identical to the definition above.
+ * q4_int8_gemv: y[M,N] (f32) = x[M,K] . dequant(W)^T for M = 1..16, x f32 or bfloat16
+ *   (device, 4-byte aligned), codes 16-byte aligned, scales 2-byte aligned, y 4-byte
+ *   aligned.  x is staged in shared memory as f32 (M*K*4 bytes; a shape whose x does not
+ *   fit returns Q4_ERR_SHAPE).  Products in f32 per group of 16 k, scaled and accumulated
+ *   in f32.  M == 0 or N == 0 is a no-op.
+ */
+Q4_API q4_status q4_int8_quantize(const float* W, int64_t N, int64_t K, int8_t* codes, uint16_t* scales,
+                                  uint32_t* flags, void* stream);
+Q4_API q4_status q4_int8_gemv(const void* x, q4_dtype x_dtype, int64_t M, int64_t K, const int8_t* codes,
+                              const uint16_t* scales, int64_t N, float* y, void* stream);
+
+/*
  * q4_f16_gemv: y[M,N] = x[M,K] . W^T for binary16 weights W (2 bytes per weight), the
  * pages' second weight format (QORA-LLM-0.8B model card, section "AVX-512 SIMD
  * Acceleration": "F16 GEMV").  Same roles as q4_gemv, without quantisation:

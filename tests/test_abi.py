@@ -202,6 +202,27 @@ def test_topk_merge_validation(lib):
     assert f(None, None, 2, 0, 20, None, None, None) == 0           # M == 0: no-op
 
 
+def test_int8_validation(lib):
+    S = None
+    q = lib.q4_int8_quantize
+    assert q(A16, 4, 96 + 8, A16, A16, None, S) == 2           # K % 32
+    assert q(A16, -1, 64, A16, A16, None, S) == 2               # N >= 0
+    assert q(None, 4, 64, A16, A16, None, S) == 1
+    assert q(A16 + 4, 4, 64, A16, A16, None, S) == 3            # W: 16 bytes
+    assert q(A16, 4, 64, A16 + 8, A16, None, S) == 3            # codes: 16 bytes
+    assert q(A16, 4, 64, A16, A16 + 1, None, S) == 3            # scales: 2 bytes
+    assert q(None, 0, 64, None, None, None, S) == 0             # N == 0: no-op
+    g = lib.q4_int8_gemv
+    assert g(A16, 7, 1, 64, A16, A16, 8, A16, S) == 4           # dtype
+    assert g(A16, 1, 17, 64, A16, A16, 8, A16, S) == 2          # M > 16
+    assert g(A16, 1, 1, 48, A16, A16, 8, A16, S) == 2           # K % 32
+    assert g(A16, 1, 1, 64, None, A16, 8, A16, S) == 1
+    assert g(A16 + 2, 1, 1, 64, A16, A16, 8, A16, S) == 3       # x: 4 bytes
+    assert g(A16, 1, 1, 64, A8, A16, 8, A16, S) == 3            # codes: 16 bytes
+    assert g(A16, 1, 1, 64, A16, A16, 8, A16 + 2, S) == 3       # y: 4 bytes
+    assert g(None, 1, 0, 64, None, None, 8, None, S) == 0       # M == 0: no-op
+
+
 def test_f16_gemv_validation(lib):
     S = None
     f = lib.q4_f16_gemv

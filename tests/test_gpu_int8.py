@@ -1,0 +1,71 @@
+"""GPU parity of the INT8 weight path (the INT8 layers of a mixed INT8/INT4 model) against
+the oracle: q4_int8_quantize bit-exact (codes, scales, flags), q4_int8_gemv within the
+GEMV tolerance (2e-3 with f32 x, 1e-2 with bf16 x, relative to the largest |y|)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth_inputs
+from tests._parity import rel_inf, to_dev_x
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f32": 2e-3, "bf16": 1e-2}
+
+
+def _quantize_dev(W):
+    import bit_weight_only_quantize_b200 as q4
+    flags = torch.zeros(1, dtype=torch.int32, device="cuda")
+    codes, scales = q4.int8_quantize(torch.from_numpy(W).cuda(), flags=flags)
+    torch.cuda.synchronize()
+    return codes, scales, int(flags.item())
+
+
+@pytest.mark.parametrize("kind,N,K", [("outliers", 256, 2560), ("normal", 1000, 96), ("student_t", 33, 32),
+                                      ("normal", 4096, 2560)])
+def test_quantize_bit_exact(kind, N, K):
+    W = synth_inputs.weights(kind, N, K, seed=N + K)
+    codes, scales, flags = _quantize_dev(W)
+    want_c, want_s, want_f = oracle.quantize8(W)
+    assert np.array_equal(codes.cpu().numpy(), want_c)
+    assert np.array_equal(scales.cpu().numpy().view(np.uint16), want_s)
+    assert flags == want_f
+
+
+def test_quantize_special_groups():
+    W = synth_inputs.weights("normal", 4, 128, seed=6)
+    W[0, 32:64] = 0.0                                       # zero group
+    W[1, 5] = np.inf                                        # non-finite
+    W[2, 64:96] = 1.0e7                                     # scale overflows binary16
+    a = np.float32(127 * 1.4 * 2.0 ** -24)                  # subnormal scale rounded down: clamp at -128
+    W[3, 96:128] = 0.0
+    W[3, 96], W[3, 97] = -a, a
+    codes, scales, flags = _quantize_dev(W)
+    want_c, want_s, want_f = oracle.quantize8(W)
+    assert np.array_equal(codes.cpu().numpy(), want_c)
+    assert np.array_equal(scales.cpu().numpy().view(np.uint16), want_s)
+    assert flags == want_f == 3
+    assert want_c[3, 96] == -128 and want_c[3, 97] == 127
+
+
+@pytest.mark.parametrize("M,N,K,x_dtype", [(1, 4096, 2560, "f32"), (1, 4096, 2560, "bf16"), (4, 1000, 1024, "bf16"),
+                                           (16, 333, 256, "bf16"), (3, 50, 96, "f32"), (2, 7, 32, "bf16")])
+def test_gemv_matches_oracle(M, N, K, x_dtype):
+    import bit_weight_only_quantize_b200 as q4
+    codes, scales, _ = oracle.quantize8(synth_inputs.weights("outliers", N, K, seed=M * 7 + N))
+    x = synth_inputs.activations(M, K, x_dtype, seed=M)
+    y = q4.int8_gemv(to_dev_x(x), torch.from_numpy(codes).cuda(), torch.from_numpy(scales.view(np.int16)).cuda())
+    torch.cuda.synchronize()
+    err = rel_inf(y.cpu().numpy(), oracle.matmul8(x, codes, scales, threads=8))
+    assert err <= TOL[x_dtype], err
+
+
+def test_gemv_x_too_large_is_rejected():
+    import bit_weight_only_quantize_b200 as q4
+    K = 8192                                               # 16 x rows of f32 x: 512 KB of shared memory
+    codes = torch.zeros((8, K), dtype=torch.int8, device="cuda")
+    scales = torch.zeros((8, K // 32), dtype=torch.int16, device="cuda")
+    x = torch.zeros((16, K), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(q4.Q4Error):
+        q4.int8_gemv(x, codes, scales)
