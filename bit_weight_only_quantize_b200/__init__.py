@@ -17,7 +17,7 @@ from . import _lib
 from ._lib import Q4Error, FLAG_NONFINITE, FLAG_SCALE_OVERFLOW, GEMV_MAX_M  # noqa: F401
 
 __all__ = [
-    "quantize", "gemv", "gemv_multi", "GemvMulti", "gemv_gate_up", "gemv_argmax", "gemv_topk",
+    "quantize", "gemv", "gemv_host", "gemv_multi", "GemvMulti", "gemv_gate_up", "gemv_argmax", "gemv_topk",
     "gemv_topk_workspace_size", "topk_merge", "f16_gemv", "int8_quantize", "int8_gemv", "gemm", "gemv_workspace_size", "gemv_multi_workspace_size",
     "Q4Error", "FLAG_NONFINITE", "FLAG_SCALE_OVERFLOW", "GEMV_MAX_M",
 ]
@@ -162,6 +162,56 @@ def gemv(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, out: torch
                          out.data_ptr(), ws_ptr, ws_bytes, _stream())
     _lib.check(st, "q4_gemv")
     return out
+
+
+def gemv_host(x_host: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, y_host: torch.Tensor | None = None,
+              x_dev: torch.Tensor | None = None, y_dev: torch.Tensor | None = None,
+              workspace: torch.Tensor | None = None, weights_static: bool = False) -> torch.Tensor:
+    """q4_gemv_host: x from host memory, y back to host memory, in one blocking call.
+
+    ``x_host`` (CPU, float32 or bfloat16, [M,K]; pin it for an asynchronous copy) is copied
+    to ``x_dev``, the product runs into ``y_dev`` and is copied to ``y_host`` (CPU f32 [M,N])
+    before the call returns.  Staging buffers and the workspace are allocated here when not
+    given (give them to keep allocation out of a loop)."""
+    if x_host.dtype == torch.float32:
+        xt = _lib.Q4_F32
+    elif x_host.dtype == torch.bfloat16:
+        xt = _lib.Q4_BF16
+    else:
+        raise TypeError("x_host must be float32 or bfloat16")
+    if x_host.is_cuda or x_host.dim() != 2 or not x_host.is_contiguous():
+        raise ValueError("x_host must be a contiguous 2-D CPU tensor")
+    _need(packed, "packed", torch.uint8, 2)
+    dev = packed.device
+    _need(scales, "scales", torch.int16, 2, dev)
+    M, K = x_host.shape
+    N = packed.shape[0]
+    if packed.shape[1] * 2 != K or tuple(scales.shape) != (N, K // 32):
+        raise ValueError("shape mismatch between x_host, packed and scales")
+    if y_host is None:
+        y_host = torch.empty((M, N), dtype=torch.float32, pin_memory=True)
+    elif y_host.is_cuda or y_host.dtype is not torch.float32 or tuple(y_host.shape) != (M, N) \
+            or not y_host.is_contiguous():
+        raise ValueError("y_host must be a contiguous float32 CPU tensor of shape (M, N)")
+    if x_dev is None:
+        x_dev = torch.empty((M, K), dtype=x_host.dtype, device=dev)
+    _need(x_dev, "x_dev", x_host.dtype, 2, dev)
+    if y_dev is None:
+        y_dev = torch.empty((M, N), dtype=torch.float32, device=dev)
+    _need(y_dev, "y_dev", torch.float32, 2, dev)
+    lib = _lib.load()
+    with _on(dev):
+        if workspace is None:
+            need = int(lib.q4_gemv_workspace_size(M, N, K))
+            if need:
+                workspace = torch.zeros(need, dtype=torch.uint8, device=dev)
+        ws_ptr = workspace.data_ptr() if workspace is not None else None
+        ws_bytes = workspace.numel() if workspace is not None else 0
+        st = lib.q4_gemv_host(x_host.data_ptr(), xt, M, K, packed.data_ptr(), scales.data_ptr(), N,
+                              y_host.data_ptr(), x_dev.data_ptr(), y_dev.data_ptr(),
+                              _lib.WEIGHTS_STATIC if weights_static else 0, ws_ptr, ws_bytes, _stream())
+    _lib.check(st, "q4_gemv_host")
+    return y_host
 
 
 def gemv_multi_workspace_size(M: int, K: int, Ns) -> int:

@@ -38,10 +38,12 @@ SIGNATURES = {
     "q4_abi_version": (_i32, []),
     "q4_status_string": (ctypes.c_char_p, [_i32]),
     "q4_device_error": (_i32, [_vp, _i32]),
+    "q4_set_consumer_wait_limit": (ctypes.c_uint64, [ctypes.c_uint64]),
     "q4_quantize": (_i32, [_vp, _i64, _i64, _vp, _vp, _vp, _vp]),
     "q4_gemv_workspace_size": (_sz, [_i64, _i64, _i64]),
     "q4_gemv": (_i32, [_vp, _i32, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _sz, _vp]),
     "q4_gemv_noalloc": (_i32, [_vp, _i32, _i64, _i64, _vp, _vp, _i64, _vp, _vp]),
+    "q4_gemv_host": (_i32, [_vp, _i32, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _vp, ctypes.c_uint32, _vp, _sz, _vp]),
     "q4_gemm": (_i32, [_vp, _i64, _i64, _vp, _vp, _i64, _vp, _vp]),
     "q4_gemv_multi_workspace_size": (_sz, [_i64, _i64, _vp, _i32]),
     "q4_gemv_multi": (_i32, [_vp, _i32, _i64, _i64, _vp, _i32, ctypes.c_uint32, _vp, _sz, _vp]),

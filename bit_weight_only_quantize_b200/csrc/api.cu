@@ -143,29 +143,47 @@ size_t workspace_for(int64_t M, int64_t K, const q4_weight* mats, int count)
     return need;
 }
 
-q4_status gemv_common(const void* x, q4_dtype x_dtype, int64_t M, int64_t K, const q4_weight* mats, int count,
-                      uint32_t flags, void* workspace, size_t workspace_bytes, void* stream)
+// Validated and planned GEMV call (nothing enqueued yet); n == 0 means nothing to do.
+struct GemvCall {
+    q4_weight kept[Q4_MULTI_MAX];
+    int n;
+    q4::GemvPlan plan;
+};
+
+q4_status gemv_prepare(const void* x, q4_dtype x_dtype, int64_t M, int64_t K, const q4_weight* mats, int count,
+                       uint32_t flags, void* workspace, size_t workspace_bytes, GemvCall* call)
 {
+    call->n = 0;
     if (x_dtype != Q4_F32 && x_dtype != Q4_BF16) return Q4_ERR_DTYPE;
     if (M < 0 || M > Q4_GEMV_MAX_M) return Q4_ERR_SHAPE;
     if (K < 32 || (K % 32) != 0 || K > INT32_MAX) return Q4_ERR_SHAPE;
     if (flags & ~Q4_WEIGHTS_STATIC) return Q4_ERR_INVALID_ARG;
-    q4_weight kept[Q4_MULTI_MAX];
     int n = 0;
-    q4_status st = collect(mats, count, K, kept, &n, M > 0);
+    q4_status st = collect(mats, count, K, call->kept, &n, M > 0);
     if (st != Q4_OK) return st;
     if (M == 0 || n == 0) return Q4_OK;
     if (!x) return Q4_ERR_INVALID_ARG;
     if (misaligned(x, 16) || (workspace && misaligned(workspace, 16))) return Q4_ERR_ALIGN;
     q4::DeviceInfo dev;
     if ((st = q4::current_device(&dev)) != Q4_OK) return st;
-    q4::GemvPlan plan;
-    if (!q4::plan_gemv(M, kept, n, K, x_dtype, dev, false, &plan)) {
+    if (!q4::plan_gemv(M, call->kept, n, K, x_dtype, dev, false, &call->plan)) {
         cudaGetLastError();
         return Q4_ERR_CUDA;
     }
-    if (plan.workspace_bytes > 0 && (!workspace || workspace_bytes < plan.workspace_bytes)) return Q4_ERR_WORKSPACE;
-    return q4::launch_gemv(x, x_dtype, M, K, kept, n, flags, workspace, plan, static_cast<cudaStream_t>(stream));
+    if (call->plan.workspace_bytes > 0 && (!workspace || workspace_bytes < call->plan.workspace_bytes))
+        return Q4_ERR_WORKSPACE;
+    call->n = n;
+    return Q4_OK;
+}
+
+q4_status gemv_common(const void* x, q4_dtype x_dtype, int64_t M, int64_t K, const q4_weight* mats, int count,
+                      uint32_t flags, void* workspace, size_t workspace_bytes, void* stream)
+{
+    GemvCall call;
+    const q4_status st = gemv_prepare(x, x_dtype, M, K, mats, count, flags, workspace, workspace_bytes, &call);
+    if (st != Q4_OK || call.n == 0) return st;
+    return q4::launch_gemv(x, x_dtype, M, K, call.kept, call.n, flags, workspace, call.plan,
+                           static_cast<cudaStream_t>(stream));
 }
 
 }  // namespace
@@ -201,6 +219,32 @@ q4_status q4_gemv_multi(const void* x, q4_dtype x_dtype, int64_t M, int64_t K, c
                         uint32_t flags, void* workspace, size_t workspace_bytes, void* stream)
 {
     return gemv_common(x, x_dtype, M, K, mats, count, flags, workspace, workspace_bytes, stream);
+}
+
+q4_status q4_gemv_host(const void* x_host, q4_dtype x_dtype, int64_t M, int64_t K, const uint8_t* packed,
+                       const uint16_t* scales, int64_t N, float* y_host, void* x_dev, float* y_dev, uint32_t flags,
+                       void* workspace, size_t workspace_bytes, void* stream)
+{
+    const q4_weight w = {packed, scales, N, y_dev};
+    GemvCall call;
+    q4_status st = gemv_prepare(x_dev, x_dtype, M, K, &w, 1, flags, workspace, workspace_bytes, &call);
+    if (st != Q4_OK || call.n == 0) return st;
+    if (!x_host || !y_host) return Q4_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t x_bytes = (size_t)M * (size_t)K * (x_dtype == Q4_F32 ? 4 : 2);
+    const size_t y_bytes = (size_t)M * (size_t)N * sizeof(float);
+    if (cudaMemcpyAsync(x_dev, x_host, x_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess) {
+        cudaGetLastError();
+        return Q4_ERR_CUDA;
+    }
+    st = q4::launch_gemv(x_dev, x_dtype, M, K, call.kept, call.n, flags, workspace, call.plan, s);
+    if (st != Q4_OK) return st;
+    if (cudaMemcpyAsync(y_host, y_dev, y_bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess) {
+        cudaGetLastError();
+        return Q4_ERR_CUDA;
+    }
+    return Q4_OK;
 }
 
 q4_status q4_gemv_gate_up(const void* x, q4_dtype x_dtype, int64_t M, int64_t K, const uint8_t* gate_packed,

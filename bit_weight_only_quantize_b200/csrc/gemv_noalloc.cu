@@ -23,7 +23,8 @@
 // current: it looks up the array's device address (in host code the array's
 // name is only a host-side stand-in, not a device address) and zero-fills it,
 // then waits for the device.  That first call must therefore come before any
-// stream capture on the device.
+// stream capture on the device.  A set-up that fails (the call returns
+// Q4_ERR_CUDA) is not remembered: the next call on the device tries it again.
 #include <mutex>
 
 #include "q4_common.cuh"
@@ -34,24 +35,27 @@ constexpr size_t kScratchBytes = size_t(1) << 20;
 __device__ __align__(256) unsigned char g_gemv_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
-std::once_flag g_setup_once[kMaxDevices];
+std::mutex g_setup_mutex[kMaxDevices];
+bool g_setup_done[kMaxDevices];          // set only by a set-up that succeeded
 void* g_scratch_addr[kMaxDevices];
-q4_status g_setup_status[kMaxDevices];
 
-void setup_device(int dev)
+// Looks up and clears the array on device `dev` (current) unless an earlier call did;
+// returns the array's device address, or nullptr when the set-up failed.
+void* scratch_of(int dev)
 {
+    std::lock_guard<std::mutex> lock(g_setup_mutex[dev]);
+    if (g_setup_done[dev]) return g_scratch_addr[dev];
     void* p = nullptr;
     cudaError_t e = cudaGetSymbolAddress(&p, g_gemv_scratch);
     if (e == cudaSuccess) e = cudaMemset(p, 0, kScratchBytes);   // the arrival counters must start at zero
     if (e == cudaSuccess) e = cudaDeviceSynchronize();
     if (e != cudaSuccess) {
         cudaGetLastError();
-        g_scratch_addr[dev] = nullptr;
-        g_setup_status[dev] = Q4_ERR_CUDA;
-        return;
+        return nullptr;
     }
     g_scratch_addr[dev] = p;
-    g_setup_status[dev] = Q4_OK;
+    g_setup_done[dev] = true;
+    return p;
 }
 
 bool misaligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) != 0; }
@@ -75,8 +79,8 @@ extern "C" q4_status q4_gemv_noalloc(const void* x, q4_dtype x_dtype, int64_t M,
     q4_status st = q4::current_device(&dev);
     if (st != Q4_OK) return st;
     if (dev.device < 0 || dev.device >= kMaxDevices) return Q4_ERR_UNSUPPORTED_DEVICE;
-    std::call_once(g_setup_once[dev.device], setup_device, dev.device);
-    if (g_setup_status[dev.device] != Q4_OK) return g_setup_status[dev.device];
+    void* scratch = scratch_of(dev.device);
+    if (!scratch) return Q4_ERR_CUDA;
 
     const q4_weight w = {packed, scales, N, y};
     q4::GemvPlan plan;
@@ -85,6 +89,6 @@ extern "C" q4_status q4_gemv_noalloc(const void* x, q4_dtype x_dtype, int64_t M,
         return Q4_ERR_CUDA;
     }
     if (plan.workspace_bytes > kScratchBytes) return Q4_ERR_WORKSPACE;
-    return q4::launch_gemv(x, x_dtype, M, K, &w, 1, 0u, g_scratch_addr[dev.device], plan,
+    return q4::launch_gemv(x, x_dtype, M, K, &w, 1, 0u, scratch, plan,
                            static_cast<cudaStream_t>(stream));
 }

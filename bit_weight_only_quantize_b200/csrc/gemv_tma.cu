@@ -59,7 +59,8 @@ constexpr double kEpilogueCost = 0.1;
 constexpr double kSplitCost = 0.9;
 constexpr size_t kCounterBytes = kCounterSlots * sizeof(unsigned);
 
-enum Mode { kF32M1 = 0, kMma8 = 1, kMma16 = 2, kMma1 = 3 };   // kMma1: kMma8 with one x row
+// kImma1: one x row (f32 or bf16) through int8 tensor-core MMAs on exact digit planes of x.
+enum Mode { kF32M1 = 0, kMma8 = 1, kMma16 = 2, kMma1 = 3, kImma1 = 4 };   // kMma1: kMma8 with one x row
 
 struct TmaMaps {
     CUtensorMap codes[Q4_MULTI_MAX];
@@ -83,6 +84,8 @@ struct TmaGemvArgs {
     int P;                            // warps per team
     int teams;                        // teams per block
     int prefetch;                     // weights may be read before the dependency wait
+    int x_f32;                        // kImma1: x is f32 (else bf16)
+    uint64_t wait_ns;                 // limit of the waits for this warp's copies (0: give up at once)
     // kEpiArgmax (greedy argmax over the rows of matrix 0, splits == 1): per x row, the
     // largest logit and its row; keys and the block counter live in a workspace that is
     // zero at rest.  (kEpiFuse: matrices 0 and 1 are gate and up, y = silu(y0) * y1 into y[0].)
@@ -208,6 +211,24 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint3
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// d = A . B + c for one m16n8k32 tile: A unsigned 8-bit, B signed 8-bit, exact int32
+// accumulation.
+__device__ __forceinline__ void imma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1, int c0, int c1)
+{
+    asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%10,%11,%10,%11};"
+        : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(c0), "r"(c1));
+}
+
+// Integer MMA results are read as f32 through a bias: the bit pattern 0x4B400000 is
+// 1.5 * 2^23, and adding an integer |v| < 2^22 to it gives the float 1.5 * 2^23 + v.
+constexpr int kBiasBits = 0x4B400000;
+// A lo-nibble column holds bias + T_lo and its hi-nibble column bias + 16 T_hi, so
+// hi * (1/16) + lo = (17/16) * 1.5 * 2^23 + T_lo + T_hi, an integer below 2^24 (exact).
+constexpr float kBias17 = 13369344.0f;
+
 __device__ __forceinline__ float scale_at(const uint4& s8, int c)
 {
     const uint32_t sw = c < 2 ? s8.x : c < 4 ? s8.y : c < 6 ? s8.z : s8.w;
@@ -233,7 +254,7 @@ __device__ __forceinline__ double sum8_bf16(const uint4 raw)
 
 template <int MODE>
 struct ModeCfg {
-    static constexpr int MP = MODE == kMma16 ? 16 : (MODE == kMma8 || MODE == kMma1) ? 8 : 1;   // MMA x rows
+    static constexpr int MP = MODE == kMma16 ? 16 : (MODE == kMma8 || MODE == kMma1) ? 8 : 1;   // x rows in red[]
     static constexpr int NT = MP >= 8 ? MP / 8 : 1;                          // n-tiles of 8 x rows
     static constexpr int kMinBlocks = 1;
 };
@@ -251,9 +272,10 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
     constexpr bool kFuse = EPI == kEpiFuse;
     constexpr bool kArgmax = EPI == kEpiArgmax;
     constexpr bool kTopk = EPI == kEpiTopk;
-    constexpr int kTkM = (MODE == kF32M1 || MODE == kMma1) ? 1 : MP;     // x rows a top-k list set covers
+    constexpr int kTkM = (MODE == kF32M1 || MODE == kMma1 || MODE == kImma1) ? 1 : MP;   // x rows of a top-k list set
     extern __shared__ unsigned char smem_raw[];
     __shared__ int s_last[kMaxWarps];
+    __shared__ uint32_t s_xmax[kMaxWarps];
     const int W = blockDim.x >> 5;
     unsigned char* smem =
         reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -351,9 +373,111 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
     //          neighbouring x rows fall on different banks.  Beside it, per group, -136 *
     //          sum(x) of the group for each x row (an f64 sum of the bf16 values, rounded
     //          once), laid out [group][n-tile][t] as the accumulator fragment of lane (g, t).
+    //  kImma1: x * 2^F rounded to an integer X (|X| < 2^30, F from max |x| of the split)
+    //          and cut into four balanced base-256 digits X = d0 2^24 + d1 2^16 + d2 2^8 + d3,
+    //          d1..d3 in [-128, 127].  The MMA's eight B columns are (digit plane p,
+    //          nibble half h) = column 2p + h: half 0 holds the digits of the even k of
+    //          each group (the low nibbles), half 1 those of the odd k (the high nibbles,
+    //          which the A operand keeps at 16 x code).  [group pair][column g][t] uint4
+    //          holds the two B registers of lane (g, t) for both groups of the pair, the
+    //          slots of the other half zero.  Then [group pair][plane][4] int: the C
+    //          operand per group and plane, bias - 8 sum(d of even k) for half 0 and
+    //          bias - 128 sum(d of odd k) for half 1, which removes the code offset 8.
     float* xoff = nullptr;
     const int rs = (ngp + 1) * 4;                                         // uint4 per staged x row
-    if constexpr (MODE == kF32M1) {
+    float plane_factor = 0.f;                                             // kImma1: 2^(-F + 8 (3 - t))
+    if constexpr (MODE == kImma1) {
+        // Item i = (group i / 4, k = 8 (i % 4) .. + 7) of the split; a thread keeps the x
+        // of its first item in registers for both passes (max |x|, then the digits).
+        const int items = ngp * 4;
+        auto load8 = [&](int i, float (&v)[8]) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[e] = 0.f;
+            const int lg = i >> 2;
+            if (i < items && lg < ng) {
+                const size_t k0 = (size_t)(g0 + lg) * 32 + (i & 3) * 8;
+                if (a.x_f32) {
+                    const float4 p = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(a.x) + k0);
+                    const float4 q = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(a.x) + k0 + 4);
+                    v[0] = p.x; v[1] = p.y; v[2] = p.z; v[3] = p.w; v[4] = q.x; v[5] = q.y; v[6] = q.z; v[7] = q.w;
+                } else {
+                    const uint4 r = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(a.x) + k0);
+                    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        v[2 * e] = __uint_as_float(w[e] << 16);
+                        v[2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+                    }
+                }
+            }
+        };
+        // max |x| over the split (bit patterns of non-negative floats order as the values)
+        float v0[8];
+        load8(threadIdx.x, v0);
+        uint32_t mx = 0u;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) mx = max(mx, __float_as_uint(v0[e]) & 0x7FFFFFFFu);
+        for (int i = threadIdx.x + blockDim.x; i < items; i += blockDim.x) {
+            float v[8];
+            load8(i, v);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) mx = max(mx, __float_as_uint(v[e]) & 0x7FFFFFFFu);
+        }
+        mx = __reduce_max_sync(0xffffffffu, mx);
+        if (lane == 0) s_xmax[warp] = mx;
+        __syncthreads();
+        mx = 0u;
+        for (int w = 0; w < W; ++w) mx = max(mx, s_xmax[w]);
+        // F with max |x| * 2^F < 2^30; 100 for a zero or subnormal maximum, 0 for a
+        // non-finite one (the product is then undefined, but every step stays defined)
+        const int ex = (int)(mx >> 23);
+        const int F = ex == 0 ? 100 : ex >= 255 ? 0 : min(29 - (ex - 127), 100);
+        const float x_scale = __uint_as_float((uint32_t)(F + 127) << 23);
+        plane_factor = __uint_as_float((uint32_t)(-F + 24 - 8 * (lane & 3) + 127) << 23);
+        uint2* xq = reinterpret_cast<uint2*>(xst);
+        int2* xc = reinterpret_cast<int2*>(xst + (size_t)ngp * 256);
+        for (int i0 = threadIdx.x - lane; i0 < items; i0 += blockDim.x) {    // warp-uniform trips
+            const int i = i0 + lane;
+            const int lg = i >> 2, t = i & 3;                                  // group, k = 8t .. 8t+7
+            float v[8];
+            if (i0 == threadIdx.x - lane) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) v[e] = v0[e];
+            } else {
+                load8(i, v);
+            }
+            uint32_t word[4][2] = {};                                          // [plane][half]
+            int dsum[4][2] = {};
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                int r = __float2int_rn(__fmul_rn(v[e], x_scale));
+#pragma unroll
+                for (int p = 3; p >= 0; --p) {
+                    const int d = p == 0 ? r : (int)((uint32_t)r << 24) >> 24;
+                    if (p > 0) r = (int)((uint32_t)r - (uint32_t)d) >> 8;
+                    word[p][e & 1] |= ((uint32_t)d & 0xFFu) << (8 * (e >> 1));
+                    dsum[p][e & 1] += d;
+                }
+            }
+#pragma unroll
+            for (int p = 0; p < 4; ++p)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    dsum[p][h] += __shfl_xor_sync(0xffffffffu, dsum[p][h], 1);
+                    dsum[p][h] += __shfl_xor_sync(0xffffffffu, dsum[p][h], 2);
+                }
+            if (i < items) {
+                const int gp = lg >> 1, half = lg & 1;
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    xq[(((gp * 8 + 2 * p) * 4 + t) << 1) + half] = make_uint2(word[p][0], 0u);
+                    xq[(((gp * 8 + 2 * p + 1) * 4 + t) << 1) + half] = make_uint2(0u, word[p][1]);
+                    if (t == 0)
+                        xc[((gp * 4 + p) << 1) + half] = make_int2(kBiasBits - 8 * dsum[p][0], kBiasBits - 128 * dsum[p][1]);
+                }
+            }
+        }
+    } else if constexpr (MODE == kF32M1) {
         float4* xf = reinterpret_cast<float4*>(xst);
         for (int i = threadIdx.x; i < ngp * 8; i += blockDim.x) {
             const int lg = i >> 3, c = i & 7;
@@ -420,7 +544,8 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
     for (int rbi = 0; rbi < nrb; ++rbi) {
         const int rb = rb_of(rbi);
         if constexpr (kFloor) floor_now = load_key_relaxed(a.tk_floor);   // used in this block's epilogue
-        float yacc = 0.f;     // kF32M1: row (lane & 15), half (lane >> 4)
+        float yacc = 0.f;     // kF32M1: row (lane & 15), half (lane >> 4); kImma1: row g, plane t
+        float yacc8 = 0.f;    // kImma1: row g + 8, plane t
         float acc[NT][4];     // MMA modes: rows g, g+8; x rows n*8 + 2t, +1
 #pragma unroll
         for (int n = 0; n < NT; ++n)
@@ -430,7 +555,7 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
         for (int jb = 0; jb < nbw; ++jb) {
             const int j = rbi * nbw + jb;
             const int s = j % kStages;
-            if (ok) ok = mbar_wait_bounded(&my_bars[s], (uint32_t)(j / kStages) & 1u, kWaitLimit);
+            if (ok) ok = a.wait_ns != 0 && mbar_wait_bounded(&my_bars[s], (uint32_t)(j / kStages) & 1u, a.wait_ns);
             if (ok) {
                 consumed = j + 1;
                 const int bf = (u0 + jb) * kBoxesPerStage;
@@ -442,7 +567,44 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
                         const unsigned char* sb = scl + (warp * kStages + s) * kStageScales + q * 16;
                         constexpr int kScaleRow = 16 * kBoxesPerStage;   // bytes per row of the scale box
                         const int gb = (bf + q) * 8;                     // first group of the box
-                        if constexpr (MODE == kF32M1) {
+                        if constexpr (MODE == kImma1) {
+                            const int g = lane >> 2, t = lane & 3;
+                            const uint4 sg = *reinterpret_cast<const uint4*>(sb + g * kScaleRow);
+                            const uint4 sg8 = *reinterpret_cast<const uint4*>(sb + (g + 8) * kScaleRow);
+                            // ldmatrix as in the bf16 modes: r0/r1 = word t of rows g/g+8 of group
+                            // 2 cp, r2/r3 the same of group 2 cp + 1 (codes 8t .. 8t+7 of each row)
+                            const int lr = lane & 7, li = lane >> 3;
+                            const uint32_t abase =
+                                smem_addr(cb) + ((li & 1) * 8 + lr) * 128 + (((li >> 1) ^ lr) << 4);
+                            const uint4* xq = reinterpret_cast<const uint4*>(xst) + ((gb >> 1) * 8 + g) * 4 + t;
+                            const int4* xc = reinterpret_cast<const int4*>(xst + (size_t)ngp * 256) + (gb >> 1) * 4 + t;
+#pragma unroll
+                            for (int cp = 0; cp < 4; ++cp) {
+                                uint32_t r0, r1, r2, r3;
+                                ldmatrix_x4(abase ^ (uint32_t)(cp << 5), r0, r1, r2, r3);
+                                const uint4 bq = xq[cp * 32];
+                                const int4 cq = xc[cp * 4];
+#pragma unroll
+                                for (int h = 0; h < 2; ++h) {
+                                    const int c = 2 * cp + h;
+                                    const uint32_t w0 = h ? r2 : r0, w1 = h ? r3 : r1;
+                                    // A: slot 4t + i holds code 8t + 2i (low nibble), slot
+                                    // 16 + 4t + i holds 16 x code 8t + 2i + 1 (high nibble in place)
+                                    int d[4];
+                                    imma_u8s8(d, w0 & 0x0F0F0F0Fu, w1 & 0x0F0F0F0Fu, w0 & 0xF0F0F0F0u,
+                                              w1 & 0xF0F0F0F0u, h ? bq.z : bq.x, h ? bq.w : bq.y, h ? cq.z : cq.x,
+                                              h ? cq.w : cq.y);
+                                    // d[0], d[2]: bias + sum over even k of (code - 8) d_t for rows
+                                    // g, g+8; d[1], d[3]: bias + 16 x the same over odd k
+                                    const float u0 =
+                                        fmaf(__int_as_float(d[1]), 0.0625f, __int_as_float(d[0])) - kBias17;
+                                    const float u1 =
+                                        fmaf(__int_as_float(d[3]), 0.0625f, __int_as_float(d[2])) - kBias17;
+                                    yacc = fmaf(scale_at(sg, c), u0, yacc);
+                                    yacc8 = fmaf(scale_at(sg8, c), u1, yacc8);
+                                }
+                            }
+                        } else if constexpr (MODE == kF32M1) {
                             const int r = lane & 15, h = lane >> 4;
                             const unsigned char* rowp = cb + r * 128 + h * 8;
                             const uint4 s8 = *reinterpret_cast<const uint4*>(sb + r * kScaleRow);
@@ -526,7 +688,18 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
 
         // ---- row block rb complete: partials -> red[warp][row][m], team sum in warp order ----
         float* my_red = red + warp * kRows * MP;
-        if constexpr (MODE == kF32M1) {
+        if constexpr (MODE == kImma1) {
+            // planes t = 0..3 of rows g and g+8 scaled by 2^(-F + 8 (3 - t)) and summed
+            float v0 = yacc * plane_factor, v1 = yacc8 * plane_factor;
+            v0 += __shfl_xor_sync(0xffffffffu, v0, 1);
+            v1 += __shfl_xor_sync(0xffffffffu, v1, 1);
+            v0 += __shfl_xor_sync(0xffffffffu, v0, 2);
+            v1 += __shfl_xor_sync(0xffffffffu, v1, 2);
+            if ((lane & 3) == 0) {
+                my_red[lane >> 2] = v0;
+                my_red[(lane >> 2) + 8] = v1;
+            }
+        } else if constexpr (MODE == kF32M1) {
             yacc += __shfl_xor_sync(0xffffffffu, yacc, 16);           // the two halves of each row
             if (lane < 16) my_red[lane] = yacc;
         } else {
@@ -758,6 +931,7 @@ size_t x_stage_bytes(int mode, int nb, int64_t M)
 {
     const int mp = mode == kMma16 ? 16 : (mode == kMma8 || mode == kMma1) ? 8 : 1;
     const size_t ngp = (size_t)nb * 8;
+    if (mode == kImma1) return ngp * 288;                  // B operands 256 B + C operands 32 B per group
     return mode == kF32M1 ? ngp * 32 * sizeof(float) : (size_t)(M + 1) * (ngp + 1) * 64 + ngp * (mp / 8) * 64;
 }
 
@@ -768,8 +942,8 @@ size_t smem_bytes(int mode, int warps, int nb, int64_t M)
 
 int mode_for(int64_t M, q4_dtype xt)
 {
-    if (M == 1 && xt == Q4_F32) return kF32M1;
-    return M == 1 ? kMma1 : M <= 8 ? kMma8 : kMma16;
+    (void)xt;
+    return M == 1 ? kImma1 : M <= 8 ? kMma8 : kMma16;
 }
 
 template <int EPI>
@@ -779,6 +953,7 @@ const void* kernel_for_epi(int mode)
     case kF32M1: return reinterpret_cast<const void*>(&gemv_tma_kernel<kF32M1, EPI>);
     case kMma8: return reinterpret_cast<const void*>(&gemv_tma_kernel<kMma8, EPI>);
     case kMma1: return reinterpret_cast<const void*>(&gemv_tma_kernel<kMma1, EPI>);
+    case kImma1: return reinterpret_cast<const void*>(&gemv_tma_kernel<kImma1, EPI>);
     default: return reinterpret_cast<const void*>(&gemv_tma_kernel<kMma16, EPI>);
     }
 }
@@ -938,6 +1113,8 @@ q4_status launch_gemv_tma(const void* x, q4_dtype xt, int64_t M, int64_t K, cons
     a.P = plan.chunk;
     a.teams = plan.xcap;
     a.prefetch = prefetch;
+    a.x_f32 = xt == Q4_F32 ? 1 : 0;
+    a.wait_ns = consumer_wait_ns();
     a.am_key = am ? am->key : nullptr;
     a.am_done = am ? am->done : nullptr;
     a.am_index = am ? am->index : nullptr;

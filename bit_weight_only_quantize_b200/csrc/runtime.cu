@@ -2,6 +2,7 @@
 // the driver entry point, and the library's device error word.
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "tma.cuh"
@@ -28,18 +29,11 @@ void load_encode()
 __device__ unsigned g_device_error = 0;
 
 constexpr int kMaxDevices = 64;
-std::once_flag g_err_once[kMaxDevices];
-unsigned* g_err_addr[kMaxDevices];
+std::mutex g_err_mutex;
+unsigned* g_err_addr[kMaxDevices];      // set once the lookup has succeeded on the device
 
-void lookup_err(int dev)
-{
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) {
-        cudaGetLastError();
-        p = nullptr;
-    }
-    g_err_addr[dev] = static_cast<unsigned*>(p);
-}
+// Limit of the kernels' waits for their own TMA copies (see q4_set_consumer_wait_limit).
+std::atomic<uint64_t> g_consumer_wait_ns{kWaitLimitNs};
 
 // Occupancy answers already obtained (a handful of kernels x shapes per process).
 struct OccEntry {
@@ -121,11 +115,26 @@ unsigned* device_error_word()
         cudaGetLastError();
         return nullptr;
     }
-    std::call_once(g_err_once[dev], lookup_err, dev);
+    std::lock_guard<std::mutex> lock(g_err_mutex);
+    if (!g_err_addr[dev]) {                // a failed lookup is retried by the next call
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) {
+            cudaGetLastError();
+            return nullptr;
+        }
+        g_err_addr[dev] = static_cast<unsigned*>(p);
+    }
     return g_err_addr[dev];
 }
 
+uint64_t consumer_wait_ns() { return g_consumer_wait_ns.load(std::memory_order_relaxed); }
+
 }  // namespace q4
+
+extern "C" uint64_t q4_set_consumer_wait_limit(uint64_t ns)
+{
+    return q4::g_consumer_wait_ns.exchange(ns);
+}
 
 extern "C" q4_status q4_device_error(uint32_t* out, int clear)
 {

@@ -117,4 +117,9 @@ bool encode_tma_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base
 constexpr uint32_t kErrWaitTimeout = 1u;
 unsigned* device_error_word();   // device address of the word (nullptr on failure)
 
+// Limit, in nanoseconds, of a GEMV warp's waits for its own TMA copies (0: give up at the
+// first wait); kWaitLimitNs unless q4_set_consumer_wait_limit changed it.  Waits that drain
+// copies still in flight always use kWaitLimitNs.
+uint64_t consumer_wait_ns();
+
 }  // namespace q4

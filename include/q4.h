@@ -99,6 +99,21 @@ Q4_API const char* q4_status_string(q4_status status);
 Q4_API q4_status q4_device_error(uint32_t* out, int clear);
 
 /*
+ * q4_set_consumer_wait_limit: sets, for every device and every later launch of the TMA
+ * GEMV kernels (q4_gemv, q4_gemv_multi, q4_gemv_noalloc, q4_gemv_host, q4_gemv_gate_up,
+ * q4_gemv_argmax, q4_gemv_topk), how long a warp waits for one of its own TMA transfers
+ * before it gives up, in nanoseconds, and returns the previous limit.  The default is
+ * 1,000,000,000 (1 s); every legitimate wait lasts microseconds.  0 makes each launch
+ * give up at its first wait: the kernel then records Q4_DEVICE_ERR_WAIT_TIMEOUT, waits
+ * (up to 1 s, a limit this call does not change) for the transfers it has in flight,
+ * leaves any workspace it shares zero at rest as a completed call does, and returns
+ * with an undefined output.  This exercises the failure path without any fault; it
+ * exists for tests of that path.  Not synchronised with launches in flight: a launch
+ * uses the value set when it was enqueued.
+ */
+Q4_API uint64_t q4_set_consumer_wait_limit(uint64_t ns);
+
+/*
  * q4_quantize: encode W[N,K] (f32, device) into the Q4 format above.
  *   W       device, f32 [N,K], 16-byte aligned.
  *   N, K    N >= 0 (N == 0 enqueues nothing and returns Q4_OK);
@@ -133,12 +148,37 @@ Q4_API size_t q4_gemv_workspace_size(int64_t M, int64_t N, int64_t K);
  *              must start at zero (the arrival counters) at zero again, so the
  *              same workspace can be reused by later calls without clearing.
  *              Calls that share a workspace must not overlap on the GPU.
- * Arithmetic: codes are expanded exactly, each group's 32 products are summed in
- * f32, multiplied by the group scale and accumulated in f32.
+ * Arithmetic.  M = 1 (f32 or bf16 x): x is scaled by a power of two 2^F with
+ * max |x| * 2^F < 2^30 (F from the x of each K split), rounded once to an integer and
+ * cut into four base-256 digits; the codes times the digits are summed exactly on the
+ * integer tensor cores per group, and each group's sum is multiplied by its scale and
+ * accumulated in f32 (per digit plane, combined at the end).  M >= 2 with bf16 x: the
+ * codes are expanded exactly and multiplied by x on the bf16 tensor cores with f32
+ * accumulation, each group's sum scaled and accumulated in f32.  Other shapes (f32 x
+ * with M >= 2, K % 256 != 0, scales not 16-byte aligned): exact expansion and f32 FMAs.
  */
 Q4_API q4_status q4_gemv(const void* x, q4_dtype x_dtype, int64_t M, int64_t K,
                   const uint8_t* packed, const uint16_t* scales, int64_t N,
                   float* y, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * q4_gemv_host: q4_gemv from and to host memory, for a caller whose activations live on
+ * the host: copies x_host into x_dev, runs q4_gemv into y_dev, copies y_dev into y_host
+ * and waits for the stream.  On return y_host holds the product.
+ *   x_host   host, [M,K] f32 or bfloat16 (x_dtype); page-locked memory makes the copy
+ *            asynchronous (pageable memory works, the runtime stages it).
+ *   y_host   host, f32 [M,N] (output).
+ *   x_dev    device staging buffer of M*K elements of x_dtype, 16-byte aligned.
+ *   y_dev    device staging buffer, f32 [M,N], 4-byte aligned (overwritten).
+ *   flags    0 or Q4_WEIGHTS_STATIC (as for q4_gemv_multi).
+ *   Other arguments, the arithmetic and the errors as for q4_gemv; argument errors return
+ *   before any copy is enqueued.  M == 0 or N == 0 is a no-op.  The call blocks the host
+ *   until the stream's work up to and including the copy of y has finished.
+ */
+Q4_API q4_status q4_gemv_host(const void* x_host, q4_dtype x_dtype, int64_t M, int64_t K,
+                              const uint8_t* packed, const uint16_t* scales, int64_t N,
+                              float* y_host, void* x_dev, float* y_dev, uint32_t flags,
+                              void* workspace, size_t workspace_bytes, void* stream);
 
 /* One weight matrix of a q4_gemv_multi call and its output. */
 typedef struct q4_weight {
@@ -332,7 +372,8 @@ Q4_API q4_status q4_gemm(const uint16_t* x, int64_t M, int64_t K, const uint8_t*
  * of a workspace argument.  It calls no cudaMalloc/cudaFree.
  *  - The first call on a device performs a one-time set-up (looks up the
  *    array's address, zero-fills it and waits for the device), so make that
- *    first call before any stream capture on the device.
+ *    first call before any stream capture on the device.  If the set-up fails
+ *    the call returns Q4_ERR_CUDA and the next call on that device retries it.
  *  - All calls on a device share the array, which keeps the last call's
  *    contents: calls that overlap on the GPU race.  Serialise them.
  *  - A shape whose split needs more than 1 MiB of scratch returns

@@ -33,15 +33,19 @@ def _rng(seed: int, stream: int) -> np.random.Generator:
     return np.random.default_rng([seed, stream])
 
 
-def weights(kind: str, N: int, K: int, seed: int = 0) -> np.ndarray:
-    """f32 [N,K] weight matrix drawn by recipe ``kind``."""
+def weights(kind: str, N: int, K: int, seed: int = 0, rows: int | None = None) -> np.ndarray:
+    """f32 [N,K] weight matrix drawn by recipe ``kind``; with ``rows``, only its first
+    ``rows`` rows (the same values, drawn without the rest of the matrix)."""
     if K % 32:
         raise ValueError("K must be a multiple of 32")
+    n = N if rows is None else max(0, min(rows, N))
+    if kind == "outliers" and n < N:
+        return weights(kind, N, K, seed)[:n]       # outlier positions are drawn over the whole matrix
     r = _rng(seed, 0)
     if kind == "student_t":
-        W = (WEIGHT_STD * r.standard_t(4.0, size=(N, K))).astype(np.float32)
+        W = (WEIGHT_STD * r.standard_t(4.0, size=(n, K))).astype(np.float32)
     else:
-        W = r.normal(0.0, WEIGHT_STD, size=(N, K)).astype(np.float32)
+        W = r.normal(0.0, WEIGHT_STD, size=(n, K)).astype(np.float32)
     if kind in ("normal", "student_t"):
         return W
     pos = _rng(seed, 2)
@@ -55,7 +59,7 @@ def weights(kind: str, N: int, K: int, seed: int = 0) -> np.ndarray:
             W[rows, groups * 32 + elem] *= np.float32(8.0)
         return W
     if kind == "lm_head":
-        for r0 in range(0, N, 1024):
+        for r0 in range(0, n, 1024):
             g = (r0 // 1024) % G
             W[r0, g * 32:(g + 1) * 32] = 0.0
         return W

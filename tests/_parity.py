@@ -33,22 +33,68 @@ def rel_inf(y: np.ndarray, ref: np.ndarray) -> float:
     return num / den
 
 
+# Unit roundoffs of the two kinds of f32 sums the kernels make.  A CUDA-core f32 add or
+# FMA rounds to nearest (u = 2^-24).  An f32 accumulation inside an mma.sync tensor-core
+# instruction is not specified to round to nearest; the tests take the truncating
+# (round-toward-zero) model for every such sum, bf16 and binary16 operands alike:
+# u = 2^-23.
+U_CUDA_CORE = 2.0 ** -24
+U_TENSOR_F32 = 2.0 ** -23
+
+
+def gamma(n: int, u: float) -> float:
+    """gamma_n = n u / (1 - n u): the relative bound of a sum reached through n roundings."""
+    return n * u / (1 - n * u)
+
+
+def x_f64(x: np.ndarray) -> np.ndarray:
+    """float32 array, or uint16 bfloat16 bits -> exact float64 values."""
+    if x.dtype == np.uint16:
+        return (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return x.astype(np.float64)
+
+
 def f32_sum_bound(x: np.ndarray, deq: np.ndarray, roundings: int) -> np.ndarray:
     """gamma_n * sum_k |x_k w'_k| per output: the classical bound on an f32 sum of
-    exact products reached through at most n roundings (u = 2^-24)."""
-    u = 2.0 ** -24
-    gamma = roundings * u / (1 - roundings * u)
-    xa = np.abs(x.astype(np.float64) if x.dtype != np.uint16 else
-                (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64))
-    return gamma * (xa @ np.abs(deq).T)
+    exact products reached through at most n round-to-nearest roundings."""
+    return gamma(roundings, U_CUDA_CORE) * (np.abs(x_f64(x)) @ np.abs(deq).T)
 
 
 def offset_path_bound(x: np.ndarray, scales: np.ndarray, roundings: int) -> np.ndarray:
-    """Bound for the bf16-activation decode path, which sums x_k * (128 + code_k) and
-    removes 136 * sum(x) per half group: every rounded partial is at most
-    144 * s_k * |x_k| per term, so |y - y_ref| <= gamma_n * sum_k |x_k| * 144 * s_k."""
-    u = 2.0 ** -24
-    gamma = roundings * u / (1 - roundings * u)
-    xa = np.abs((x.astype(np.uint32) << 16).view(np.float32).astype(np.float64))
+    """Bound for the bf16-activation path of M >= 2, which sums x_k * (128 + code_k) on
+    the tensor cores and removes 136 * sum(x) per half group: every partial is at most
+    144 * s_k * |x_k| per term, so |y - y_ref| <= gamma_n * sum_k |x_k| * 144 * s_k,
+    with the tensor-core unit roundoff."""
+    xa = np.abs(x_f64(x))
     s = np.repeat(scales.view(np.float16).astype(np.float64), 32, axis=1)
-    return gamma * (xa @ (144.0 * s).T)
+    return gamma(roundings, U_TENSOR_F32) * (xa @ (144.0 * s).T)
+
+
+def digit_shift(x_row: np.ndarray) -> int:
+    """The power of two F the M = 1 path scales x by: max |x| * 2^F < 2^30 (F <= 100)."""
+    mx = float(np.max(np.abs(x_row))) if x_row.size else 0.0
+    if mx == 0.0 or mx < 2.0 ** -126:
+        return 100
+    e = int(np.floor(np.log2(mx)))
+    if 2.0 ** e > mx:              # guard log2 rounding at exact powers of two
+        e -= 1
+    if 2.0 ** (e + 1) <= mx:
+        e += 1
+    return min(29 - e, 100)
+
+
+def digit_path_bound(x: np.ndarray, deq: np.ndarray, roundings: int) -> np.ndarray:
+    """Bound for the M = 1 path.  x is rounded once to the integer X = rint(x 2^F) (error
+    <= 2^(-F-1) per element) and cut into four base-256 digit planes X_p; the integer MMAs
+    are exact, and plane p's f32 sum (CUDA-core FMAs of scale x exact group sums) is
+    bounded by gamma_n sum_k |w'_k| |X_p,k|.  Scaled back by 2^(-F + 8 (3 - p)) and summed
+    over p this is at most gamma_n sum_k |w'_k| (|x_k| + 1.01 * 2^(24 - F)).  Split-K
+    splits take F from their own part of x, which only shrinks both terms."""
+    xs = x_f64(x)
+    wa = np.abs(deq)
+    out = np.empty((xs.shape[0], deq.shape[0]))
+    for m in range(xs.shape[0]):
+        q = 2.0 ** -digit_shift(xs[m])
+        rows = wa.sum(axis=1)
+        out[m] = 0.5 * q * rows + gamma(roundings, U_CUDA_CORE) * (wa @ (np.abs(xs[m]) + 1.01 * 2.0 ** 24 * q))
+    return out

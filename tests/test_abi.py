@@ -235,3 +235,11 @@ def test_f16_gemv_validation(lib):
     assert f(A16, 1, 1, 64, A8, 8, A16, 0, S) == 3                  # w alignment
     assert f(A16, 1, 1, 64, A16, 8, A16 + 2, 0, S) == 3             # y alignment
     assert f(None, 1, 0, 64, None, 8, None, 0, S) == 0              # M == 0: no-op
+
+
+def test_consumer_wait_limit_round_trips(lib):
+    """The failure-path hook keeps the value it is given and defaults to 1 s."""
+    prev = lib.q4_set_consumer_wait_limit(12345)
+    assert prev == 10 ** 9
+    assert lib.q4_set_consumer_wait_limit(prev) == 12345
+    assert lib.q4_set_consumer_wait_limit(prev) == prev

@@ -65,6 +65,16 @@ def test_tile_128x128():
     check(1024, 2560, 512, seed=4, m_sample=96, n_sample=96)
 
 
+@pytest.mark.parametrize("M,N,K", [
+    (2048, 2432, 128),     # 8 x 19 = 152 tiles of 256 x 128 (>= 148 SMs): the two-accumulator tile
+    (512, 2048, 256),      # the M = 512 prefill tiling (128 x 64 tiles)
+    (2176, 4160, 64),      # ragged in M and N at the 256 x 128 tiling
+])
+def test_large_tiles_full_output(M, N, K):
+    """Every output element of the large-tile paths against the oracle (not a sample)."""
+    check(M, N, K, kind="outliers", seed=M + K)
+
+
 def test_zero_weights_give_zero():
     M, N, K = 256, 64, 512
     W = np.zeros((N, K), np.float32)

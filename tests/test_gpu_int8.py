@@ -7,7 +7,7 @@ import torch
 
 import oracle
 import synth_inputs
-from tests._parity import rel_inf, to_dev_x
+from tests._parity import f32_sum_bound, rel_inf, to_dev_x
 
 pytestmark = pytest.mark.gpu
 
@@ -50,15 +50,26 @@ def test_quantize_special_groups():
 
 
 @pytest.mark.parametrize("M,N,K,x_dtype", [(1, 4096, 2560, "f32"), (1, 4096, 2560, "bf16"), (4, 1000, 1024, "bf16"),
-                                           (16, 333, 256, "bf16"), (3, 50, 96, "f32"), (2, 7, 32, "bf16")])
+                                           (16, 333, 256, "bf16"), (3, 50, 96, "f32"), (2, 7, 32, "bf16"),
+                                           # more rows than the grid holds warps: rows are walked in rounds
+                                           (1, 20000, 2560, "bf16"),
+                                           # 160 KB of f32 x in shared memory: one block per SM
+                                           (16, 300, 2560, "f32")])
 def test_gemv_matches_oracle(M, N, K, x_dtype):
     import bit_weight_only_quantize_b200 as q4
     codes, scales, _ = oracle.quantize8(synth_inputs.weights("outliers", N, K, seed=M * 7 + N))
     x = synth_inputs.activations(M, K, x_dtype, seed=M)
     y = q4.int8_gemv(to_dev_x(x), torch.from_numpy(codes).cuda(), torch.from_numpy(scales.view(np.int16)).cuda())
     torch.cuda.synchronize()
-    err = rel_inf(y.cpu().numpy(), oracle.matmul8(x, codes, scales, threads=8))
+    got = y.cpu().numpy()
+    ref = oracle.matmul8(x, codes, scales, threads=8)
+    err = rel_inf(got, ref)
     assert err <= TOL[x_dtype], err
+    # per element: exact code x exact x products summed in f32 (16 per block of k, one
+    # scale FMA per block, a lane's blocks, the warp's 5 shuffle adds): gamma_n sum |x w'|
+    n = 16 + K // 16 + 8
+    bound = f32_sum_bound(x, oracle.dequantize8(codes, scales), n)
+    assert np.all(np.abs(got - ref) <= bound + 1e-30)
 
 
 def test_gemv_x_too_large_is_rejected():

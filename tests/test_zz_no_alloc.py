@@ -42,7 +42,11 @@ def test_noalloc_matches_gemv_on_consecutive_calls(M, N, K):
         _lib.check(lib.q4_gemv_noalloc(x.data_ptr(), _lib.Q4_BF16, M, K, pk.data_ptr(), sc.data_ptr(), N,
                                        y.data_ptr(), stream), "q4_gemv_noalloc")
         torch.cuda.synchronize()
-        assert rel_inf(y.cpu().numpy(), y_ref.cpu().numpy().astype(np.float64)) <= 1e-5
+        got = y.cpu().numpy()
+        assert rel_inf(got, y_ref.cpu().numpy().astype(np.float64)) <= 1e-5
+        # and against the oracle itself, not only against the other entry point
+        ref = oracle.matmul(synth_inputs.activations(M, K, "bf16", seed=call), packed, scales, threads=8)
+        assert rel_inf(got, ref) <= 1e-5
 
 
 def test_noalloc_validates_like_gemv():
