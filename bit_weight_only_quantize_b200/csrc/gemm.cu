@@ -24,6 +24,8 @@
 // overlaps the MMAs of the next.  Every mbarrier wait is bounded; on a timeout the
 // block records kErrWaitTimeout, all roles stop, outstanding copies and MMAs are
 // waited for (bounded) and tensor memory is freed before the block exits.
+#include <algorithm>
+
 #include "tma.cuh"
 
 namespace q4 {
@@ -411,6 +413,345 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     if (warp == kMmaWarp) tmem_dealloc(tmem_base, C::kTmemCols);
 }
 
+// ------------------------------------------------------------------------------------
+// CTA-pair kernel (cta_group::2).  Two CTAs of a cluster share one 256 x BNP output tile:
+// CTA r holds x rows m0 + 128 r .. + 127 and dequantises weight rows n0 + (BNP/2) r ..
+// + BNP/2 - 1; one thread of CTA 0 issues tcgen05.mma.cta_group::2 (M = 256, N = BNP),
+// which reads the A and B halves from both CTAs' shared memory, and each CTA's tensor
+// memory receives its 128 rows x BNP f32 accumulators.  Per SM this halves the
+// shared-memory operand traffic and the dequantisation per flop of a single-CTA tile.
+// Both CTAs' dequantise warps arrive on CTA 0's "B ready" barrier and both CTAs'
+// epilogue warps on its "accumulator empty" barrier; MMA completion is committed to the
+// barriers of both CTAs (multicast commit).  No TMA load uses cluster multicast: each
+// CTA loads its own x and code tiles.
+
+__device__ __forceinline__ uint32_t cluster_rank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// Shared::cluster address of `p` (this CTA's shared memory) in the CTA of rank `rank`.
+__device__ __forceinline__ uint32_t peer_addr(const void* p, uint32_t rank)
+{
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr(p)), "r"(rank));
+    return r;
+}
+
+// Arrive on an mbarrier of a CTA of this cluster (address from peer_addr).  The writes
+// the arrival publishes are the dequantised tiles (ordered for the tensor cores by
+// fence.proxy.async before the arrive) and completed tensor-memory loads.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr)
+{
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// Waits on barriers the peer CTA arrives on use the plain bounded wait.
+__device__ __forceinline__ bool mbar_wait_cluster_bounded(uint64_t* bar, uint32_t parity, uint64_t limit_ns)
+{
+    return mbar_wait_bounded(bar, parity, limit_ns);
+}
+
+__device__ __forceinline__ void cluster_sync_all()
+{
+    asm volatile("barrier.cluster.arrive.release;\n barrier.cluster.wait.acquire;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc2(uint32_t* dst_smem, uint32_t ncols)
+{
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish2()
+{
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc2(uint32_t taddr, uint32_t ncols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+__device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                              uint32_t accumulate)
+{
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive once on the mbarrier at the same offset in both CTAs of the pair when every
+// tcgen05 operation this thread issued so far has completed.
+__device__ __forceinline__ void mma_commit_pair(uint64_t* bar)
+{
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            smem_addr(bar)),
+        "h"((uint16_t)3)
+        : "memory");
+}
+
+template <int BNP>
+struct PairCfg {
+    static constexpr int BH = BNP / 2;                            // weight rows per CTA
+    static constexpr int kStages = BNP == 256 ? 5 : 7;
+    static constexpr uint32_t kABytes = 128 * kBK * 2;            // this CTA's 128 x rows
+    static constexpr uint32_t kBBytes = BH * kBK * 2;             // this CTA's dequantised weight rows
+    static constexpr uint32_t kRawBytes = BH * (kBK / 2);
+    static constexpr uint32_t kScaleBytes = BH * 16;
+    static constexpr uint32_t kStageBytes = kABytes + kBBytes + kRawBytes + kScaleBytes;
+    static constexpr uint32_t kTxBytes = kABytes + kRawBytes;
+    static constexpr uint32_t kTmemCols = 2 * BNP;                // double-buffered 128 x BNP f32
+    static constexpr size_t kSmem = 1024 + (size_t)kStages * kStageBytes + 256;
+    static_assert(kTmemCols == 256 || kTmemCols == 512, "tensor memory columns");
+    static_assert(kStageBytes % 1024 == 0, "stage alignment");
+};
+
+template <int BNP>
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_codes,
+                 const __grid_constant__ CUtensorMap tm_scales, const GemmArgs a)
+{
+    using C = PairCfg<BNP>;
+    constexpr int S = C::kStages;
+    constexpr int BH = C::BH;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* smem =
+        reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // Per stage: [A tile][B tile][raw codes][scales]; the layout is the same in both CTAs,
+    // so one descriptor names the operand halves of both.
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes);
+    uint64_t* full = bars;               // producer -> dequant (own TMA bytes)
+    uint64_t* bready = bars + S;         // dequant of both CTAs -> MMA (CTA 0's copy is used)
+    uint64_t* empty = bars + 2 * S;      // MMA -> producers of both CTAs (multicast commit)
+    uint64_t* accfull = bars + 3 * S;    // MMA -> epilogues of both CTAs, 2 buffers
+    uint64_t* accempty = accfull + 2;    // epilogues of both CTAs -> MMA (CTA 0's copy)
+    uint64_t* drain = accempty + 2;      // final commit on abort
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();
+    const int cluster = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
+    const int tiles = a.tiles_m * a.tiles_n;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&bready[s], 2 * kDeqWarps);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&accfull[b], 1);
+            mbar_init(&accempty[b], 8);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&tm_x);
+        tma_prefetch_desc(&tm_codes);
+        if (a.scale_tma) tma_prefetch_desc(&tm_scales);
+    }
+    if (warp == kMmaWarp) {
+        tmem_alloc2(tmem_slot, C::kTmemCols);
+        tmem_relinquish2();
+    }
+    tc_fence_before();
+    cluster_sync_all();                  // both CTAs' barriers initialised before any remote arrive
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    pdl_launch_dependents();
+    pdl_wait();
+
+    auto fail = [&]() {
+        *abort_flag = 1;
+        atomicOr(a.err, kErrWaitTimeout);
+    };
+
+    if (warp == kProducerWarp) {
+        if (lane == 0) {
+            int it = 0;
+            int last_phase[16];
+            for (int s = 0; s < S; ++s) last_phase[s] = -1;
+            for (int t = cluster; t < tiles && !*abort_flag; t += nclusters) {
+                const int m0 = (t % a.tiles_m) * 256 + (int)rank * 128;
+                const int n0 = (t / a.tiles_m) * BNP + (int)rank * BH;
+                for (int kb = 0; kb < a.kblocks; ++kb, ++it) {
+                    const int s = it % S;
+                    const uint32_t ph = (uint32_t)(it / S) & 1u;
+                    if (!mbar_wait_cluster_bounded(&empty[s], ph ^ 1u, kWaitLimit)) { fail(); break; }
+                    if (*abort_flag) break;
+                    unsigned char* st = smem + s * C::kStageBytes;
+                    mbar_arrive_expect_tx(&full[s], C::kTxBytes + (a.scale_tma ? C::kScaleBytes : 0u));
+                    tma_load_2d(st, &tm_x, kb * kBK, m0, &full[s]);
+                    tma_load_2d(st + C::kABytes + C::kBBytes, &tm_codes, kb * (kBK / 2), n0, &full[s]);
+                    if (a.scale_tma)
+                        tma_load_2d(st + C::kABytes + C::kBBytes + C::kRawBytes, &tm_scales, (kb * 2) & ~7, n0,
+                                    &full[s]);
+                    last_phase[s] = (int)ph;
+                }
+            }
+            if (*abort_flag)
+                for (int s = 0; s < S; ++s)
+                    if (last_phase[s] >= 0) mbar_wait_bounded(&full[s], (uint32_t)last_phase[s], kWaitLimit);
+        }
+    } else if (warp == kMmaWarp) {
+        if (rank == 0 && lane == 0) {
+            constexpr uint32_t idesc = instr_desc(256, BNP);
+            int it = 0, tcount = 0;
+            bool issued_any = false;
+            for (int t = cluster; t < tiles && !*abort_flag; t += nclusters, ++tcount) {
+                const int buf = tcount & 1;
+                if (!mbar_wait_cluster_bounded(&accempty[buf], ((uint32_t)(tcount >> 1) & 1u) ^ 1u, kWaitLimit)) {
+                    fail();
+                    break;
+                }
+                tc_fence_after();
+                bool ok = true;
+                for (int kb = 0; kb < a.kblocks; ++kb, ++it) {
+                    const int s = it % S;
+                    if (!mbar_wait_cluster_bounded(&bready[s], (uint32_t)(it / S) & 1u, kWaitLimit)) {
+                        fail();
+                        ok = false;
+                        break;
+                    }
+                    if (*abort_flag) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t st = smem_addr(smem + s * C::kStageBytes);
+                    const uint32_t d = tmem_base + (uint32_t)(buf * BNP);
+#pragma unroll
+                    for (int j = 0; j < kBK / 16; ++j)
+                        mma_bf16_pair(d, sw128_desc(st + j * 32), sw128_desc(st + C::kABytes + j * 32), idesc,
+                                      (kb > 0 || j > 0) ? 1u : 0u);
+                    mma_commit_pair(&empty[s]);    // both CTAs' stages reusable once these MMAs have read them
+                    issued_any = true;
+                }
+                if (!ok) break;
+                mma_commit_pair(&accfull[buf]);
+            }
+            if (*abort_flag && issued_any) {
+                mma_commit_pair(drain);
+                mbar_wait_bounded(drain, 0, kWaitLimit);
+            }
+        }
+    } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 4) {
+        const int quad = warp & 3;             // tensor-memory lanes 32*quad .. 32*quad+31
+        int tcount = 0;
+        const bool vec_ok = (a.N % 8) == 0 && (reinterpret_cast<uintptr_t>(a.y) & 15) == 0;
+        const uint32_t accempty0 = peer_addr(accempty, 0);     // CTA 0's accempty[0]; buffer b at + 8 b
+        for (int t = cluster; t < tiles && !*abort_flag; t += nclusters, ++tcount) {
+            const int buf = tcount & 1;
+            if (!mbar_wait_cluster_bounded(&accfull[buf], (uint32_t)(tcount >> 1) & 1u, kWaitLimit)) { fail(); break; }
+            tc_fence_after();
+            const int row = (t % a.tiles_m) * 256 + (int)rank * 128 + quad * 32 + lane;
+            const int n0 = (t / a.tiles_m) * BNP;
+#pragma unroll 1
+            for (int c0 = 0; c0 < BNP; c0 += 32) {
+                uint32_t r[32];
+                tmem_ld32(tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(buf * BNP + c0), r);
+                const int col = n0 + c0;
+                if (row < a.M) {
+                    uint16_t* dst = a.y + (size_t)row * a.N + col;
+                    if (vec_ok && col + 32 <= a.N) {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            uint4 o;
+                            o.x = pack_bf16x2(__uint_as_float(r[8 * q + 0]), __uint_as_float(r[8 * q + 1]));
+                            o.y = pack_bf16x2(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3]));
+                            o.z = pack_bf16x2(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5]));
+                            o.w = pack_bf16x2(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7]));
+                            *reinterpret_cast<uint4*>(dst + 8 * q) = o;
+                        }
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < 32; ++q)
+                            if (col + q < a.N) dst[q] = (uint16_t)(pack_bf16x2(__uint_as_float(r[q]), 0.f) & 0xFFFFu);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(accempty0 + 8u * (uint32_t)buf);
+        }
+    } else {
+        // Dequantise this CTA's BH weight rows of every stage; each thread owns BH*8/512
+        // chunks (row n, 16-byte k chunk c).
+        const int dt = threadIdx.x - kDeqWarp0 * 32;
+        constexpr int kChunks = BH * 8 / (kDeqWarps * 32);
+        const DequantConsts dk;
+        const uint32_t bready0 = peer_addr(bready, 0);         // CTA 0's bready[0]; stage s at + 8 s
+        int it = 0;
+        for (int t = cluster; t < tiles && !*abort_flag; t += nclusters) {
+            const int n0 = (t / a.tiles_m) * BNP + (int)rank * BH;
+            float sc0[kChunks], sc1[kChunks], sc2[kChunks];
+            auto load_scales = [&](int kb, float (&dst)[kChunks]) {
+#pragma unroll
+                for (int q = 0; q < kChunks; ++q) {
+                    const int idx = dt + q * kDeqWarps * 32;
+                    const int n = n0 + idx / 8, g = kb * 2 + (idx & 7) / 4;
+                    dst[q] = (kb < a.kblocks && n < a.N && g < a.G)
+                                 ? __half2float(__ushort_as_half(__ldg(a.scales + (size_t)n * a.G + g)))
+                                 : 0.f;
+                }
+            };
+            if (!a.scale_tma) {
+                load_scales(0, sc0);
+                load_scales(1, sc1);
+            }
+            bool ok = true;
+            for (int kb = 0; kb < a.kblocks; ++kb, ++it) {
+                if (!a.scale_tma) load_scales(kb + 2, sc2);
+                const int s = it % S;
+                if (!mbar_wait_bounded(&full[s], (uint32_t)(it / S) & 1u, kWaitLimit)) { fail(); ok = false; break; }
+                if (*abort_flag) { ok = false; break; }
+                unsigned char* st = smem + s * C::kStageBytes;
+                unsigned char* bt = st + C::kABytes;
+                const unsigned char* raw = bt + C::kBBytes;
+                const __half* sst = reinterpret_cast<const __half*>(raw + C::kRawBytes);
+#pragma unroll
+                for (int q = 0; q < kChunks; ++q) {
+                    const int idx = dt + q * kDeqWarps * 32;
+                    const int n = idx >> 3, c = idx & 7;
+                    const uint32_t v = *reinterpret_cast<const uint32_t*>(raw + n * 32 + c * 4);
+                    const float sc = a.scale_tma ? __half2float(sst[n * 8 + ((kb * 2 + c / 4) & 7)]) : sc0[q];
+                    *reinterpret_cast<uint4*>(bt + n * 128 + ((c ^ (n & 7)) << 4)) = dequant8(v, sc, dk);
+                }
+                fence_proxy_async_smem();      // generic-proxy writes -> tensor-core reads
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(bready0 + 8u * (uint32_t)s);
+#pragma unroll
+                for (int q = 0; q < kChunks; ++q) {
+                    sc0[q] = sc1[q];
+                    sc1[q] = sc2[q];
+                }
+            }
+            if (!ok) break;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();                  // no CTA leaves while the pair's MMAs may read its shared memory
+    tc_fence_after();
+    if (warp == kMmaWarp) tmem_dealloc2(tmem_base, C::kTmemCols);
+}
+
+template <int BNP>
+bool setup_pair_kernel(size_t* smem)
+{
+    *smem = PairCfg<BNP>::kSmem;
+    const void* fn = reinterpret_cast<const void*>(&gemm_pair_kernel<BNP>);
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 0) != cudaSuccess) {
+        cudaGetLastError();
+    }
+    return blocks_per_sm(fn, kThreads, *smem) >= 1;
+}
+
 template <int MA, int BN>
 bool setup_kernel(size_t* smem)
 {
@@ -420,9 +761,73 @@ bool setup_kernel(size_t* smem)
 
 }  // namespace
 
+namespace {
+
+// The CTA-pair kernel with BNP output columns per pair tile.
+template <int BNP>
+q4_status launch_gemm_pair(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed, const uint16_t* scales,
+                           int64_t N, uint16_t* y, cudaStream_t stream, const DeviceInfo& dev)
+{
+    constexpr int BH = BNP / 2;
+    CUtensorMap tm_x, tm_codes;
+    if (!encode_tma_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_UINT16, x, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, kBK, 128,
+                       CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_tma_2d(&tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2,
+                       kBK / 2, (uint32_t)BH, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return Q4_ERR_CUDA;
+    CUtensorMap tm_scales = tm_codes;
+    const bool scale_tma = (K / 32) % 8 == 0 && (reinterpret_cast<uintptr_t>(scales) & 15) == 0;
+    if (scale_tma && !encode_tma_2d(&tm_scales, CU_TENSOR_MAP_DATA_TYPE_UINT16, scales, (uint64_t)(K / 32),
+                                    (uint64_t)N, (uint64_t)(K / 32) * 2, 8, (uint32_t)BH, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return Q4_ERR_CUDA;
+    unsigned* err = device_error_word();
+    if (!err) return Q4_ERR_CUDA;
+    GemmArgs a;
+    a.scales = scales;
+    a.scale_tma = scale_tma ? 1 : 0;
+    a.y = y;
+    a.err = err;
+    a.M = (int)M;
+    a.N = (int)N;
+    a.K = (int)K;
+    a.G = (int)(K / 32);
+    a.tiles_m = (int)((M + 255) / 256);
+    a.tiles_n = (int)((N + BNP - 1) / BNP);
+    a.kblocks = (int)((K + kBK - 1) / kBK);
+    const long long tiles = (long long)a.tiles_m * a.tiles_n;
+    size_t smem = 0;
+    if (!setup_pair_kernel<BNP>(&smem)) return Q4_ERR_CUDA;
+    const long long clusters = std::min<long long>(tiles, dev.sm_count / 2);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(2 * clusters));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 2;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel<BNP>, tm_x, tm_codes, tm_scales, a);
+    return e == cudaSuccess ? Q4_OK : Q4_ERR_CUDA;
+}
+
+}  // namespace
+
 q4_status launch_gemm(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed, const uint16_t* scales,
                       int64_t N, uint16_t* y, cudaStream_t stream, const DeviceInfo& dev)
 {
+    // CTA pairs (256-row tiles) from M = 256 on: 256 x 256 pair tiles when they give every
+    // pair of SMs a tile, else 256 x 128.
+    if (M >= 256 && dev.sm_count >= 2) {
+        const long long p256 = ((M + 255) / 256) * ((N + 255) / 256);
+        if (p256 >= dev.sm_count / 2) return launch_gemm_pair<256>(x, M, K, packed, scales, N, y, stream, dev);
+        return launch_gemm_pair<128>(x, M, K, packed, scales, N, y, stream, dev);
+    }
     // Tile shape: 256 x 128 when that still gives every SM a tile, else 128 x 128, else 128 x 64.
     const long long t256 = ((M + 255) / 256) * ((N + 127) / 128);
     const long long t128 = ((M + 127) / 128) * ((N + 127) / 128);

@@ -24,9 +24,11 @@ def bf16_bits_to_f64(b):
 
 def run_gemm(x_bits, packed, scales):
     import bit_weight_only_quantize_b200 as q4
+    from bit_weight_only_quantize_b200 import _lib
     x = torch.from_numpy(x_bits.view(np.int16)).view(torch.bfloat16).cuda()
     y = q4.gemm(x, torch.from_numpy(packed).cuda(), torch.from_numpy(scales.view(np.int16)).cuda())
     torch.cuda.synchronize()
+    assert _lib.device_error() == 0        # no bounded wait ran out
     return bf16_bits_to_f64(y.view(torch.int16).cpu().numpy().view(np.uint16))
 
 
