@@ -821,11 +821,13 @@ q4_status launch_gemm_pair(const uint16_t* x, int64_t M, int64_t K, const uint8_
 q4_status launch_gemm(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed, const uint16_t* scales,
                       int64_t N, uint16_t* y, cudaStream_t stream, const DeviceInfo& dev)
 {
-    // CTA pairs (256-row tiles) from M = 256 on: 256 x 256 pair tiles when they give every
-    // pair of SMs a tile, else 256 x 128.
+    // CTA pairs (256-row tiles) from M = 256 on.  A 256 x 128 pair tile is bound by the
+    // latency of its stage ring (measured on B200: about 0.45 us per 64-k block against
+    // 0.55 us for a 256 x 256 tile, which does twice the work), so 256 x 256 tiles are
+    // used whenever they occupy at least half of the SM pairs.
     if (M >= 256 && dev.sm_count >= 2) {
         const long long p256 = ((M + 255) / 256) * ((N + 255) / 256);
-        if (p256 >= dev.sm_count / 2) return launch_gemm_pair<256>(x, M, K, packed, scales, N, y, stream, dev);
+        if (2 * p256 >= dev.sm_count / 2) return launch_gemm_pair<256>(x, M, K, packed, scales, N, y, stream, dev);
         return launch_gemm_pair<128>(x, M, K, packed, scales, N, y, stream, dev);
     }
     // Tile shape: 256 x 128 when that still gives every SM a tile, else 128 x 128, else 128 x 64.

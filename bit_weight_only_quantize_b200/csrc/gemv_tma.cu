@@ -1,5 +1,5 @@
 // q4_gemv / q4_gemv_multi for the shapes the TMA path serves (K % 256 == 0, scales
-// 16-byte aligned; M = 1 with f32 or bf16 x, M = 1..16 with bf16 x).
+// 16-byte aligned; M = 1 with f32 or bf16 x, M = 2..16 with bf16 x).
 //
 // Decode streams every weight once, so the kernels are built around keeping HBM busy
 // and spending few instructions per weight (QORA-LLM-0.8B model card, section "AVX-512
@@ -17,16 +17,22 @@
 //    Skinny shapes may also split K across blocks (last-arriver reduction, no
 //    waiting).  The plan picks splits, P and teams per block with a small cost model.
 //  * Arithmetic per mode:
-//      f32 x, M = 1:  nibble p OR-ed into the mantissa of 2^(23-4p) is exactly
-//                     2^(23-4p) + code; a packed f32x2 add leaves code - 8; packed
-//                     f32x2 FMAs accumulate each group in f32.  Two lanes per row.
-//      bf16 x, M = 1..16: nibble pair (j, j+4) of a word OR-ed into 0x4300 (one LOP3)
-//                     is the bf16 pair (128 + c_j, 128 + c_{j+4}); such pairs, read
-//                     with ldmatrix, are the A operand of mma.sync.m16n8k16 (f32
-//                     accumulate) and x rows the B operand, in a permuted k order that
-//                     matches the pairs.  The MMA's C operand is -136 * sum(x) of the
-//                     group (an f64 sum rounded once), so each result is the exact
-//                     group dot product up to f32 accumulation.
+//      M = 1 (kImma1, f32 or bf16 x): no code becomes a float.  Each group of 32 x values
+//          is scaled by a power of two 2^F_g (max |x| of the group * 2^F_g < 2^30),
+//          rounded once to integers and cut into four balanced base-256 digit planes;
+//          the codes stay bytes (even k as is, odd k at 16 x code, one AND each) and
+//          mma.sync.m16n8k32 (u8 codes x s8 digits) sums code x digit exactly in int32,
+//          the eight B columns being (plane, even/odd half).  The C operand, a bias
+//          0x4B400000 minus 8 (or 128) x the digit sum, removes the code offset 8 and
+//          makes the int32 result the bit pattern of the exact float 1.5 * 2^23 + sum.
+//          Each group's sum is multiplied by its scale times 2^-F_g and accumulated in
+//          f32 per plane; the planes are combined at the end.
+//      M = 2..16 (bf16 x): nibble pair (j, j+4) of a word OR-ed into 0x4300 (one LOP3)
+//          is the bf16 pair (128 + c_j, 128 + c_{j+4}); such pairs, read with ldmatrix,
+//          are the A operand of mma.sync.m16n8k16 (f32 accumulate) and x rows the B
+//          operand, in a permuted k order that matches the pairs.  The MMA's C operand
+//          is -136 * sum(x) of the group (an f64 sum rounded once), so each result is
+//          the exact group dot product up to f32 accumulation.
 //    In every mode each group's sum is scaled by its binary16 scale and added in f32.
 //  * Every mbarrier wait is bounded.  If one runs out the kernel records
 //    kErrWaitTimeout in the library error word, stops issuing and computing, waits
@@ -59,8 +65,8 @@ constexpr double kEpilogueCost = 0.1;
 constexpr double kSplitCost = 0.9;
 constexpr size_t kCounterBytes = kCounterSlots * sizeof(unsigned);
 
-// kImma1: one x row (f32 or bf16) through int8 tensor-core MMAs on exact digit planes of x.
-enum Mode { kF32M1 = 0, kMma8 = 1, kMma16 = 2, kMma1 = 3, kImma1 = 4 };   // kMma1: kMma8 with one x row
+// kImma1: one x row on the integer tensor cores; kMma8 / kMma16: 2..8 / 9..16 bf16 x rows.
+enum Mode { kMma8 = 1, kMma16 = 2, kImma1 = 4 };
 
 struct TmaMaps {
     CUtensorMap codes[Q4_MULTI_MAX];
@@ -118,15 +124,6 @@ __device__ __forceinline__ int matrix_of(const TmaGemvArgs& a, int rb)
     return m;
 }
 
-// A value the compiler must keep in a register (it cannot rematerialise it as an
-// immediate); used for the packed-add constants so they are not rebuilt per use.
-__device__ __forceinline__ float pinned(float v)
-{
-    float r;
-    asm volatile("mov.b32 %0, %1;" : "=f"(r) : "f"(v));
-    return r;
-}
-
 // (a & m) | c as one LOP3; m and c are kept in registers (pinned) by the callers, since the
 // instruction takes a single immediate.
 __device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t m, uint32_t c)
@@ -141,38 +138,6 @@ __device__ __forceinline__ uint32_t pinned_u32(uint32_t v)
     uint32_t r;
     asm volatile("mov.b32 %0, %1;" : "=r"(r) : "r"(v));
     return r;
-}
-
-// Constants of word_dot_f32 held in registers: the offsets 2^(23-4p) + 8 to remove, the
-// nibble masks 0xF << 4i and the exponents 2^(23-4i) a nibble at bit 4i is OR-ed into.
-struct ExpandConsts {
-    float2 c01, c23, c45, c67;
-    uint32_t mask[5], magic[5];
-};
-
-// f32 x: eight codes of one word dotted with eight x values (exact code - 8).
-__device__ __forceinline__ float2 word_dot_f32(uint32_t v, const float4* xw, const ExpandConsts& k)
-{
-    const uint32_t u = v >> 12;
-    const float f0 = __uint_as_float(and_or(v, k.mask[0], k.magic[0]));   // 2^23 + c0
-    const float f1 = __uint_as_float(and_or(v, k.mask[1], k.magic[1]));   // 2^19 + c1
-    const float f2 = __uint_as_float(and_or(v, k.mask[2], k.magic[2]));   // 2^15 + c2
-    const float f3 = __uint_as_float(and_or(v, k.mask[3], k.magic[3]));   // 2^11 + c3
-    const float f4 = __uint_as_float(and_or(v, k.mask[4], k.magic[4]));   // 2^7  + c4
-    const float f5 = __uint_as_float(and_or(u, k.mask[2], k.magic[2]));   // 2^15 + c5
-    const float f6 = __uint_as_float(and_or(u, k.mask[3], k.magic[3]));   // 2^11 + c6
-    const float f7 = __uint_as_float(and_or(u, k.mask[4], k.magic[4]));   // 2^7  + c7
-    const float2 d01 = __fadd2_rn(make_float2(f0, f1), k.c01);
-    const float2 d23 = __fadd2_rn(make_float2(f2, f3), k.c23);
-    const float2 d45 = __fadd2_rn(make_float2(f4, f5), k.c45);
-    const float2 d67 = __fadd2_rn(make_float2(f6, f7), k.c67);
-    const float4 xa = xw[0];
-    const float4 xb = xw[1];
-    float2 acc = __fmul2_rn(make_float2(xa.x, xa.y), d01);
-    acc = __ffma2_rn(make_float2(xa.z, xa.w), d23, acc);
-    acc = __ffma2_rn(make_float2(xb.x, xb.y), d45, acc);
-    acc = __ffma2_rn(make_float2(xb.z, xb.w), d67, acc);
-    return acc;
 }
 
 // Nibble pair (j, j+4) of a word as the bf16 pair (128 + c_j, 128 + c_{j+4}); mask and
@@ -252,9 +217,47 @@ __device__ __forceinline__ double sum8_bf16(const uint4 raw)
     return s;
 }
 
+// Eight x values (k = 8t .. 8t+7 of a group) as balanced base-256 digit planes of
+// X = rint(v * x_scale) (|X| < 2^30): X = d0 2^24 + d1 2^16 + d2 2^8 + d3, d1..d3 in
+// [-128, 127].  The digits' bytes are bytes of X plus carries: d3 = byte 0 of X, d2 = byte
+// 1 of X + 0x80, d1 = byte 2 of X + 0x8080, d0 = byte 3 of X + 0x808080 (each read as a
+// signed byte).  word[p][h] packs plane p's digits of k = 8t + h, + 2, + 4, + 6 (byte i =
+// k 8t + 2i + h); dsum[p][h] is their sum.
+__device__ __forceinline__ void digits8(const float (&v)[8], float x_scale, uint32_t (&word)[4][2], int (&dsum)[4][2])
+{
+    int X[8], Y1[8], Y2[8], Y3[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        X[e] = __float2int_rn(__fmul_rn(v[e], x_scale));
+        Y1[e] = (int)((uint32_t)X[e] + 0x80u);        // wraps (defined) only for non-finite x
+        Y2[e] = (int)((uint32_t)X[e] + 0x8080u);
+        Y3[e] = (int)((uint32_t)X[e] + 0x808080u);
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        word[3][h] = __byte_perm(__byte_perm(X[h], X[h + 2], 0x0040), __byte_perm(X[h + 4], X[h + 6], 0x0040), 0x5410);
+        word[2][h] = __byte_perm(__byte_perm(Y1[h], Y1[h + 2], 0x0051), __byte_perm(Y1[h + 4], Y1[h + 6], 0x0051), 0x5410);
+        word[1][h] = __byte_perm(__byte_perm(Y2[h], Y2[h + 2], 0x0062), __byte_perm(Y2[h + 4], Y2[h + 6], 0x0062), 0x5410);
+        word[0][h] = __byte_perm(__byte_perm(Y3[h], Y3[h + 2], 0x0073), __byte_perm(Y3[h + 4], Y3[h + 6], 0x0073), 0x5410);
+        int s0 = 0, s1 = 0, s2 = 0, s3 = 0;
+#pragma unroll
+        for (int e = h; e < 8; e += 2) {
+            const int x1 = Y1[e] >> 8, x2 = Y2[e] >> 16, x3 = Y3[e] >> 24;   // arithmetic shifts
+            s3 += (int)((uint32_t)X[e] - ((uint32_t)x1 << 8));
+            s2 += (int)((uint32_t)x1 - ((uint32_t)x2 << 8));
+            s1 += (int)((uint32_t)x2 - ((uint32_t)x3 << 8));
+            s0 += x3;
+        }
+        dsum[0][h] = s0;
+        dsum[1][h] = s1;
+        dsum[2][h] = s2;
+        dsum[3][h] = s3;
+    }
+}
+
 template <int MODE>
 struct ModeCfg {
-    static constexpr int MP = MODE == kMma16 ? 16 : (MODE == kMma8 || MODE == kMma1) ? 8 : 1;   // x rows in red[]
+    static constexpr int MP = MODE == kMma16 ? 16 : MODE == kMma8 ? 8 : 1;   // x rows in red[]
     static constexpr int NT = MP >= 8 ? MP / 8 : 1;                          // n-tiles of 8 x rows
     static constexpr int kMinBlocks = 1;
 };
@@ -272,10 +275,9 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
     constexpr bool kFuse = EPI == kEpiFuse;
     constexpr bool kArgmax = EPI == kEpiArgmax;
     constexpr bool kTopk = EPI == kEpiTopk;
-    constexpr int kTkM = (MODE == kF32M1 || MODE == kMma1 || MODE == kImma1) ? 1 : MP;   // x rows of a top-k list set
+    constexpr int kTkM = MODE == kImma1 ? 1 : MP;                         // x rows of a top-k list set
     extern __shared__ unsigned char smem_raw[];
     __shared__ int s_last[kMaxWarps];
-    __shared__ uint32_t s_xmax[kMaxWarps];
     const int W = blockDim.x >> 5;
     unsigned char* smem =
         reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -316,18 +318,6 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
         fence_mbar_init();
     }
     __syncwarp();
-    ExpandConsts kc = {};
-    if constexpr (MODE == kF32M1) {
-        kc.c01 = make_float2(pinned(-8388616.0f), pinned(-524296.0f));
-        kc.c23 = make_float2(pinned(-32776.0f), pinned(-2056.0f));
-        kc.c45 = make_float2(pinned(-136.0f), pinned(-32776.0f));
-        kc.c67 = make_float2(pinned(-2056.0f), pinned(-136.0f));
-#pragma unroll
-        for (int i = 0; i < 5; ++i) {
-            kc.mask[i] = pinned_u32(0xFu << (4 * i));
-            kc.magic[i] = pinned_u32((uint32_t)(150 - 4 * i) << 23);
-        }
-    }
 
     // Job j: unit (u0 + j % nbw) of the warp's (j / nbw)-th row block; a unit is up to
     // kBoxesPerStage consecutive code boxes plus one scale box spanning all of them.  Jobs
@@ -367,35 +357,40 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
         for (int j = 0; j < issued; ++j) issue(j);
 
     // ---- stage x for this split (zero past the split and past K) ----
-    //  kF32M1: f32 [group][32]
     //  kMma* : bf16 pairs [m][group][word][4] for m < M, then one zero row that lanes
     //          of x rows >= M read; each row is padded by one group so that lanes of
     //          neighbouring x rows fall on different banks.  Beside it, per group, -136 *
     //          sum(x) of the group for each x row (an f64 sum of the bf16 values, rounded
     //          once), laid out [group][n-tile][t] as the accumulator fragment of lane (g, t).
-    //  kImma1: x * 2^F rounded to an integer X (|X| < 2^30, F from max |x| of the split)
-    //          and cut into four balanced base-256 digits X = d0 2^24 + d1 2^16 + d2 2^8 + d3,
+    //  kImma1: each group g of 32 x values is scaled by 2^F_g (the largest F with
+    //          max |x| of the group * 2^F < 2^30, at most 100), rounded to integers X and
+    //          cut into four balanced base-256 digits X = d0 2^24 + d1 2^16 + d2 2^8 + d3,
     //          d1..d3 in [-128, 127].  The MMA's eight B columns are (digit plane p,
     //          nibble half h) = column 2p + h: half 0 holds the digits of the even k of
-    //          each group (the low nibbles), half 1 those of the odd k (the high nibbles,
+    //          the group (the low nibbles), half 1 those of the odd k (the high nibbles,
     //          which the A operand keeps at 16 x code).  [group pair][column g][t] uint4
     //          holds the two B registers of lane (g, t) for both groups of the pair, the
     //          slots of the other half zero.  Then [group pair][plane][4] int: the C
     //          operand per group and plane, bias - 8 sum(d of even k) for half 0 and
     //          bias - 128 sum(d of odd k) for half 1, which removes the code offset 8.
+    //          Then [group] float: 2^-F_g.  One pass: the four lanes of a group find its
+    //          maximum with two shuffles, so no block-wide reduction is needed.
     float* xoff = nullptr;
     const int rs = (ngp + 1) * 4;                                         // uint4 per staged x row
-    float plane_factor = 0.f;                                             // kImma1: 2^(-F + 8 (3 - t))
     if constexpr (MODE == kImma1) {
-        // Item i = (group i / 4, k = 8 (i % 4) .. + 7) of the split; a thread keeps the x
-        // of its first item in registers for both passes (max |x|, then the digits).
-        const int items = ngp * 4;
-        auto load8 = [&](int i, float (&v)[8]) {
+        const int items = ngp * 4;                                        // (group, k = 8t .. 8t+7)
+        uint2* xq = reinterpret_cast<uint2*>(xst);
+        int2* xc = reinterpret_cast<int2*>(xst + (size_t)ngp * 256);
+        float* xf = reinterpret_cast<float*>(xst + (size_t)ngp * 288);
+#pragma unroll 2
+        for (int i0 = threadIdx.x - lane; i0 < items; i0 += blockDim.x) {    // warp-uniform trips
+            const int i = i0 + lane;
+            const int lg = i >> 2, t = i & 3;
+            float v[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) v[e] = 0.f;
-            const int lg = i >> 2;
             if (i < items && lg < ng) {
-                const size_t k0 = (size_t)(g0 + lg) * 32 + (i & 3) * 8;
+                const size_t k0 = (size_t)(g0 + lg) * 32 + t * 8;
                 if (a.x_f32) {
                     const float4 p = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(a.x) + k0);
                     const float4 q = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(a.x) + k0 + 4);
@@ -410,55 +405,19 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
                     }
                 }
             }
-        };
-        // max |x| over the split (bit patterns of non-negative floats order as the values)
-        float v0[8];
-        load8(threadIdx.x, v0);
-        uint32_t mx = 0u;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) mx = max(mx, __float_as_uint(v0[e]) & 0x7FFFFFFFu);
-        for (int i = threadIdx.x + blockDim.x; i < items; i += blockDim.x) {
-            float v[8];
-            load8(i, v);
+            // the group's max |x| (bit patterns of non-negative floats order as the values)
+            uint32_t mx = 0u;
 #pragma unroll
             for (int e = 0; e < 8; ++e) mx = max(mx, __float_as_uint(v[e]) & 0x7FFFFFFFu);
-        }
-        mx = __reduce_max_sync(0xffffffffu, mx);
-        if (lane == 0) s_xmax[warp] = mx;
-        __syncthreads();
-        mx = 0u;
-        for (int w = 0; w < W; ++w) mx = max(mx, s_xmax[w]);
-        // F with max |x| * 2^F < 2^30; 100 for a zero or subnormal maximum, 0 for a
-        // non-finite one (the product is then undefined, but every step stays defined)
-        const int ex = (int)(mx >> 23);
-        const int F = ex == 0 ? 100 : ex >= 255 ? 0 : min(29 - (ex - 127), 100);
-        const float x_scale = __uint_as_float((uint32_t)(F + 127) << 23);
-        plane_factor = __uint_as_float((uint32_t)(-F + 24 - 8 * (lane & 3) + 127) << 23);
-        uint2* xq = reinterpret_cast<uint2*>(xst);
-        int2* xc = reinterpret_cast<int2*>(xst + (size_t)ngp * 256);
-        for (int i0 = threadIdx.x - lane; i0 < items; i0 += blockDim.x) {    // warp-uniform trips
-            const int i = i0 + lane;
-            const int lg = i >> 2, t = i & 3;                                  // group, k = 8t .. 8t+7
-            float v[8];
-            if (i0 == threadIdx.x - lane) {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) v[e] = v0[e];
-            } else {
-                load8(i, v);
-            }
-            uint32_t word[4][2] = {};                                          // [plane][half]
-            int dsum[4][2] = {};
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                int r = __float2int_rn(__fmul_rn(v[e], x_scale));
-#pragma unroll
-                for (int p = 3; p >= 0; --p) {
-                    const int d = p == 0 ? r : (int)((uint32_t)r << 24) >> 24;
-                    if (p > 0) r = (int)((uint32_t)r - (uint32_t)d) >> 8;
-                    word[p][e & 1] |= ((uint32_t)d & 0xFFu) << (8 * (e >> 1));
-                    dsum[p][e & 1] += d;
-                }
-            }
+            mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+            mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+            // F_g: 100 for a zero or subnormal maximum, 0 for a non-finite one (the product
+            // is then undefined, but every step stays defined)
+            const int ex = (int)(mx >> 23);
+            const int F = ex == 0 ? 100 : ex >= 255 ? 0 : min(29 - (ex - 127), 100);
+            uint32_t word[4][2];
+            int dsum[4][2];
+            digits8(v, __uint_as_float((uint32_t)(F + 127) << 23), word, dsum);
 #pragma unroll
             for (int p = 0; p < 4; ++p)
 #pragma unroll
@@ -475,16 +434,8 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
                     if (t == 0)
                         xc[((gp * 4 + p) << 1) + half] = make_int2(kBiasBits - 8 * dsum[p][0], kBiasBits - 128 * dsum[p][1]);
                 }
+                if (t == 0) xf[lg] = __uint_as_float((uint32_t)(127 - F) << 23);
             }
-        }
-    } else if constexpr (MODE == kF32M1) {
-        float4* xf = reinterpret_cast<float4*>(xst);
-        for (int i = threadIdx.x; i < ngp * 8; i += blockDim.x) {
-            const int lg = i >> 3, c = i & 7;
-            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (lg < ng)
-                v = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(a.x) + (size_t)(g0 + lg) * 32 + c * 4);
-            xf[i] = v;
         }
     } else {
         uint4* xp = reinterpret_cast<uint4*>(xst);
@@ -544,7 +495,7 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
     for (int rbi = 0; rbi < nrb; ++rbi) {
         const int rb = rb_of(rbi);
         if constexpr (kFloor) floor_now = load_key_relaxed(a.tk_floor);   // used in this block's epilogue
-        float yacc = 0.f;     // kF32M1: row (lane & 15), half (lane >> 4); kImma1: row g, plane t
+        float yacc = 0.f;     // kImma1: row g, plane t
         float yacc8 = 0.f;    // kImma1: row g + 8, plane t
         float acc[NT][4];     // MMA modes: rows g, g+8; x rows n*8 + 2t, +1
 #pragma unroll
@@ -578,6 +529,9 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
                                 smem_addr(cb) + ((li & 1) * 8 + lr) * 128 + (((li >> 1) ^ lr) << 4);
                             const uint4* xq = reinterpret_cast<const uint4*>(xst) + ((gb >> 1) * 8 + g) * 4 + t;
                             const int4* xc = reinterpret_cast<const int4*>(xst + (size_t)ngp * 256) + (gb >> 1) * 4 + t;
+                            const float4* xf = reinterpret_cast<const float4*>(xst + (size_t)ngp * 288) + (gb >> 2);
+                            const float4 f0 = xf[0], f1 = xf[1];     // 2^-F_g of the box's 8 groups
+                            const float fgs[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
 #pragma unroll
                             for (int cp = 0; cp < 4; ++cp) {
                                 uint32_t r0, r1, r2, r3;
@@ -600,21 +554,9 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
                                         fmaf(__int_as_float(d[1]), 0.0625f, __int_as_float(d[0])) - kBias17;
                                     const float u1 =
                                         fmaf(__int_as_float(d[3]), 0.0625f, __int_as_float(d[2])) - kBias17;
-                                    yacc = fmaf(scale_at(sg, c), u0, yacc);
-                                    yacc8 = fmaf(scale_at(sg8, c), u1, yacc8);
+                                    yacc = fmaf(scale_at(sg, c) * fgs[c], u0, yacc);
+                                    yacc8 = fmaf(scale_at(sg8, c) * fgs[c], u1, yacc8);
                                 }
-                            }
-                        } else if constexpr (MODE == kF32M1) {
-                            const int r = lane & 15, h = lane >> 4;
-                            const unsigned char* rowp = cb + r * 128 + h * 8;
-                            const uint4 s8 = *reinterpret_cast<const uint4*>(sb + r * kScaleRow);
-#pragma unroll
-                            for (int c = 0; c < 8; ++c) {
-                                const uint2 w2 = *reinterpret_cast<const uint2*>(rowp + ((c ^ (r & 7)) << 4));
-                                const float4* xg = reinterpret_cast<const float4*>(xst) + (gb + c) * 8 + h * 4;
-                                const float2 d2 =
-                                    __fadd2_rn(word_dot_f32(w2.x, xg, kc), word_dot_f32(w2.y, xg + 2, kc));
-                                yacc = fmaf(scale_at(s8, c), d2.x + d2.y, yacc);
                             }
                         } else {
                             const int g = lane >> 2, t = lane & 3;
@@ -665,10 +607,8 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
                                     for (int n = 0; n < NT; ++n) {
                                         acc[n][0] = fmaf(s0, d[c - c0][n][0], acc[n][0]);
                                         acc[n][2] = fmaf(s1, d[c - c0][n][2], acc[n][2]);
-                                        if constexpr (MODE != kMma1) {          // columns 2t + 1
-                                            acc[n][1] = fmaf(s0, d[c - c0][n][1], acc[n][1]);
-                                            acc[n][3] = fmaf(s1, d[c - c0][n][3], acc[n][3]);
-                                        }
+                                        acc[n][1] = fmaf(s0, d[c - c0][n][1], acc[n][1]);
+                                        acc[n][3] = fmaf(s1, d[c - c0][n][3], acc[n][3]);
                                     }
                                 }
                             }
@@ -689,7 +629,9 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
         // ---- row block rb complete: partials -> red[warp][row][m], team sum in warp order ----
         float* my_red = red + warp * kRows * MP;
         if constexpr (MODE == kImma1) {
-            // planes t = 0..3 of rows g and g+8 scaled by 2^(-F + 8 (3 - t)) and summed
+            // planes t = 0..3 of rows g and g+8 scaled by 2^(8 (3 - t)) and summed (the
+            // groups' 2^-F_g went in with their scales)
+            const float plane_factor = __uint_as_float((uint32_t)(24 - 8 * (lane & 3) + 127) << 23);
             float v0 = yacc * plane_factor, v1 = yacc8 * plane_factor;
             v0 += __shfl_xor_sync(0xffffffffu, v0, 1);
             v1 += __shfl_xor_sync(0xffffffffu, v1, 1);
@@ -699,9 +641,6 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
                 my_red[lane >> 2] = v0;
                 my_red[(lane >> 2) + 8] = v1;
             }
-        } else if constexpr (MODE == kF32M1) {
-            yacc += __shfl_xor_sync(0xffffffffu, yacc, 16);           // the two halves of each row
-            if (lane < 16) my_red[lane] = yacc;
         } else {
             const int g = lane >> 2, t = lane & 3;
 #pragma unroll
@@ -923,16 +862,16 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
 
 size_t per_warp_bytes(int mode)
 {
-    const int mp = mode == kMma16 ? 16 : (mode == kMma8 || mode == kMma1) ? 8 : 1;
+    const int mp = mode == kMma16 ? 16 : mode == kMma8 ? 8 : 1;
     return (size_t)kStages * (kStageCodes + kStageScales + sizeof(uint64_t)) + (size_t)kRows * mp * sizeof(float);
 }
 
 size_t x_stage_bytes(int mode, int nb, int64_t M)
 {
-    const int mp = mode == kMma16 ? 16 : (mode == kMma8 || mode == kMma1) ? 8 : 1;
+    const int mp = mode == kMma16 ? 16 : mode == kMma8 ? 8 : 1;
     const size_t ngp = (size_t)nb * 8;
-    if (mode == kImma1) return ngp * 288;                  // B operands 256 B + C operands 32 B per group
-    return mode == kF32M1 ? ngp * 32 * sizeof(float) : (size_t)(M + 1) * (ngp + 1) * 64 + ngp * (mp / 8) * 64;
+    if (mode == kImma1) return ngp * 292;      // per group: B operands 256 B, C operands 32 B, 2^-F_g 4 B
+    return (size_t)(M + 1) * (ngp + 1) * 64 + ngp * (mp / 8) * 64;
 }
 
 size_t smem_bytes(int mode, int warps, int nb, int64_t M)
@@ -950,9 +889,7 @@ template <int EPI>
 const void* kernel_for_epi(int mode)
 {
     switch (mode) {
-    case kF32M1: return reinterpret_cast<const void*>(&gemv_tma_kernel<kF32M1, EPI>);
     case kMma8: return reinterpret_cast<const void*>(&gemv_tma_kernel<kMma8, EPI>);
-    case kMma1: return reinterpret_cast<const void*>(&gemv_tma_kernel<kMma1, EPI>);
     case kImma1: return reinterpret_cast<const void*>(&gemv_tma_kernel<kImma1, EPI>);
     default: return reinterpret_cast<const void*>(&gemv_tma_kernel<kMma16, EPI>);
     }

@@ -148,10 +148,10 @@ Q4_API size_t q4_gemv_workspace_size(int64_t M, int64_t N, int64_t K);
  *              must start at zero (the arrival counters) at zero again, so the
  *              same workspace can be reused by later calls without clearing.
  *              Calls that share a workspace must not overlap on the GPU.
- * Arithmetic.  M = 1 (f32 or bf16 x): x is scaled by a power of two 2^F with
- * max |x| * 2^F < 2^30 (F from the x of each K split), rounded once to an integer and
- * cut into four base-256 digits; the codes times the digits are summed exactly on the
- * integer tensor cores per group, and each group's sum is multiplied by its scale and
+ * Arithmetic.  M = 1 (f32 or bf16 x): each group of 32 x values is scaled by a power of
+ * two 2^F_g with max |x| * 2^F_g < 2^30, rounded once to integers and cut into four
+ * base-256 digits; the codes times the digits are summed exactly on the integer tensor
+ * cores per group, and each group's sum is multiplied by its scale times 2^-F_g and
  * accumulated in f32 (per digit plane, combined at the end).  M >= 2 with bf16 x: the
  * codes are expanded exactly and multiplied by x on the bf16 tensor cores with f32
  * accumulation, each group's sum scaled and accumulated in f32.  Other shapes (f32 x

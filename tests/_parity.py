@@ -34,10 +34,9 @@ def rel_inf(y: np.ndarray, ref: np.ndarray) -> float:
 
 
 # Unit roundoffs of the two kinds of f32 sums the kernels make.  A CUDA-core f32 add or
-# FMA rounds to nearest (u = 2^-24).  An f32 accumulation inside an mma.sync tensor-core
-# instruction is not specified to round to nearest; the tests take the truncating
-# (round-toward-zero) model for every such sum, bf16 and binary16 operands alike:
-# u = 2^-23.
+# FMA rounds to nearest (u = 2^-24).  An f32 accumulation inside a tensor-core MMA
+# instruction (the binary16 GEMV) is not specified to round to nearest; the tests take
+# the truncating (round-toward-zero) model for every such sum: u = 2^-23.
 U_CUDA_CORE = 2.0 ** -24
 U_TENSOR_F32 = 2.0 ** -23
 
@@ -70,9 +69,10 @@ def offset_path_bound(x: np.ndarray, scales: np.ndarray, roundings: int) -> np.n
     return gamma(roundings, U_TENSOR_F32) * (xa @ (144.0 * s).T)
 
 
-def digit_shift(x_row: np.ndarray) -> int:
-    """The power of two F the M = 1 path scales x by: max |x| * 2^F < 2^30 (F <= 100)."""
-    mx = float(np.max(np.abs(x_row))) if x_row.size else 0.0
+def digit_shift(x_group: np.ndarray) -> int:
+    """The power of two F the M = 1 path scales a group of x by: max |x| * 2^F < 2^30
+    (F <= 100)."""
+    mx = float(np.max(np.abs(x_group))) if x_group.size else 0.0
     if mx == 0.0 or mx < 2.0 ** -126:
         return 100
     e = int(np.floor(np.log2(mx)))
@@ -84,17 +84,17 @@ def digit_shift(x_row: np.ndarray) -> int:
 
 
 def digit_path_bound(x: np.ndarray, deq: np.ndarray, roundings: int) -> np.ndarray:
-    """Bound for the M = 1 path.  x is rounded once to the integer X = rint(x 2^F) (error
-    <= 2^(-F-1) per element) and cut into four base-256 digit planes X_p; the integer MMAs
-    are exact, and plane p's f32 sum (CUDA-core FMAs of scale x exact group sums) is
-    bounded by gamma_n sum_k |w'_k| |X_p,k|.  Scaled back by 2^(-F + 8 (3 - p)) and summed
-    over p this is at most gamma_n sum_k |w'_k| (|x_k| + 1.01 * 2^(24 - F)).  Split-K
-    splits take F from their own part of x, which only shrinks both terms."""
+    """Bound for the M = 1 path (K % 256 == 0).  Each group of 32 x values is rounded once
+    to integers X = rint(x 2^F_g) (error <= 2^(-F_g-1) per element) and cut into four
+    base-256 digit planes X_p; the integer MMAs are exact, and plane p's f32 sum
+    (CUDA-core FMAs of scale 2^-F_g x exact group sums) is bounded by
+    gamma_n sum_k |w'_k| |X_p,k| 2^-F_g.  Scaled by 2^(8 (3 - p)) and summed over p this
+    is at most gamma_n sum_k |w'_k| (|x_k| + 1.01 * 2^(24 - F_g))."""
     xs = x_f64(x)
     wa = np.abs(deq)
-    out = np.empty((xs.shape[0], deq.shape[0]))
-    for m in range(xs.shape[0]):
-        q = 2.0 ** -digit_shift(xs[m])
-        rows = wa.sum(axis=1)
-        out[m] = 0.5 * q * rows + gamma(roundings, U_CUDA_CORE) * (wa @ (np.abs(xs[m]) + 1.01 * 2.0 ** 24 * q))
+    M, K = xs.shape
+    out = np.empty((M, deq.shape[0]))
+    for m in range(M):
+        q = np.repeat(np.array([2.0 ** -digit_shift(xs[m, g:g + 32]) for g in range(0, K, 32)]), 32)
+        out[m] = wa @ (0.5 * q) + gamma(roundings, U_CUDA_CORE) * (wa @ (np.abs(xs[m]) + 1.01 * 2.0 ** 24 * q))
     return out

@@ -37,11 +37,11 @@ def check(x, W, x_dtype, tight=True):
     err = rel_inf(y, ref)
     assert err <= TOL[x_dtype], err
     if tight:
-        # the bound of the path the shape takes: M = 1 runs on exact integer digit planes
-        # of x (any K), M >= 2 with bf16 x on the tensor cores with an offset, f32 x with
-        # M >= 2 on CUDA-core FMAs (the fallback kernel)
+        # the bound of the path the shape takes: M = 1 with K % 256 == 0 runs on exact
+        # integer digit planes of x, M >= 2 with bf16 x and K % 256 == 0 on the bf16
+        # tensor cores with an offset, every other shape on CUDA-core FMAs (the fallback)
         n, deq = roundings(W.shape[1]), oracle.dequantize(packed, scales)
-        if x.shape[0] == 1 and W.shape[1] % 256 == 0:
+        if W.shape[1] % 256 == 0 and x.shape[0] == 1:
             bound = digit_path_bound(x, deq, n)
         else:
             bound = f32_sum_bound(x, deq, n)
