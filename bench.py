@@ -569,6 +569,58 @@ def measure_rows(torch, q4, lib, device, peaks, l2):
                                   "frac_hbm": b / ms / 1e6 / hbm, "bytes": b}
     del cs
 
+    # INT8 weights at the LM-head shape (642 MB, far above L2).
+    N = synth_inputs.LM_HEAD.N
+    W8 = torch.from_numpy(synth_inputs.weights("normal", N, K, 0)).to(device)
+    codes, sc8 = q4.int8_quantize(W8)
+    del W8
+    yl = torch.empty((1, N), dtype=torch.float32, device=device)
+
+    def i8l(i):
+        st = lib.q4_int8_gemv(x8.data_ptr(), 1, 1, K, codes.data_ptr(), sc8.data_ptr(), N, yl.data_ptr(),
+                              stream.cuda_stream)
+        assert st == 0
+    log("rows: int8 gemv lm head")
+    ms = time_launches(torch, i8l, 10, device, stream)
+    b = N * K + N * (K // 32) * 2 + K * 2 + N * 4
+    out["int8_gemv_lm_head"] = {"workload": f"INT8 weights M=1 K={K} N={N} bf16 x", "ms": ms, "GB/s": b / ms / 1e6,
+                                "frac_hbm": b / ms / 1e6 / hbm, "bytes": b}
+    del codes, sc8, yl
+
+    # A decode layer of mixed precision in one q4_gemv_mixed launch: attention q, k, v in
+    # INT8 (4096, 1024, 1024 rows) beside an MLP projection in Q4 (4096 rows), sharing x.
+    spec = [(4096, 8), (1024, 8), (1024, 8), (4096, 4)]
+    sets = []
+    setb = 0
+    for i, (n, bits) in enumerate(spec):
+        Wm = torch.from_numpy(synth_inputs.weights("outliers", n, K, i)).to(device)
+        c, sm = q4.int8_quantize(Wm) if bits == 8 else q4.quantize(Wm)
+        sets.append((c, sm, bits))
+        setb += c.numel() + sm.numel() * 2
+        del Wm
+    copies = rotating_copies(setb, l2)
+    allsets = [sets] + [[(c.clone(), sm.clone(), bits) for c, sm, bits in sets] for _ in range(copies - 1)]
+    ym = [torch.empty((1, n), dtype=torch.float32, device=device) for n, _ in spec]
+    wsm = torch.zeros(max(16, q4.gemv_mixed_workspace_size(1, K, spec)), dtype=torch.uint8, device=device)
+    arrs = []
+    for st_ in allsets:
+        arr = (L.MixedWeight * len(spec))()
+        for j, ((c, sm, bits), y) in enumerate(zip(st_, ym)):
+            arr[j] = L.MixedWeight(c.data_ptr(), sm.data_ptr(), c.shape[0], y.data_ptr(), bits, 0)
+        arrs.append((arr, ctypes.cast(arr, ctypes.c_void_p)))
+
+    def mixed(i):
+        st = lib.q4_gemv_mixed(x8.data_ptr(), 1, 1, K, arrs[i % copies][1], len(spec), L.WEIGHTS_STATIC,
+                               wsm.data_ptr(), wsm.numel(), stream.cuda_stream)
+        assert st == 0
+    log("rows: mixed int8/q4 layer")
+    ms = time_launches(torch, mixed, copies * 2, device, stream)
+    b = setb + K * 2 + sum(n for n, _ in spec) * 4
+    out["mixed_int8_q4_layer"] = {"workload": "q4_gemv_mixed M=1 K=2560: INT8 q/k/v (4096, 1024, 1024 rows) + Q4 "
+                                              "4096 rows, bf16 x, one launch", "ms": ms, "GB/s": b / ms / 1e6,
+                                  "frac_hbm": b / ms / 1e6 / hbm, "bytes": b, "l2": f"{copies} rotating weight sets"}
+    del allsets, arrs
+
     # Prefill q4_gemm (bf16 x, bf16 y, f32 accumulate); inputs rotated to exceed 3x L2.
     for gw in synth_inputs.PREFILL:
         _, packed, scales = make_quantized(torch, q4, gw, 0, device)
@@ -712,8 +764,8 @@ def run_reference(args, world, rank):
 
 # ---------------------------------------------------------------- ncu cases
 PROFILE_CASES = ["decode", "decode_small", "decode_multi", "lm_head", "lm_head_argmax", "lm_head_topk", "gemv_m2",
-                 "gemv_m4", "gemv_m8", "gemv_m16", "gate_up", "f16", "int8", "int8_quantize", "quantize", "gemm",
-                 "gemm_m2048", "gemm_m512", "topk_merge", "ffma"]
+                 "gemv_m4", "gemv_m8", "gemv_m16", "gate_up", "f16", "int8", "int8_m4", "int8_quantize", "quantize",
+                 "mixed", "gemm", "gemm_m2048", "gemm_m512", "topk_merge", "ffma"]
 
 
 def run_profile_case(args):
@@ -774,14 +826,24 @@ def run_profile_case(args):
         x = bf16_dev(torch, synth_inputs.activations(1, K, "bf16", 0), device)
         for _ in range(n):
             q4.f16_gemv(x, w16.view(torch.float16))
-    elif case == "int8":
+    elif case in ("int8", "int8_m4"):
         N, K = 4096 * 16, 2560                                            # 168 MB of codes > L2
         W8 = torch.from_numpy(synth_inputs.weights("normal", N, K, 0)).to(device)
         codes, sc8 = q4.int8_quantize(W8)
         del W8
-        x = bf16_dev(torch, synth_inputs.activations(1, K, "bf16", 0), device)
+        x = bf16_dev(torch, synth_inputs.activations(1 if case == "int8" else 4, K, "bf16", 0), device)
         for _ in range(n):
             q4.int8_gemv(x, codes, sc8)
+    elif case == "mixed":
+        K = 2560
+        mats = []
+        for i, (nr, bits) in enumerate([(4096, 8), (1024, 8), (1024, 8), (4096, 4)]):
+            Wm = torch.from_numpy(synth_inputs.weights("outliers", nr, K, i)).to(device)
+            c, sm = q4.int8_quantize(Wm) if bits == 8 else q4.quantize(Wm)
+            mats.append((c, sm, bits))
+        x = bf16_dev(torch, synth_inputs.activations(1, K, "bf16", 0), device)
+        for _ in range(n):
+            q4.gemv_mixed(x, mats, weights_static=True)
     elif case == "topk_merge":
         S, M, k = 8, 1, 20
         vals = torch.randn((S, M, k), device=device).sort(dim=-1, descending=True).values.contiguous()

@@ -17,7 +17,7 @@ from . import _lib
 from ._lib import Q4Error, FLAG_NONFINITE, FLAG_SCALE_OVERFLOW, GEMV_MAX_M  # noqa: F401
 
 __all__ = [
-    "quantize", "gemv", "gemv_host", "gemv_multi", "GemvMulti", "gemv_gate_up", "gemv_argmax", "gemv_topk",
+    "quantize", "gemv", "gemv_host", "gemv_multi", "gemv_mixed", "gemv_mixed_workspace_size", "GemvMulti", "gemv_gate_up", "gemv_argmax", "gemv_topk",
     "gemv_topk_workspace_size", "topk_merge", "f16_gemv", "int8_quantize", "int8_gemv", "gemm", "gemv_workspace_size", "gemv_multi_workspace_size",
     "Q4Error", "FLAG_NONFINITE", "FLAG_SCALE_OVERFLOW", "GEMV_MAX_M",
 ]
@@ -212,6 +212,71 @@ def gemv_host(x_host: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, 
                               _lib.WEIGHTS_STATIC if weights_static else 0, ws_ptr, ws_bytes, _stream())
     _lib.check(st, "q4_gemv_host")
     return y_host
+
+
+def _mixed_array(weights, outs):
+    arr = (_lib.MixedWeight * len(weights))()
+    for i, ((codes, scales, bits), y) in enumerate(zip(weights, outs)):
+        arr[i] = _lib.MixedWeight(codes.data_ptr(), scales.data_ptr(), codes.shape[0], y.data_ptr(), bits, 0)
+    return arr
+
+
+def gemv_mixed_workspace_size(M: int, K: int, Ns_bits) -> int:
+    """Workspace bytes of gemv_mixed for matrices [(N, bits), ...]."""
+    arr = (_lib.MixedWeight * len(Ns_bits))()
+    for i, (n, bits) in enumerate(Ns_bits):
+        arr[i] = _lib.MixedWeight(None, None, n, None, bits, 0)
+    return int(_lib.load().q4_gemv_mixed_workspace_size(M, K, ctypes.cast(arr, ctypes.c_void_p), len(Ns_bits)))
+
+
+def gemv_mixed(x: torch.Tensor, weights, outs=None, workspace: torch.Tensor | None = None,
+               weights_static: bool = False):
+    """y_i[M,N_i] (f32) = x . dequant(W_i)^T for matrices of mixed precision sharing x:
+    ``weights`` is a list of (codes, scales, bits) with bits 4 (Q4: codes uint8 [N, K/2]) or
+    8 (INT8: codes int8 [N, K]), scales binary16 bits as int16 [N, K/32]."""
+    if x.dtype == torch.float32:
+        xt = _lib.Q4_F32
+    elif x.dtype == torch.bfloat16:
+        xt = _lib.Q4_BF16
+    else:
+        raise TypeError("x must be float32 or bfloat16")
+    _need(x, "x", x.dtype, 2)
+    M, K = x.shape
+    if not 1 <= len(weights) <= _lib.MULTI_MAX:
+        raise ValueError(f"between 1 and {_lib.MULTI_MAX} weight matrices")
+    for codes, scales, bits in weights:
+        if bits == 4:
+            _need(codes, "codes", torch.uint8, 2, x.device)
+            if codes.shape[1] * 2 != K:
+                raise ValueError("Q4 codes must be [N, K/2]")
+        elif bits == 8:
+            _need(codes, "codes", torch.int8, 2, x.device)
+            if codes.shape[1] != K:
+                raise ValueError("INT8 codes must be [N, K]")
+        else:
+            raise ValueError("bits must be 4 or 8")
+        _need(scales, "scales", torch.int16, 2, x.device)
+        if tuple(scales.shape) != (codes.shape[0], K // 32):
+            raise ValueError("scales must be [N, K/32]")
+    if outs is None:
+        outs = [torch.empty((M, c.shape[0]), dtype=torch.float32, device=x.device) for c, _, _ in weights]
+    for y, (c, _, _) in zip(outs, weights):
+        _need(y, "out", torch.float32, 2, x.device)
+        if tuple(y.shape) != (M, c.shape[0]):
+            raise ValueError("out has the wrong shape")
+    arr = _mixed_array(weights, outs)
+    lib = _lib.load()
+    with _on(x.device):
+        if workspace is None:
+            need = gemv_mixed_workspace_size(M, K, [(c.shape[0], b) for c, _, b in weights])
+            if need:
+                workspace = torch.zeros(need, dtype=torch.uint8, device=x.device)
+        ws_ptr = workspace.data_ptr() if workspace is not None else None
+        ws_bytes = workspace.numel() if workspace is not None else 0
+        st = lib.q4_gemv_mixed(x.data_ptr(), xt, M, K, ctypes.cast(arr, ctypes.c_void_p), len(weights),
+                               _lib.WEIGHTS_STATIC if weights_static else 0, ws_ptr, ws_bytes, _stream())
+    _lib.check(st, "q4_gemv_mixed")
+    return outs
 
 
 def gemv_multi_workspace_size(M: int, K: int, Ns) -> int:

@@ -32,6 +32,12 @@ class Weight(ctypes.Structure):
     _fields_ = [("packed", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("N", ctypes.c_int64),
                 ("y", ctypes.c_void_p)]
 
+
+class MixedWeight(ctypes.Structure):
+    """struct q4_mixed_weight of include/q4.h."""
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("N", ctypes.c_int64),
+                ("y", ctypes.c_void_p), ("bits", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
 # Every symbol include/q4.h declares, with (restype, argtypes).
 _i64, _vp, _sz, _i32 = ctypes.c_int64, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
 SIGNATURES = {
@@ -54,6 +60,8 @@ SIGNATURES = {
                               _vp]),
     "q4_int8_quantize": (_i32, [_vp, _i64, _i64, _vp, _vp, _vp, _vp]),
     "q4_int8_gemv": (_i32, [_vp, _i32, _i64, _i64, _vp, _vp, _i64, _vp, _vp]),
+    "q4_gemv_mixed_workspace_size": (_sz, [_i64, _i64, _vp, _i32]),
+    "q4_gemv_mixed": (_i32, [_vp, _i32, _i64, _i64, _vp, _i32, ctypes.c_uint32, _vp, _sz, _vp]),
     "q4_topk_merge": (_i32, [_vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp]),
     "q4_gemv_topk_workspace_size": (_sz, [_i64, _i64, _i64, _i64, _i32]),
     "q4_gemv_topk": (_i32, [_vp, _i32, _i64, _i64, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp, ctypes.c_uint32,

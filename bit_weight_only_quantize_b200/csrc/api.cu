@@ -415,11 +415,142 @@ q4_status q4_int8_gemv(const void* x, q4_dtype x_dtype, int64_t M, int64_t K, co
     if (st != Q4_OK) return st;
     if (M == 0 || N == 0) return Q4_OK;
     if (!x || !codes || !scales || !y) return Q4_ERR_INVALID_ARG;
-    if (misaligned(x, 4) || misaligned(codes, 16) || misaligned(scales, 2) || misaligned(y, 4)) return Q4_ERR_ALIGN;
+    if (misaligned(x, 16) || misaligned(codes, 16) || misaligned(scales, 2) || misaligned(y, 4)) return Q4_ERR_ALIGN;
     q4::DeviceInfo dev;
     if ((st = q4::current_device(&dev)) != Q4_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // M = 1: the TMA kernel's integer path (codes straight into the tensor cores), K whole
+    if (M == 1 && K % 256 == 0 && !misaligned(scales, 16)) {
+        const int fmt = 1;
+        const q4_weight w = {reinterpret_cast<const uint8_t*>(codes), scales, N, y};
+        q4::GemvPlan plan;
+        if (q4::plan_gemv_tma(M, &N, 1, K, x_dtype, dev, &plan, q4::kGemvPlain, &fmt, false))
+            return q4::launch_gemv_tma(x, x_dtype, M, K, &w, 1, 0, nullptr, plan, s, q4::kGemvPlain, nullptr, &fmt);
+        cudaGetLastError();
+    }
     if ((size_t)M * (size_t)K * sizeof(float) > (size_t)dev.max_smem_optin) return Q4_ERR_SHAPE;
-    return q4::launch_int8_gemv(x, x_dtype, M, K, codes, scales, N, y, static_cast<cudaStream_t>(stream), dev);
+    return q4::launch_int8_gemv(x, x_dtype, M, K, codes, scales, N, y, s, dev);
+}
+
+namespace {
+
+// Validates a mixed matrix list: N >= 0, bits 4 or 8, pointers and alignment of the kept
+// (N > 0) matrices.
+q4_status collect_mixed(const q4_mixed_weight* mats, int count, int64_t K, q4_mixed_weight* out, int* kept)
+{
+    if (!mats || count < 1 || count > Q4_MULTI_MAX) return Q4_ERR_INVALID_ARG;
+    int n = 0;
+    for (int i = 0; i < count; ++i) {
+        q4_status st = check_nk(mats[i].N, K);
+        if (st != Q4_OK) return st;
+        if ((mats[i].bits != 4 && mats[i].bits != 8) || mats[i].reserved != 0) return Q4_ERR_INVALID_ARG;
+        if (mats[i].N == 0) continue;
+        if (!mats[i].codes || !mats[i].scales || !mats[i].y) return Q4_ERR_INVALID_ARG;
+        if (misaligned(mats[i].codes, 16) || misaligned(mats[i].scales, 2) || misaligned(mats[i].y, 4))
+            return Q4_ERR_ALIGN;
+        out[n++] = mats[i];
+    }
+    *kept = n;
+    return Q4_OK;
+}
+
+// One launch for every matrix: M == 1, K % 256 == 0, 16-byte aligned x and scales.
+bool mixed_single_launch(int64_t M, int64_t K, const void* x, const q4_mixed_weight* mats, int n)
+{
+    if (M != 1 || K % 256 != 0 || misaligned(x, 16)) return false;
+    for (int i = 0; i < n; ++i)
+        if (misaligned(mats[i].scales, 16)) return false;
+    return true;
+}
+
+}  // namespace
+
+size_t q4_gemv_mixed_workspace_size(int64_t M, int64_t K, const q4_mixed_weight* mats, int count)
+{
+    if (M < 1 || M > Q4_GEMV_MAX_M || !mats || count < 1 || count > Q4_MULTI_MAX) return 0;
+    q4::DeviceInfo dev;
+    if (q4::current_device(&dev) != Q4_OK) return 0;
+    int64_t Ns[Q4_MULTI_MAX];
+    int fmts[Q4_MULTI_MAX];
+    q4_weight q4m[Q4_MULTI_MAX];
+    int n = 0, nq = 0;
+    for (int i = 0; i < count; ++i) {
+        if (check_nk(mats[i].N, K) != Q4_OK) return 0;
+        if (mats[i].N == 0) continue;
+        Ns[n] = mats[i].N;
+        fmts[n++] = mats[i].bits == 8 ? 1 : 0;
+        if (mats[i].bits != 8) q4m[nq++] = q4_weight{nullptr, nullptr, mats[i].N, nullptr};
+    }
+    size_t need = 0;
+    q4::GemvPlan plan;
+    if (n && M == 1 && K % 256 == 0 && q4::plan_gemv_tma(M, Ns, n, K, Q4_BF16, dev, &plan, q4::kGemvPlain, fmts))
+        need = plan.workspace_bytes;
+    if (n && M == 1 && K % 256 == 0 && q4::plan_gemv_tma(M, Ns, n, K, Q4_F32, dev, &plan, q4::kGemvPlain, fmts) &&
+        plan.workspace_bytes > need)
+        need = plan.workspace_bytes;
+    if (nq) {                                  // the Q4 matrices in their own launch
+        const size_t q = workspace_for(M, K, q4m, nq);
+        if (q > need) need = q;
+    }
+    return need;
+}
+
+q4_status q4_gemv_mixed(const void* x, q4_dtype x_dtype, int64_t M, int64_t K, const q4_mixed_weight* mats,
+                        int count, uint32_t flags, void* workspace, size_t workspace_bytes, void* stream)
+{
+    if (x_dtype != Q4_F32 && x_dtype != Q4_BF16) return Q4_ERR_DTYPE;
+    if (M < 0 || M > Q4_GEMV_MAX_M) return Q4_ERR_SHAPE;
+    if (K < 32 || (K % 32) != 0 || K > INT32_MAX) return Q4_ERR_SHAPE;
+    if (flags & ~Q4_WEIGHTS_STATIC) return Q4_ERR_INVALID_ARG;
+    q4_mixed_weight kept[Q4_MULTI_MAX];
+    int n = 0;
+    q4_status st = collect_mixed(mats, count, K, kept, &n);
+    if (st != Q4_OK) return st;
+    if (M == 0 || n == 0) return Q4_OK;
+    if (!x) return Q4_ERR_INVALID_ARG;
+    if (misaligned(x, 16) || (workspace && misaligned(workspace, 16))) return Q4_ERR_ALIGN;
+    q4::DeviceInfo dev;
+    if ((st = q4::current_device(&dev)) != Q4_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    q4_weight w[Q4_MULTI_MAX];
+    int64_t Ns[Q4_MULTI_MAX];
+    int fmts[Q4_MULTI_MAX];
+    for (int i = 0; i < n; ++i) {
+        w[i] = q4_weight{reinterpret_cast<const uint8_t*>(kept[i].codes), kept[i].scales, kept[i].N, kept[i].y};
+        Ns[i] = kept[i].N;
+        fmts[i] = kept[i].bits == 8 ? 1 : 0;
+    }
+    if (mixed_single_launch(M, K, x, kept, n)) {
+        q4::GemvPlan plan;
+        if (q4::plan_gemv_tma(M, Ns, n, K, x_dtype, dev, &plan, q4::kGemvPlain, fmts)) {
+            if (plan.workspace_bytes > 0 && (!workspace || workspace_bytes < plan.workspace_bytes))
+                return Q4_ERR_WORKSPACE;
+            return q4::launch_gemv_tma(x, x_dtype, M, K, w, n, (flags & Q4_WEIGHTS_STATIC) ? 1 : 0, workspace, plan,
+                                       s, q4::kGemvPlain, nullptr, fmts);
+        }
+        cudaGetLastError();
+    }
+    // Otherwise: the Q4 matrices in one q4_gemv_multi launch, each INT8 matrix on its own.
+    q4_weight q4m[Q4_MULTI_MAX];
+    int nq = 0;
+    for (int i = 0; i < n; ++i)
+        if (!fmts[i]) q4m[nq++] = w[i];
+    for (int i = 0; i < n; ++i)           // argument checks of every launch before the first
+        if (fmts[i] && (size_t)M * (size_t)K * sizeof(float) > (size_t)dev.max_smem_optin) return Q4_ERR_SHAPE;
+    if (nq) {
+        GemvCall call;
+        st = gemv_prepare(x, x_dtype, M, K, q4m, nq, flags, workspace, workspace_bytes, &call);
+        if (st != Q4_OK) return st;
+        st = q4::launch_gemv(x, x_dtype, M, K, call.kept, call.n, flags, workspace, call.plan, s);
+        if (st != Q4_OK) return st;
+    }
+    for (int i = 0; i < n; ++i) {
+        if (!fmts[i]) continue;
+        st = q4_int8_gemv(x, x_dtype, M, K, reinterpret_cast<const int8_t*>(kept[i].codes), kept[i].scales, kept[i].N,
+                          kept[i].y, stream);
+        if (st != Q4_OK) return st;
+    }
+    return Q4_OK;
 }
 
 q4_status q4_f16_gemv(const void* x, q4_dtype x_dtype, int64_t M, int64_t K, const uint16_t* w, int64_t N, float* y,

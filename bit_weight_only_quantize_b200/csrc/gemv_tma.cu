@@ -91,6 +91,8 @@ struct TmaGemvArgs {
     int teams;                        // teams per block
     int prefetch;                     // weights may be read before the dependency wait
     int x_f32;                        // kImma1: x is f32 (else bf16)
+    int fmt[Q4_MULTI_MAX];            // kImma1: 1 = matrix i holds INT8 codes [N][K], 0 = Q4
+    int has_int8;                     // some matrix is INT8 (the natural-order digits are staged)
     uint64_t wait_ns;                 // limit of the waits for this warp's copies (0: give up at once)
     // kEpiArgmax (greedy argmax over the rows of matrix 0, splits == 1): per x row, the
     // largest logit and its row; keys and the block counter live in a workspace that is
@@ -187,12 +189,23 @@ __device__ __forceinline__ void imma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1,
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(c0), "r"(c1));
 }
 
+// d = A . B + c for one m16n8k32 tile of signed 8-bit operands, exact int32 accumulation.
+__device__ __forceinline__ void imma_s8s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1, int c0, int c1)
+{
+    asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%10,%11,%10,%11};"
+        : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(c0), "r"(c1));
+}
+
 // Integer MMA results are read as f32 through a bias: the bit pattern 0x4B400000 is
 // 1.5 * 2^23, and adding an integer |v| < 2^22 to it gives the float 1.5 * 2^23 + v.
 constexpr int kBiasBits = 0x4B400000;
 // A lo-nibble column holds bias + T_lo and its hi-nibble column bias + 16 T_hi, so
 // hi * (1/16) + lo = (17/16) * 1.5 * 2^23 + T_lo + T_hi, an integer below 2^24 (exact).
 constexpr float kBias17 = 13369344.0f;
+constexpr float kBiasF = 12582912.0f;          // 1.5 * 2^23, the float of kBiasBits
 
 __device__ __forceinline__ float scale_at(const uint4& s8, int c)
 {
@@ -223,7 +236,8 @@ __device__ __forceinline__ double sum8_bf16(const uint4 raw)
 // 1 of X + 0x80, d1 = byte 2 of X + 0x8080, d0 = byte 3 of X + 0x808080 (each read as a
 // signed byte).  word[p][h] packs plane p's digits of k = 8t + h, + 2, + 4, + 6 (byte i =
 // k 8t + 2i + h); dsum[p][h] is their sum.
-__device__ __forceinline__ void digits8(const float (&v)[8], float x_scale, uint32_t (&word)[4][2], int (&dsum)[4][2])
+__device__ __forceinline__ void digits8(const float (&v)[8], float x_scale, uint32_t (&word)[4][2], int (&dsum)[4][2],
+                                        uint32_t (*nat)[2] = nullptr)
 {
     int X[8], Y1[8], Y2[8], Y3[8];
 #pragma unroll
@@ -232,6 +246,16 @@ __device__ __forceinline__ void digits8(const float (&v)[8], float x_scale, uint
         Y1[e] = (int)((uint32_t)X[e] + 0x80u);        // wraps (defined) only for non-finite x
         Y2[e] = (int)((uint32_t)X[e] + 0x8080u);
         Y3[e] = (int)((uint32_t)X[e] + 0x808080u);
+    }
+    if (nat) {        // natural k order: nat[p][0] = plane p of k 8t .. 8t+3, nat[p][1] = 8t+4 .. 8t+7
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int e = 4 * h;
+            nat[3][h] = __byte_perm(__byte_perm(X[e], X[e + 1], 0x0040), __byte_perm(X[e + 2], X[e + 3], 0x0040), 0x5410);
+            nat[2][h] = __byte_perm(__byte_perm(Y1[e], Y1[e + 1], 0x0051), __byte_perm(Y1[e + 2], Y1[e + 3], 0x0051), 0x5410);
+            nat[1][h] = __byte_perm(__byte_perm(Y2[e], Y2[e + 1], 0x0062), __byte_perm(Y2[e + 2], Y2[e + 3], 0x0062), 0x5410);
+            nat[0][h] = __byte_perm(__byte_perm(Y3[e], Y3[e + 1], 0x0073), __byte_perm(Y3[e + 2], Y3[e + 3], 0x0073), 0x5410);
+        }
     }
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -298,6 +322,12 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
     const int ngp = nb * 8;                                               // groups, padded
     const int nu = (nb + kBoxesPerStage - 1) / kBoxesPerStage;            // stage units of this split
     const int u0 = wt * nu / P, nbw = (wt + 1) * nu / P - u0;             // this warp's units
+    // INT8 matrices (kImma1): a box holds 4 groups (16 rows x 128 bytes), so a split has
+    // twice the boxes and units of a Q4 matrix.
+    const int nb8 = (ng + 3) >> 2;
+    const int nu8 = (nb8 + kBoxesPerStage - 1) / kBoxesPerStage;
+    const int u08 = wt * nu8 / P, nbw8 = (wt + 1) * nu8 / P - u08;
+    const bool mixed = MODE == kImma1 && a.has_int8;
     // A team walks row blocks first_rb, first_rb + rb_stride, ...  With fuse it walks the
     // row-block pairs of the gate and up matrices instead, visiting gate block p and then
     // up block p (= p + the gate's block count) of each pair in turn.
@@ -309,7 +339,13 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
     auto rb_of = [&](int i) {
         return kFuse ? first_rb + (i >> 1) * rb_stride + (i & 1) * a.rb_begin[1] : first_rb + i * rb_stride;
     };
-    const int njobs = nrb * nbw;
+    // INT8 row block: the matrix of row block rb holds INT8 codes
+    auto is_int8 = [&](int rb) { return mixed && a.fmt[matrix_of(a, rb)] != 0; };
+    int njobs = nrb * nbw;
+    if (mixed) {
+        njobs = 0;
+        for (int i = 0; i < nrb; ++i) njobs += is_int8(rb_of(i)) ? nbw8 : nbw;
+    }
     uint64_t* my_bars = bars + warp * kStages;
     const size_t K = (size_t)a.G * 32;
 
@@ -323,24 +359,33 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
     // kBoxesPerStage consecutive code boxes plus one scale box spanning all of them.  Jobs
     // are issued in order, so a cursor (unit, row block and its matrix) replaces the
     // division and the matrix lookup.
-    int iss_u = 0, iss_vis = 0, iss_mi = 0, iss_lrow = 0;
+    // A row block in which this warp has no unit (possible when a team's warps split an
+    // INT8 and a Q4 row block differently) is skipped.
+    int iss_u = 0, iss_vis = 0, iss_mi = 0, iss_lrow = 0, iss_i8 = 0;
     auto locate = [&]() {
-        const int rb = rb_of(iss_vis);
-        iss_mi = matrix_of(a, rb);
-        iss_lrow = (rb - a.rb_begin[iss_mi]) * kRows;
+        while (true) {
+            const int rb = rb_of(iss_vis);
+            iss_mi = matrix_of(a, rb);
+            iss_lrow = (rb - a.rb_begin[iss_mi]) * kRows;
+            iss_i8 = mixed && a.fmt[iss_mi] != 0;
+            if ((iss_i8 ? nbw8 : nbw) > 0 || iss_vis + 1 >= nrb) break;
+            ++iss_vis;
+        }
     };
     if (lane == 0 && njobs > 0) locate();
     auto issue = [&](int j) {
         const int s = j % kStages;
-        const int bf = (u0 + iss_u) * kBoxesPerStage;
-        const int nbox = min(kBoxesPerStage, nb - bf);
+        const int bf = ((iss_i8 ? u08 : u0) + iss_u) * kBoxesPerStage;
+        const int nbox = min(kBoxesPerStage, (iss_i8 ? nb8 : nb) - bf);
+        const int gpb = iss_i8 ? 4 : 8;                                   // groups per box
         uint64_t* bar = &my_bars[s];
         const CUtensorMap* cmap = &maps.codes[iss_mi];
         unsigned char* dst = codes + (warp * kStages + s) * kStageCodes;
-        mbar_arrive_expect_tx(bar, nbox * kCodeBox + kStageScales);
-        for (int q = 0; q < nbox; ++q) tma_load_2d(dst + q * kCodeBox, cmap, (g0 + 8 * (bf + q)) * 16, iss_lrow, bar);
-        tma_load_2d(scl + (warp * kStages + s) * kStageScales, &maps.scales[iss_mi], g0 + 8 * bf, iss_lrow, bar);
-        if (++iss_u == nbw) {
+        mbar_arrive_expect_tx(bar, nbox * kCodeBox + (iss_i8 ? kStageScales / 2 : kStageScales));
+        for (int q = 0; q < nbox; ++q)
+            tma_load_2d(dst + q * kCodeBox, cmap, (g0 + gpb * (bf + q)) * (iss_i8 ? 32 : 16), iss_lrow, bar);
+        tma_load_2d(scl + (warp * kStages + s) * kStageScales, &maps.scales[iss_mi], g0 + gpb * bf, iss_lrow, bar);
+        if (++iss_u == (iss_i8 ? nbw8 : nbw)) {
             iss_u = 0;
             ++iss_vis;
             if (j + 1 < njobs) locate();
@@ -362,8 +407,8 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
     //          neighbouring x rows fall on different banks.  Beside it, per group, -136 *
     //          sum(x) of the group for each x row (an f64 sum of the bf16 values, rounded
     //          once), laid out [group][n-tile][t] as the accumulator fragment of lane (g, t).
-    //  kImma1: each group g of 32 x values is scaled by 2^F_g (the largest F with
-    //          max |x| of the group * 2^F < 2^30, at most 100), rounded to integers X and
+    //  kImma1: each box of 8 groups (256 x values) is scaled by 2^F (the largest F with
+    //          max |x| of the box * 2^F < 2^30, at most 100), rounded to integers X and
     //          cut into four balanced base-256 digits X = d0 2^24 + d1 2^16 + d2 2^8 + d3,
     //          d1..d3 in [-128, 127].  The MMA's eight B columns are (digit plane p,
     //          nibble half h) = column 2p + h: half 0 holds the digits of the even k of
@@ -373,8 +418,8 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
     //          slots of the other half zero.  Then [group pair][plane][4] int: the C
     //          operand per group and plane, bias - 8 sum(d of even k) for half 0 and
     //          bias - 128 sum(d of odd k) for half 1, which removes the code offset 8.
-    //          Then [group] float: 2^-F_g.  One pass: the four lanes of a group find its
-    //          maximum with two shuffles, so no block-wide reduction is needed.
+    //          Then [box] float: 2^-F.  One pass: the 32 lanes that stage a box find its
+    //          maximum with five shuffles, so no block-wide reduction is needed.
     float* xoff = nullptr;
     const int rs = (ngp + 1) * 4;                                         // uint4 per staged x row
     if constexpr (MODE == kImma1) {
@@ -409,15 +454,17 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
             uint32_t mx = 0u;
 #pragma unroll
             for (int e = 0; e < 8; ++e) mx = max(mx, __float_as_uint(v[e]) & 0x7FFFFFFFu);
-            mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-            mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-            // F_g: 100 for a zero or subnormal maximum, 0 for a non-finite one (the product
+            // the warp's 32 items are the 8 groups of one box: one exponent per box
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            // F: 100 for a zero or subnormal maximum, 0 for a non-finite one (the product
             // is then undefined, but every step stays defined)
             const int ex = (int)(mx >> 23);
             const int F = ex == 0 ? 100 : ex >= 255 ? 0 : min(29 - (ex - 127), 100);
             uint32_t word[4][2];
             int dsum[4][2];
-            digits8(v, __uint_as_float((uint32_t)(F + 127) << 23), word, dsum);
+            uint32_t nat[4][2];
+            digits8(v, __uint_as_float((uint32_t)(F + 127) << 23), word, dsum, mixed ? nat : nullptr);
 #pragma unroll
             for (int p = 0; p < 4; ++p)
 #pragma unroll
@@ -434,7 +481,22 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
                     if (t == 0)
                         xc[((gp * 4 + p) << 1) + half] = make_int2(kBiasBits - 8 * dsum[p][0], kBiasBits - 128 * dsum[p][1]);
                 }
-                if (t == 0) xf[lg] = __uint_as_float((uint32_t)(127 - F) << 23);
+                if (lane == 0) xf[lg >> 3] = __uint_as_float((uint32_t)(127 - F) << 23);
+                if (mixed) {
+                    // INT8 operands, natural k order: [group][column g][t'] uint2 = (k 4t'..4t'+3,
+                    // k 16 + 4t' .. 16 + 4t'+3) of plane g for g < 4, zero for g >= 4; this
+                    // item's k = 8t .. 8t+7 are the chunks 2t and 2t+1 of 4.
+                    uint32_t* x8 = reinterpret_cast<uint32_t*>(xst + (size_t)ngp * 292);
+                    const int hf = t >> 1;
+#pragma unroll
+                    for (int p = 0; p < 4; ++p)
+#pragma unroll
+                        for (int c = 0; c < 2; ++c) {
+                            const int tq = (2 * t + c) & 3;
+                            x8[((lg * 8 + p) * 4 + tq) * 2 + hf] = nat[p][c];
+                            x8[((lg * 8 + p + 4) * 4 + tq) * 2 + hf] = 0u;
+                        }
+                }
             }
         }
     } else {
@@ -492,6 +554,7 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
     // A team reads it when it starts a row block and publishes its own when it rises.
     constexpr bool kFloor = kTopk && kTkM == 1;
     unsigned long long floor_now = 0ull, floor_pub = 0ull;
+    int jnext = 0;                                         // this warp's next job
     for (int rbi = 0; rbi < nrb; ++rbi) {
         const int rb = rb_of(rbi);
         if constexpr (kFloor) floor_now = load_key_relaxed(a.tk_floor);   // used in this block's epilogue
@@ -503,16 +566,59 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
 #pragma unroll
             for (int e = 0; e < 4; ++e) acc[n][e] = 0.f;
 
-        for (int jb = 0; jb < nbw; ++jb) {
-            const int j = rbi * nbw + jb;
+        const bool i8 = is_int8(rb);
+        const int nbw_c = i8 ? nbw8 : nbw;
+        for (int jb = 0; jb < nbw_c; ++jb) {
+            const int j = jnext++;
             const int s = j % kStages;
             if (ok) ok = a.wait_ns != 0 && mbar_wait_bounded(&my_bars[s], (uint32_t)(j / kStages) & 1u, a.wait_ns);
             if (ok) {
                 consumed = j + 1;
-                const int bf = (u0 + jb) * kBoxesPerStage;
-                const int nbox = min(kBoxesPerStage, nb - bf);
-#pragma unroll 1
-                for (int q = 0; q < nbox; ++q) {
+                const int bf = ((i8 ? u08 : u0) + jb) * kBoxesPerStage;
+                const int nbox = min(kBoxesPerStage, (i8 ? nb8 : nb) - bf);
+#pragma unroll
+                for (int q = 0; q < kBoxesPerStage; ++q) {
+                    if (q >= nbox) break;
+                    if (MODE == kImma1 && i8) {
+                        // INT8 box: 4 groups of 32 signed codes per row.  ldmatrix at the
+                        // Q4 addresses gives the A operand as is (a0/a2: k 4t .. 4t+3 and
+                        // 16 + 4t .. of row g, a1/a3 the same of row g+8); B column g < 4 is
+                        // digit plane g in natural k order, columns 4..7 are zero, and the
+                        // C operand is the bias alone (the codes carry no offset).  Lane t of
+                        // rows g, g+8 gets planes 2t, 2t+1 (t < 2): scaled onto the plane-t
+                        // accumulator they are u(2t) 2^(-8t) + u(2t+1) 2^(-8t-8) (t = 0, 1).
+                        const unsigned char* cb = codes + ((warp * kStages + s) * kBoxesPerStage + q) * kCodeBox;
+                        const unsigned char* sb = scl + (warp * kStages + s) * kStageScales + q * 8;
+                        const int g = lane >> 2, t = lane & 3;
+                        const int gb = (bf + q) * 4;                     // first group of the box
+                        const uint2 sg = *reinterpret_cast<const uint2*>(sb + g * 16);
+                        const uint2 sg8 = *reinterpret_cast<const uint2*>(sb + (g + 8) * 16);
+                        const int lr = lane & 7, li = lane >> 3;
+                        const uint32_t abase = smem_addr(cb) + ((li & 1) * 8 + lr) * 128 + (((li >> 1) ^ lr) << 4);
+                        const uint2* x8 = reinterpret_cast<const uint2*>(xst + (size_t)ngp * 292) + ((size_t)gb * 8 + g) * 4 + t;
+                        const float fb = reinterpret_cast<const float*>(xst + (size_t)ngp * 288)[gb >> 3];
+                        float part = 0.f, part8 = 0.f;
+                        const float lc0 = t == 0 ? 1.0f : t == 1 ? 0.00390625f : 0.0f;
+                        const float lc1 = t == 0 ? 0.00390625f : t == 1 ? 1.52587890625e-05f : 0.0f;
+#pragma unroll
+                        for (int cg = 0; cg < 4; ++cg) {
+                            uint32_t r0, r1, r2, r3;
+                            ldmatrix_x4(abase ^ (uint32_t)(cg << 5), r0, r1, r2, r3);
+                            const uint2 bq = x8[cg * 32];
+                            int d[4];
+                            imma_s8s8(d, r0, r1, r2, r3, bq.x, bq.y, kBiasBits, kBiasBits);
+                            const float v0 = (__int_as_float(d[0]) - kBiasF) * lc0 + (__int_as_float(d[1]) - kBiasF) * lc1;
+                            const float v1 = (__int_as_float(d[2]) - kBiasF) * lc0 + (__int_as_float(d[3]) - kBiasF) * lc1;
+                            const uint32_t sw = cg < 2 ? sg.x : sg.y, sw8 = cg < 2 ? sg8.x : sg8.y;
+                            const float s0 = __half2float(__ushort_as_half((unsigned short)((cg & 1) ? (sw >> 16) : (sw & 0xFFFFu))));
+                            const float s1 = __half2float(__ushort_as_half((unsigned short)((cg & 1) ? (sw8 >> 16) : (sw8 & 0xFFFFu))));
+                            part = fmaf(s0, v0, part);
+                            part8 = fmaf(s1, v1, part8);
+                        }
+                        yacc = fmaf(fb, part, yacc);
+                        yacc8 = fmaf(fb, part8, yacc8);
+                        continue;
+                    }
                     {
                         const unsigned char* cb = codes + ((warp * kStages + s) * kBoxesPerStage + q) * kCodeBox;
                         const unsigned char* sb = scl + (warp * kStages + s) * kStageScales + q * 16;
@@ -529,9 +635,9 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
                                 smem_addr(cb) + ((li & 1) * 8 + lr) * 128 + (((li >> 1) ^ lr) << 4);
                             const uint4* xq = reinterpret_cast<const uint4*>(xst) + ((gb >> 1) * 8 + g) * 4 + t;
                             const int4* xc = reinterpret_cast<const int4*>(xst + (size_t)ngp * 256) + (gb >> 1) * 4 + t;
-                            const float4* xf = reinterpret_cast<const float4*>(xst + (size_t)ngp * 288) + (gb >> 2);
-                            const float4 f0 = xf[0], f1 = xf[1];     // 2^-F_g of the box's 8 groups
-                            const float fgs[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
+                            // the box's sums are scaled and added here, then once by 2^-F
+                            const float fb = reinterpret_cast<const float*>(xst + (size_t)ngp * 288)[gb >> 3];
+                            float part = 0.f, part8 = 0.f;
 #pragma unroll
                             for (int cp = 0; cp < 4; ++cp) {
                                 uint32_t r0, r1, r2, r3;
@@ -554,10 +660,12 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
                                         fmaf(__int_as_float(d[1]), 0.0625f, __int_as_float(d[0])) - kBias17;
                                     const float u1 =
                                         fmaf(__int_as_float(d[3]), 0.0625f, __int_as_float(d[2])) - kBias17;
-                                    yacc = fmaf(scale_at(sg, c) * fgs[c], u0, yacc);
-                                    yacc8 = fmaf(scale_at(sg8, c) * fgs[c], u1, yacc8);
+                                    part = fmaf(scale_at(sg, c), u0, part);
+                                    part8 = fmaf(scale_at(sg8, c), u1, part8);
                                 }
                             }
+                            yacc = fmaf(fb, part, yacc);
+                            yacc8 = fmaf(fb, part8, yacc8);
                         } else {
                             const int g = lane >> 2, t = lane & 3;
                             const uint4 sg = *reinterpret_cast<const uint4*>(sb + g * kScaleRow);
@@ -866,17 +974,19 @@ size_t per_warp_bytes(int mode)
     return (size_t)kStages * (kStageCodes + kStageScales + sizeof(uint64_t)) + (size_t)kRows * mp * sizeof(float);
 }
 
-size_t x_stage_bytes(int mode, int nb, int64_t M)
+// kImma1 per group: B operands 256 B, C operands 32 B, 2^-F_g 4 B, and with INT8
+// matrices in the launch the natural-order B operands, 256 B more.
+size_t x_stage_bytes(int mode, int nb, int64_t M, bool int8 = false)
 {
     const int mp = mode == kMma16 ? 16 : mode == kMma8 ? 8 : 1;
     const size_t ngp = (size_t)nb * 8;
-    if (mode == kImma1) return ngp * 292;      // per group: B operands 256 B, C operands 32 B, 2^-F_g 4 B
+    if (mode == kImma1) return ngp * (int8 ? 548 : 292);
     return (size_t)(M + 1) * (ngp + 1) * 64 + ngp * (mp / 8) * 64;
 }
 
-size_t smem_bytes(int mode, int warps, int nb, int64_t M)
+size_t smem_bytes(int mode, int warps, int nb, int64_t M, bool int8 = false)
 {
-    return 1024 + (size_t)warps * per_warp_bytes(mode) + x_stage_bytes(mode, nb, M);
+    return 1024 + (size_t)warps * per_warp_bytes(mode) + x_stage_bytes(mode, nb, M, int8);
 }
 
 int mode_for(int64_t M, q4_dtype xt)
@@ -915,11 +1025,17 @@ bool tma_gemv_eligible(int64_t M, int64_t K, q4_dtype xt, const void* packed, co
 }
 
 bool plan_gemv_tma(int64_t M, const int64_t* Ns, int count, int64_t K, q4_dtype xt, const DeviceInfo& dev,
-                   GemvPlan* p, int epi)
+                   GemvPlan* p, int epi, const int* fmts, bool allow_split)
 {
-    const bool fuse = epi == kEpiFuse, whole_k = epi != kEpiPlain;
+    const bool fuse = epi == kEpiFuse, whole_k = epi != kEpiPlain || !allow_split;
     if (fuse && (count != 2 || Ns[0] != Ns[1])) return false;
     const int mode = mode_for(M, xt);
+    int n_int8 = 0;
+    for (int i = 0; fmts && i < count; ++i) n_int8 += fmts[i] != 0;
+    if (n_int8 && (mode != kImma1 || epi != kEpiPlain)) return false;
+    const bool int8 = n_int8 > 0;
+    // INT8 row blocks have twice the stage units of Q4 ones
+    const double unit_scale = !int8 ? 1.0 : n_int8 == count ? 2.0 : 1.5;
     const int G = (int)(K / 32);
     long long rbl = 0;
     for (int i = 0; i < count; ++i) rbl += (Ns[i] + kRows - 1) / kRows;
@@ -938,7 +1054,7 @@ bool plan_gemv_tma(int64_t M, const int64_t* Ns, int count, int64_t K, q4_dtype 
     };
     // Splits forced by shared memory: the staged x of one split leaves room for 4 warps.
     int splits_min = 1;
-    while (1024 + 4 * pw + x_stage_bytes(mode, split_boxes(splits_min), M) > budget) {
+    while (1024 + 4 * pw + x_stage_bytes(mode, split_boxes(splits_min), M, int8) > budget) {
         if (split_boxes(splits_min) <= kBoxesPerStage) return false;
         ++splits_min;
     }
@@ -953,7 +1069,7 @@ bool plan_gemv_tma(int64_t M, const int64_t* Ns, int count, int64_t K, q4_dtype 
     for (int sp = splits_min; sp <= max_splits; ++sp) {
         const int nbs = split_boxes(sp);
         if ((boxes + nbs - 1) / nbs != sp) continue;                  // same cut as fewer splits
-        const size_t xs = x_stage_bytes(mode, nbs, M);
+        const size_t xs = x_stage_bytes(mode, nbs, M, int8);
         if (1024 + pw + xs > budget) continue;
         const size_t fitw = (budget - 1024 - xs) / pw;
         const int wbs = (int)(fitw < (size_t)kMaxWarps ? fitw : (size_t)kMaxWarps);
@@ -969,7 +1085,8 @@ bool plan_gemv_tma(int64_t M, const int64_t* Ns, int count, int64_t K, q4_dtype 
                 const long long gxs = std::min(((long long)walk + tm - 1) / tm, sms);
                 const long long rounds = visits * (((long long)walk + gxs * tm - 1) / (gxs * tm));
                 const double share = std::max((double)(tm * pp), kMinWarpShare) / 16.0;
-                const double cost = (double)rounds * (pwu + kEpilogueCost) * share + (sp > 1 ? kSplitCost : 0.0);
+                const double cost = (double)rounds * (pwu * unit_scale + kEpilogueCost) * share +
+                                    (sp > 1 ? kSplitCost : 0.0);
                 if (splits == 0 || cost < best - 1e-9) {
                     splits = sp;
                     P = pp;
@@ -983,7 +1100,7 @@ bool plan_gemv_tma(int64_t M, const int64_t* Ns, int count, int64_t K, q4_dtype 
     const int ksg = split_boxes(splits) * 8;
     const int nb = ksg / 8;
     const int warps = P * teams;
-    const size_t smem = smem_bytes(mode, warps, nb, M);
+    const size_t smem = smem_bytes(mode, warps, nb, M, int8);
     if (smem > budget) return false;
     const int per_sm = blocks_per_sm(kernel_for(mode, epi), warps * 32, smem);
     if (per_sm < 1) return false;
@@ -1001,23 +1118,28 @@ bool plan_gemv_tma(int64_t M, const int64_t* Ns, int count, int64_t K, q4_dtype 
     p->smem_bytes = (int)smem;
     p->workspace_bytes =
         splits > 1 ? kCounterBytes + (size_t)splits * (size_t)M * (size_t)row_blocks * kRows * sizeof(float) : 0;
+    p->has_int8 = int8 ? 1 : 0;
     return true;
 }
 
 q4_status launch_gemv_tma(const void* x, q4_dtype xt, int64_t M, int64_t K, const q4_weight* mats, int count,
                           int prefetch, void* workspace, const GemvPlan& plan, cudaStream_t stream, int epi,
-                          const ArgmaxOut* am)
+                          const ArgmaxOut* am, const int* fmts)
 {
     TmaMaps maps;
     TmaGemvArgs a;
     const uint64_t G = (uint64_t)(K / 32);
     int rb = 0;
     for (int i = 0; i < count; ++i) {
-        if (!encode_tma_2d(&maps.codes[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, mats[i].packed, (uint64_t)K / 2,
-                           (uint64_t)mats[i].N, (uint64_t)K / 2, 128, kRows, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        // Q4: K/2 code bytes per row, a box is 8 groups; INT8: K bytes per row, 4 groups
+        const bool i8 = fmts && fmts[i] != 0;
+        const uint64_t row_bytes = i8 ? (uint64_t)K : (uint64_t)K / 2;
+        if (!encode_tma_2d(&maps.codes[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, mats[i].packed, row_bytes,
+                           (uint64_t)mats[i].N, row_bytes, 128, kRows, CU_TENSOR_MAP_SWIZZLE_128B) ||
             !encode_tma_2d(&maps.scales[i], CU_TENSOR_MAP_DATA_TYPE_UINT16, mats[i].scales, G, (uint64_t)mats[i].N,
-                           G * 2, 8 * kBoxesPerStage, kRows, CU_TENSOR_MAP_SWIZZLE_NONE))
+                           G * 2, (i8 ? 4 : 8) * kBoxesPerStage, kRows, CU_TENSOR_MAP_SWIZZLE_NONE))
             return Q4_ERR_CUDA;
+        a.fmt[i] = i8 ? 1 : 0;
         a.y[i] = mats[i].y;
         a.N[i] = (int)mats[i].N;
         a.rb_begin[i] = rb;
@@ -1029,7 +1151,9 @@ q4_status launch_gemv_tma(const void* x, q4_dtype xt, int64_t M, int64_t K, cons
         a.y[i] = nullptr;
         a.N[i] = 0;
         a.rb_begin[i] = rb;
+        a.fmt[i] = 0;
     }
+    a.has_int8 = plan.has_int8;
     a.rb_begin[Q4_MULTI_MAX] = rb;
     unsigned* err = device_error_word();
     if (!err) return Q4_ERR_CUDA;

@@ -38,6 +38,7 @@ struct GemvPlan {
     int xcap;               // groups of x staged in shared memory at once
     int smem_bytes;         // dynamic shared memory per block
     size_t workspace_bytes; // partial sums + counters (0 when splits == 1)
+    int has_int8;           // TMA kernel: some matrix holds INT8 codes
 };
 
 // Chooses the kernels for one or more weight matrices sharing x (all N > 0).
@@ -67,12 +68,14 @@ struct ArgmaxOut {
     unsigned row_base;         // added to every reported row
 };
 
+// fmts: per matrix 1 = INT8 codes [N][K] (M == 1, plain epilogue only), 0 = Q4; null = all
+// Q4.  allow_split = false keeps K whole (no workspace).
 bool plan_gemv_tma(int64_t M, const int64_t* Ns, int count, int64_t K, q4_dtype xt, const DeviceInfo& dev,
-                   GemvPlan* plan, int epi = kGemvPlain);
-// am: non-null for an argmax or top-k launch.
+                   GemvPlan* plan, int epi = kGemvPlain, const int* fmts = nullptr, bool allow_split = true);
+// am: non-null for an argmax or top-k launch.  For an INT8 matrix, mats[i].packed holds its codes.
 q4_status launch_gemv_tma(const void* x, q4_dtype xt, int64_t M, int64_t K, const q4_weight* mats, int count,
                           int prefetch, void* workspace, const GemvPlan& plan, cudaStream_t stream,
-                          int epi = kGemvPlain, const ArgmaxOut* am = nullptr);
+                          int epi = kGemvPlain, const ArgmaxOut* am = nullptr, const int* fmts = nullptr);
 
 q4_status launch_topk_merge(const float* values, const int64_t* indices, int64_t S, int64_t M, int64_t k,
                             int64_t* out_index, float* out_value, cudaStream_t stream);

@@ -314,15 +314,52 @@ Q4_API q4_status q4_topk_merge(const float* values, const int64_t* indices, int6
  *   16-byte aligned) + scales binary16 bits [N,K/32] (2-byte aligned); flags as for
  *   q4_quantize.  N, K as for q4_quantize.  Bit-identical to the definition above.
  * q4_int8_gemv: y[M,N] (f32) = x[M,K] . dequant(W)^T for M = 1..16, x f32 or bfloat16
- *   (device, 4-byte aligned), codes 16-byte aligned, scales 2-byte aligned, y 4-byte
- *   aligned.  x is staged in shared memory as f32 (M*K*4 bytes; a shape whose x does not
- *   fit returns Q4_ERR_SHAPE).  Products in f32 per group of 16 k, scaled and accumulated
- *   in f32.  M == 0 or N == 0 is a no-op.
+ *   (device, 16-byte aligned, the same contract as q4_gemv, so one x serves both formats),
+ *   codes 16-byte aligned, scales 2-byte aligned, y 4-byte aligned.  M == 1 with
+ *   K % 256 == 0 and 16-byte aligned scales runs on the Q4 GEMV's TMA kernel: x is cut
+ *   into exact digit planes as for q4_gemv (per group of 32, max |x| * 2^F_g < 2^30) and
+ *   the codes multiply them on the integer tensor cores with exact int32 group sums, each
+ *   scaled by its binary16 scale times 2^-F_g and accumulated in f32.  Other shapes stage
+ *   x in shared memory as f32 (M*K*4 bytes; a shape whose x does not fit returns
+ *   Q4_ERR_SHAPE) and form products in f32 per group of 16 k, scaled and accumulated in
+ *   f32.  No workspace.  M == 0 or N == 0 is a no-op.
  */
 Q4_API q4_status q4_int8_quantize(const float* W, int64_t N, int64_t K, int8_t* codes, uint16_t* scales,
                                   uint32_t* flags, void* stream);
 Q4_API q4_status q4_int8_gemv(const void* x, q4_dtype x_dtype, int64_t M, int64_t K, const int8_t* codes,
                               const uint16_t* scales, int64_t N, float* y, void* stream);
+
+/*
+ * q4_gemv_mixed: the projections of one token against weights of mixed precision, INT8
+ * and Q4 matrices side by side (QKV-Core thread, section "自适应混合量化": precision-
+ * sensitive layers in INT8, the rest in INT4): y_i = x . dequant_i(W_i)^T for up to
+ * Q4_MULTI_MAX matrices sharing x and K.
+ *   mats[i].codes   device: Q4 packed codes [N, K/2] (bits == 4, the q4_quantize format) or
+ *                   INT8 codes [N, K] (bits == 8, the q4_int8_quantize format), 16-byte aligned.
+ *   mats[i].scales  device, binary16 bits [N, K/32], 2-byte aligned.
+ *   mats[i].y       device, f32 [M, N], 4-byte aligned (output, overwritten).
+ *   mats[i].bits    4 or 8; mats[i].reserved must be 0 (Q4_ERR_INVALID_ARG otherwise).
+ *   x, M, K, flags  as for q4_gemv_multi (x 16-byte aligned).
+ *   workspace  at least q4_gemv_mixed_workspace_size(M, K, mats, count) bytes, as for
+ *              q4_gemv_multi (zero before its first use, left zero by every call).
+ * With M == 1, K % 256 == 0 and 16-byte aligned scales every matrix streams through one
+ * launch of the TMA kernel (the INT8 rows take the q4_int8_gemv arithmetic, the Q4 rows
+ * the q4_gemv arithmetic); otherwise the Q4 matrices run in one q4_gemv_multi launch and
+ * each INT8 matrix in its own q4_int8_gemv launch, in that order on the stream.
+ * Matrices with N == 0 are skipped; M == 0 is a no-op.
+ */
+typedef struct q4_mixed_weight {
+    const void* codes;        /* device: Q4 packed [N, K/2] or INT8 [N, K] codes */
+    const uint16_t* scales;   /* device, binary16 bits [N, K/32] */
+    int64_t N;                /* output features (rows), >= 0 */
+    float* y;                 /* device, f32 [M, N] (output) */
+    int32_t bits;             /* 4 or 8 */
+    int32_t reserved;         /* 0 */
+} q4_mixed_weight;
+
+Q4_API size_t q4_gemv_mixed_workspace_size(int64_t M, int64_t K, const q4_mixed_weight* mats, int count);
+Q4_API q4_status q4_gemv_mixed(const void* x, q4_dtype x_dtype, int64_t M, int64_t K, const q4_mixed_weight* mats,
+                               int count, uint32_t flags, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * q4_f16_gemv: y[M,N] = x[M,K] . W^T for binary16 weights W (2 bytes per weight), the

@@ -70,8 +70,8 @@ def offset_path_bound(x: np.ndarray, scales: np.ndarray, roundings: int) -> np.n
 
 
 def digit_shift(x_group: np.ndarray) -> int:
-    """The power of two F the M = 1 path scales a group of x by: max |x| * 2^F < 2^30
-    (F <= 100)."""
+    """The power of two F the M = 1 path scales a box of 256 x values by:
+    max |x| * 2^F < 2^30 (F <= 100)."""
     mx = float(np.max(np.abs(x_group))) if x_group.size else 0.0
     if mx == 0.0 or mx < 2.0 ** -126:
         return 100
@@ -84,17 +84,17 @@ def digit_shift(x_group: np.ndarray) -> int:
 
 
 def digit_path_bound(x: np.ndarray, deq: np.ndarray, roundings: int) -> np.ndarray:
-    """Bound for the M = 1 path (K % 256 == 0).  Each group of 32 x values is rounded once
-    to integers X = rint(x 2^F_g) (error <= 2^(-F_g-1) per element) and cut into four
-    base-256 digit planes X_p; the integer MMAs are exact, and plane p's f32 sum
-    (CUDA-core FMAs of scale 2^-F_g x exact group sums) is bounded by
-    gamma_n sum_k |w'_k| |X_p,k| 2^-F_g.  Scaled by 2^(8 (3 - p)) and summed over p this
-    is at most gamma_n sum_k |w'_k| (|x_k| + 1.01 * 2^(24 - F_g))."""
+    """Bound for the M = 1 path (K % 256 == 0).  Each box of 256 x values (8 groups) is
+    rounded once to integers X = rint(x 2^F) (error <= 2^(-F-1) per element) and cut into
+    four base-256 digit planes X_p; the integer MMAs are exact, and plane p's f32 sums
+    (CUDA-core FMAs of scale x exact group sums, then 2^-F per box) are bounded by
+    gamma_n sum_k |w'_k| |X_p,k| 2^-F.  Scaled by 2^(8 (3 - p)) and summed over p this is
+    at most gamma_n sum_k |w'_k| (|x_k| + 1.01 * 2^(24 - F))."""
     xs = x_f64(x)
     wa = np.abs(deq)
     M, K = xs.shape
     out = np.empty((M, deq.shape[0]))
     for m in range(M):
-        q = np.repeat(np.array([2.0 ** -digit_shift(xs[m, g:g + 32]) for g in range(0, K, 32)]), 32)
+        q = np.repeat(np.array([2.0 ** -digit_shift(xs[m, g:g + 256]) for g in range(0, K, 256)]), 256)[:K]
         out[m] = wa @ (0.5 * q) + gamma(roundings, U_CUDA_CORE) * (wa @ (np.abs(xs[m]) + 1.01 * 2.0 ** 24 * q))
     return out

@@ -217,7 +217,8 @@ def test_int8_validation(lib):
     assert g(A16, 1, 17, 64, A16, A16, 8, A16, S) == 2          # M > 16
     assert g(A16, 1, 1, 48, A16, A16, 8, A16, S) == 2           # K % 32
     assert g(A16, 1, 1, 64, None, A16, 8, A16, S) == 1
-    assert g(A16 + 2, 1, 1, 64, A16, A16, 8, A16, S) == 3       # x: 4 bytes
+    assert g(A16 + 2, 1, 1, 64, A16, A16, 8, A16, S) == 3       # x: 16 bytes
+    assert g(A16 + 4, 1, 1, 64, A16, A16, 8, A16, S) == 3
     assert g(A16, 1, 1, 64, A8, A16, 8, A16, S) == 3            # codes: 16 bytes
     assert g(A16, 1, 1, 64, A16, A16, 8, A16 + 2, S) == 3       # y: 4 bytes
     assert g(None, 1, 0, 64, None, None, 8, None, S) == 0       # M == 0: no-op
@@ -243,3 +244,25 @@ def test_consumer_wait_limit_round_trips(lib):
     assert prev == 10 ** 9
     assert lib.q4_set_consumer_wait_limit(prev) == 12345
     assert lib.q4_set_consumer_wait_limit(prev) == prev
+
+
+def test_mixed_validation(lib):
+    """q4_gemv_mixed checks its matrix list before touching a device."""
+    S = None
+    W = _lib.MixedWeight
+
+    def call(mats, M=1, K=64, x=A16, dtype=1, flags=0):
+        arr = (W * len(mats))(*mats)
+        return lib.q4_gemv_mixed(x, dtype, M, K, ctypes.cast(arr, ctypes.c_void_p), len(mats), flags, None, 0, S)
+    ok = W(A16, A16, 8, A16, 8, 0)
+    assert call([ok], dtype=7) == 4                                  # dtype
+    assert call([ok], M=17) == 2                                     # M > 16
+    assert call([ok], K=48) == 2                                     # K % 32
+    assert call([ok], flags=2) == 1                                  # unknown flag
+    assert call([W(A16, A16, 8, A16, 5, 0)]) == 1                    # bits must be 4 or 8
+    assert call([W(A16, A16, 8, A16, 8, 1)]) == 1                    # reserved must be 0
+    assert call([W(None, A16, 8, A16, 8, 0)]) == 1                   # null codes
+    assert call([W(A8, A16, 8, A16, 4, 0)]) == 3                     # codes 16-byte aligned
+    assert call([ok], x=A16 + 8) == 3                                # x 16-byte aligned
+    assert call([W(None, None, 0, None, 8, 0)]) == 0                 # N == 0: nothing to do
+    assert call([ok], M=0) == 0                                      # M == 0: no-op

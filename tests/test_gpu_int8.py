@@ -7,7 +7,7 @@ import torch
 
 import oracle
 import synth_inputs
-from tests._parity import f32_sum_bound, rel_inf, to_dev_x
+from tests._parity import digit_path_bound, f32_sum_bound, rel_inf, to_dev_x
 
 pytestmark = pytest.mark.gpu
 
@@ -65,11 +65,78 @@ def test_gemv_matches_oracle(M, N, K, x_dtype):
     ref = oracle.matmul8(x, codes, scales, threads=8)
     err = rel_inf(got, ref)
     assert err <= TOL[x_dtype], err
-    # per element: exact code x exact x products summed in f32 (16 per block of k, one
-    # scale FMA per block, a lane's blocks, the warp's 5 shuffle adds): gamma_n sum |x w'|
-    n = 16 + K // 16 + 8
-    bound = f32_sum_bound(x, oracle.dequantize8(codes, scales), n)
-    assert np.all(np.abs(got - ref) <= bound + 1e-30)
+    assert np.all(np.abs(got - ref) <= int8_bound(x, codes, scales) + 1e-30)
+
+
+def int8_bound(x, codes, scales):
+    """Per-element bound of the path the shape takes.  M = 1 with K % 256 == 0: the
+    digit-plane path (x rounded per group of 32, exact integer group sums, one rounding
+    combining two planes, the scale FMA and the f32 accumulation per plane).  Otherwise:
+    exact code x exact x products summed in f32 (16 per block of k, one scale FMA per
+    block, a lane's blocks, the warp's 5 shuffle adds)."""
+    M, K = x.shape
+    deq = oracle.dequantize8(codes, scales)
+    if M == 1 and K % 256 == 0:
+        return digit_path_bound(x, deq, 2 * (K // 32) + 40)
+    return f32_sum_bound(x, deq, 16 + K // 16 + 8)
+
+
+@pytest.mark.parametrize("N,x_dtype", [(4096, "bf16"), (33, "f32"), (20000, "bf16"), (1, "bf16")])
+def test_gemv_tma_path_k_large(N, x_dtype):
+    """M = 1, K % 256 == 0: the TMA kernel's integer path, K = 2560 and K = 8192."""
+    import bit_weight_only_quantize_b200 as q4
+    for K in (2560, 8192):
+        codes, scales, _ = oracle.quantize8(synth_inputs.weights("outliers", N, K, seed=N + K))
+        x = synth_inputs.activations(1, K, x_dtype, seed=K)
+        y = q4.int8_gemv(to_dev_x(x), torch.from_numpy(codes).cuda(), torch.from_numpy(scales.view(np.int16)).cuda())
+        torch.cuda.synchronize()
+        got, ref = y.cpu().numpy(), oracle.matmul8(x, codes, scales, threads=8)
+        assert rel_inf(got, ref) <= 1e-5
+        assert np.all(np.abs(got - ref) <= int8_bound(x, codes, scales) + 1e-30)
+
+
+def _mixed_case(M, K, spec, x_dtype, seed):
+    """Matrices [(N, bits)] quantised by the oracle, on the device."""
+    import bit_weight_only_quantize_b200 as q4
+    host, dev = [], []
+    for i, (n, bits) in enumerate(spec):
+        W = synth_inputs.weights("outliers", n, K, seed=seed + i)
+        codes, scales, _ = (oracle.quantize8 if bits == 8 else oracle.quantize)(W)
+        host.append((codes, scales, bits))
+        dev.append((torch.from_numpy(codes).cuda(), torch.from_numpy(scales.view(np.int16)).cuda(), bits))
+    x = synth_inputs.activations(M, K, x_dtype, seed=seed)
+    ys = q4.gemv_mixed(to_dev_x(x), dev)
+    torch.cuda.synchronize()
+    for (codes, scales, bits), y in zip(host, ys):
+        got = y.cpu().numpy()
+        if bits == 8:
+            ref = oracle.matmul8(x, codes, scales, threads=8)
+            bound = int8_bound(x, codes, scales)
+        else:
+            ref = oracle.matmul(x, codes, scales, threads=8)
+            bound = None
+            if M == 1 and K % 256 == 0:
+                bound = digit_path_bound(x, oracle.dequantize(codes, scales), 2 * (K // 32) + 40)
+        assert rel_inf(got, ref) <= 1e-5, bits
+        if bound is not None:
+            assert np.all(np.abs(got - ref) <= bound + 1e-30)
+
+
+@pytest.mark.parametrize("spec", [
+    [(2048, 4), (1024, 8), (4096, 4)],          # attention INT8 beside Q4 projections, one launch
+    [(4096, 8), (4096, 8)],                      # INT8 only
+    [(33, 8), (17, 4), (0, 8), (300, 8)],        # ragged row blocks, an empty matrix
+    [(16, 8), (16, 4)],                          # skinny: K split across blocks
+])
+def test_mixed_single_launch(spec):
+    _mixed_case(1, 2560, spec, "bf16", seed=len(spec))
+    _mixed_case(1, 8192, spec, "f32", seed=7)
+
+
+@pytest.mark.parametrize("M,K", [(3, 2560), (1, 96), (16, 512)])
+def test_mixed_separate_launches(M, K):
+    """Shapes the single launch does not take: Q4 in one launch, each INT8 matrix in its own."""
+    _mixed_case(M, K, [(1000, 8), (500, 4), (64, 8)], "bf16", seed=M + K)
 
 
 def test_gemv_x_too_large_is_rejected():
