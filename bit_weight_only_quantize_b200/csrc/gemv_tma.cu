@@ -302,6 +302,7 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
     constexpr int kTkM = MODE == kImma1 ? 1 : MP;                         // x rows of a top-k list set
     extern __shared__ unsigned char smem_raw[];
     __shared__ int s_last[kMaxWarps];
+    __shared__ uint64_t s_xbar;                                            // kMma*: x rows in flight
     const int W = blockDim.x >> 5;
     unsigned char* smem =
         reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -422,6 +423,7 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
     //          maximum with five shuffles, so no block-wide reduction is needed.
     float* xoff = nullptr;
     const int rs = (ngp + 1) * 4;                                         // uint4 per staged x row
+    bool x_ok = true;                                                     // kMma*: x rows arrived
     if constexpr (MODE == kImma1) {
         const int items = ngp * 4;                                        // (group, k = 8t .. 8t+7)
         uint2* xq = reinterpret_cast<uint2*>(xst);
@@ -502,16 +504,27 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
     } else {
         uint4* xp = reinterpret_cast<uint4*>(xst);
         xoff = reinterpret_cast<float*>(xp + (a.M + 1) * rs);
+        // The split's part of each x row arrives by one bulk copy, straight where its
+        // staged words go (all rows in flight at once), and is then permuted in place.
+        if (threadIdx.x == 0) {
+            mbar_init(&s_xbar, 1);
+            fence_mbar_init();
+            mbar_arrive_expect_tx(&s_xbar, (uint32_t)(a.M * ng * 64));
+            for (int m = 0; m < a.M; ++m)
+                bulk_load(xp + m * rs, reinterpret_cast<const uint16_t*>(a.x) + (size_t)m * K + (size_t)g0 * 32,
+                          (uint32_t)(ng * 64), &s_xbar);
+        }
+        __syncthreads();
+        x_ok = mbar_wait_bounded(&s_xbar, 0, kWaitLimit);
         const int total = (a.M + 1) * ngp * 4;
         for (int i0 = threadIdx.x - lane; i0 < total; i0 += blockDim.x) {    // warp-uniform trips
             const int i = i0 + lane;
             const int m = i / (ngp * 4);
             const int rem = i - m * ngp * 4;
-            const int lg = rem >> 2, wd = rem & 3;
+            const int lg = rem >> 2;
+            const int wd = rem & 3;
             uint4 raw = make_uint4(0u, 0u, 0u, 0u);
-            if (i < total && m < a.M && lg < ng)
-                raw = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(a.x) + (size_t)m * K +
-                                                      (size_t)(g0 + lg) * 32 + wd * 8);
+            if (i < total && m < a.M && lg < ng && x_ok) raw = xp[m * rs + rem];
             if (i < total) xp[m * rs + rem] = pairs_of(raw);
             double sum = sum8_bf16(raw);
             sum += __shfl_xor_sync(0xffffffffu, sum, 1);                    // words (0,1) and (2,3)
@@ -543,7 +556,7 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
 #pragma unroll
     for (int n = 0; n < NT; ++n) xrow[n] = reinterpret_cast<const uint4*>(xst) + min(n * 8 + (lane >> 2), a.M) * rs;
 
-    bool ok = true;
+    bool ok = x_ok;
     int consumed = 0;
     float gsave[kFuse ? kRows * Q4_GEMV_MAX_M / 32 : 1];   // fuse: the gate totals of the current pair
     unsigned long long tk[kTopk ? kTkM + 1 : 1];           // top-k: the team's list per x row
@@ -855,6 +868,7 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
         for (int j = consumed; j < issued; ++j)    // copies still in flight into this warp's ring
             if (!mbar_wait_bounded(&my_bars[j % kStages], (uint32_t)(j / kStages) & 1u, kWaitLimit)) break;
     }
+    if (!x_ok && threadIdx.x == 0) mbar_wait_bounded(&s_xbar, 0, kWaitLimit);   // x rows still in flight
 
     if constexpr (kArgmax) {                                // the last block to finish reports and resets
         __syncthreads();
