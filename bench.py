@@ -765,7 +765,7 @@ def run_reference(args, world, rank):
 # ---------------------------------------------------------------- ncu cases
 PROFILE_CASES = ["decode", "decode_small", "decode_multi", "lm_head", "lm_head_argmax", "lm_head_topk", "gemv_m2",
                  "gemv_m4", "gemv_m8", "gemv_m16", "gate_up", "f16", "int8", "int8_m4", "int8_quantize", "quantize",
-                 "mixed", "gemm", "gemm_m2048", "gemm_m512", "topk_merge", "ffma"]
+                 "mixed", "gemm", "gemm_m2048", "gemm_m512", "gemm_m512n2048", "topk_merge", "ffma"]
 
 
 def run_profile_case(args):
@@ -791,7 +791,7 @@ def run_profile_case(args):
             (q4.quantize if case == "quantize" else q4.int8_quantize)(Wd)
     elif case.startswith("gemm"):
         gw = {"gemm": synth_inputs.PREFILL[-2], "gemm_m2048": synth_inputs.PREFILL[2],
-              "gemm_m512": synth_inputs.PREFILL[0]}[case]
+              "gemm_m512": synth_inputs.PREFILL[0], "gemm_m512n2048": synth_inputs.PREFILL[1]}[case]
         _, packed, scales = make_quantized(torch, q4, gw, 0, device)
         x = x_of(gw)
         y = torch.empty((gw.M, gw.N), dtype=torch.bfloat16, device=device)

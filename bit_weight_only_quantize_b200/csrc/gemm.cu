@@ -25,6 +25,7 @@
 // block records kErrWaitTimeout, all roles stop, outstanding copies and MMAs are
 // waited for (bounded) and tensor memory is freed before the block exits.
 #include <algorithm>
+#include <mutex>
 
 #include "tma.cuh"
 
@@ -37,6 +38,7 @@ constexpr int kMmaWarp = 1;
 constexpr int kEpiWarp0 = 2;                  // warps 2..5
 constexpr int kDeqWarp0 = 6;                  // warps 6..21
 constexpr int kDeqWarps = 16;
+constexpr int kDeqGroups = 2;                 // CTA-pair kernel: dequantising warp groups taking alternate stages
 constexpr int kThreads = (kDeqWarp0 + kDeqWarps) * 32;   // 704
 constexpr uint64_t kWaitLimit = kWaitLimitNs;
 
@@ -84,6 +86,25 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar)
 }
 
 // 32 consecutive f32 columns of this warp's 32 accumulator lanes.
+// 32 consecutive f32 columns of this warp's 32 tensor-memory lanes, without waiting
+// (tmem_wait_ld makes them usable).
+__device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, uint32_t (&r)[32])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld()
+{
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32])
 {
     asm volatile(
@@ -484,15 +505,27 @@ __device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t a_desc, 
         : "memory");
 }
 
-// Arrive once on the mbarrier at the same offset in both CTAs of the pair when every
-// tcgen05 operation this thread issued so far has completed.
-__device__ __forceinline__ void mma_commit_pair(uint64_t* bar)
+// Arrive once on the mbarrier at the same offset in both CTAs of the pair (the cluster
+// ranks set in `mask`) when every tcgen05 operation this thread issued so far has completed.
+__device__ __forceinline__ void mma_commit_pair(uint64_t* bar, uint16_t mask)
 {
     asm volatile(
         "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
             smem_addr(bar)),
-        "h"((uint16_t)3)
+        "h"(mask)
         : "memory");
+}
+
+// Four floats from the shared memory of a CTA of this cluster (address from peer_addr).
+// No memory clobber: the loads read data fixed by an earlier cluster barrier, so several
+// may be in flight at once.
+__device__ __forceinline__ float4 ld_cluster_f4(uint32_t cluster_addr)
+{
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(cluster_addr));
+    return v;
 }
 
 template <int BNP>
@@ -511,7 +544,12 @@ struct PairCfg {
     static_assert(kStageBytes % 1024 == 0, "stage alignment");
 };
 
-template <int BNP>
+// SPL > 1: a cluster of SPL pairs computes one pair tile, pair j over the j-th of SPL
+// consecutive k ranges; after its last MMA each CTA stages its f32 partial tile in its
+// own stage ring (idle by then), and each CTA sums the SPL partials of its 128 rows over
+// 1/SPL of the columns through distributed shared memory, in pair order, and stores them
+// as bf16.  One tile per cluster: the launch has one cluster per tile.
+template <int BNP, int SPL>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_codes,
                  const __grid_constant__ CUtensorMap tm_scales, const GemmArgs a)
@@ -535,14 +573,22 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const uint32_t rank = cluster_rank();
-    const int cluster = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
+    const uint32_t crank = cluster_rank();
+    const uint32_t rank = crank & 1u;                    // half of the pair
+    const uint32_t lead = crank & ~1u;                   // cluster rank of the pair's MMA CTA
+    const uint16_t pair_mask = (uint16_t)(3u << lead);
+    const int ks = (int)(crank >> 1);                    // k range of this pair
+    const int kb0 = ks * a.kblocks / SPL, kb1 = (ks + 1) * a.kblocks / SPL;
+    const int cluster = blockIdx.x / (2 * SPL), nclusters = gridDim.x / (2 * SPL);
     const int tiles = a.tiles_m * a.tiles_n;
+    float* stg = reinterpret_cast<float*>(smem);         // SPL > 1: staged partial tile, [128][kStgStride]
+    constexpr int kStgStride = BNP + 4;                  // floats per staged row (spreads the banks)
+    static_assert(SPL == 1 || 128 * kStgStride * 4 <= S * C::kStageBytes, "staging fits the ring");
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&bready[s], 2 * kDeqWarps);
+            mbar_init(&bready[s], 2 * kDeqWarps / kDeqGroups);
             mbar_init(&empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -581,7 +627,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
             for (int t = cluster; t < tiles && !*abort_flag; t += nclusters) {
                 const int m0 = (t % a.tiles_m) * 256 + (int)rank * 128;
                 const int n0 = (t / a.tiles_m) * BNP + (int)rank * BH;
-                for (int kb = 0; kb < a.kblocks; ++kb, ++it) {
+                for (int kb = kb0; kb < kb1; ++kb, ++it) {
                     const int s = it % S;
                     const uint32_t ph = (uint32_t)(it / S) & 1u;
                     if (!mbar_wait_cluster_bounded(&empty[s], ph ^ 1u, kWaitLimit)) { fail(); break; }
@@ -601,7 +647,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
                     if (last_phase[s] >= 0) mbar_wait_bounded(&full[s], (uint32_t)last_phase[s], kWaitLimit);
         }
     } else if (warp == kMmaWarp) {
-        if (rank == 0 && lane == 0) {
+        if (rank == 0 && lane == 0) {                      // the pair's even CTA issues its MMAs
             constexpr uint32_t idesc = instr_desc(256, BNP);
             int it = 0, tcount = 0;
             bool issued_any = false;
@@ -613,7 +659,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
                 }
                 tc_fence_after();
                 bool ok = true;
-                for (int kb = 0; kb < a.kblocks; ++kb, ++it) {
+                for (int kb = kb0; kb < kb1; ++kb, ++it) {
                     const int s = it % S;
                     if (!mbar_wait_cluster_bounded(&bready[s], (uint32_t)(it / S) & 1u, kWaitLimit)) {
                         fail();
@@ -627,15 +673,15 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
 #pragma unroll
                     for (int j = 0; j < kBK / 16; ++j)
                         mma_bf16_pair(d, sw128_desc(st + j * 32), sw128_desc(st + C::kABytes + j * 32), idesc,
-                                      (kb > 0 || j > 0) ? 1u : 0u);
-                    mma_commit_pair(&empty[s]);    // both CTAs' stages reusable once these MMAs have read them
+                                      (kb > kb0 || j > 0) ? 1u : 0u);
+                    mma_commit_pair(&empty[s], pair_mask);   // both CTAs' stages reusable once read
                     issued_any = true;
                 }
                 if (!ok) break;
-                mma_commit_pair(&accfull[buf]);
+                mma_commit_pair(&accfull[buf], pair_mask);
             }
             if (*abort_flag && issued_any) {
-                mma_commit_pair(drain);
+                mma_commit_pair(drain, pair_mask);
                 mbar_wait_bounded(drain, 0, kWaitLimit);
             }
         }
@@ -643,15 +689,35 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
         const int quad = warp & 3;             // tensor-memory lanes 32*quad .. 32*quad+31
         int tcount = 0;
         const bool vec_ok = (a.N % 8) == 0 && (reinterpret_cast<uintptr_t>(a.y) & 15) == 0;
-        const uint32_t accempty0 = peer_addr(accempty, 0);     // CTA 0's accempty[0]; buffer b at + 8 b
+        const uint32_t accempty0 = peer_addr(accempty, lead);  // the MMA CTA's accempty[0]; buffer b at + 8 b
         for (int t = cluster; t < tiles && !*abort_flag; t += nclusters, ++tcount) {
             const int buf = tcount & 1;
             if (!mbar_wait_cluster_bounded(&accfull[buf], (uint32_t)(tcount >> 1) & 1u, kWaitLimit)) { fail(); break; }
             tc_fence_after();
             const int row = (t % a.tiles_m) * 256 + (int)rank * 128 + quad * 32 + lane;
             const int n0 = (t / a.tiles_m) * BNP;
+            if constexpr (SPL > 1) {
+                // stage the f32 partial tile (64 columns per tensor-memory wait); the
+                // reduction after the role loops stores y
 #pragma unroll 1
-            for (int c0 = 0; c0 < BNP; c0 += 32) {
+                for (int c0 = 0; c0 < BNP; c0 += 64) {
+                    uint32_t r0[32], r1[32];
+                    const uint32_t ta = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(buf * BNP + c0);
+                    tmem_ld32_nowait(ta, r0);
+                    tmem_ld32_nowait(ta + 32, r1);
+                    tmem_wait_ld();
+                    float4* dst = reinterpret_cast<float4*>(stg + (quad * 32 + lane) * kStgStride + c0);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        dst[q] = make_float4(__uint_as_float(r0[4 * q]), __uint_as_float(r0[4 * q + 1]),
+                                             __uint_as_float(r0[4 * q + 2]), __uint_as_float(r0[4 * q + 3]));
+                        dst[8 + q] = make_float4(__uint_as_float(r1[4 * q]), __uint_as_float(r1[4 * q + 1]),
+                                                 __uint_as_float(r1[4 * q + 2]), __uint_as_float(r1[4 * q + 3]));
+                    }
+                }
+            }
+#pragma unroll 1
+            for (int c0 = 0; c0 < (SPL > 1 ? 0 : BNP); c0 += 32) {
                 uint32_t r[32];
                 tmem_ld32(tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(buf * BNP + c0), r);
                 const int col = n0 + c0;
@@ -679,33 +745,34 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
             if (lane == 0) mbar_arrive_cluster(accempty0 + 8u * (uint32_t)buf);
         }
     } else {
-        // Dequantise this CTA's BH weight rows of every stage; each thread owns BH*8/512
-        // chunks (row n, 16-byte k chunk c).
-        const int dt = threadIdx.x - kDeqWarp0 * 32;
-        constexpr int kChunks = BH * 8 / (kDeqWarps * 32);
+        // Dequantise this CTA's BH weight rows.  The dequantising warps form kDeqGroups
+        // groups that take alternate stages, so a group has kDeqGroups stage periods for
+        // the latency of one stage (shared-memory reads, the proxy fence and the remote
+        // arrival); each thread owns BH*8/(threads of a group) chunks (row n, 16-byte k
+        // chunk c) of its stages.
+        constexpr int kGroupThreads = kDeqWarps * 32 / kDeqGroups;
+        const int dq = threadIdx.x - kDeqWarp0 * 32;
+        const int grp = dq / kGroupThreads, dt = dq - grp * kGroupThreads;
+        constexpr int kChunks = BH * 8 / kGroupThreads;
         const DequantConsts dk;
-        const uint32_t bready0 = peer_addr(bready, 0);         // CTA 0's bready[0]; stage s at + 8 s
+        const uint32_t bready0 = peer_addr(bready, lead);      // the MMA CTA's bready[0]; stage s at + 8 s
         int it = 0;
         for (int t = cluster; t < tiles && !*abort_flag; t += nclusters) {
             const int n0 = (t / a.tiles_m) * BNP + (int)rank * BH;
-            float sc0[kChunks], sc1[kChunks], sc2[kChunks];
-            auto load_scales = [&](int kb, float (&dst)[kChunks]) {
-#pragma unroll
-                for (int q = 0; q < kChunks; ++q) {
-                    const int idx = dt + q * kDeqWarps * 32;
-                    const int n = n0 + idx / 8, g = kb * 2 + (idx & 7) / 4;
-                    dst[q] = (kb < a.kblocks && n < a.N && g < a.G)
-                                 ? __half2float(__ushort_as_half(__ldg(a.scales + (size_t)n * a.G + g)))
-                                 : 0.f;
-                }
-            };
-            if (!a.scale_tma) {
-                load_scales(0, sc0);
-                load_scales(1, sc1);
-            }
             bool ok = true;
-            for (int kb = 0; kb < a.kblocks; ++kb, ++it) {
-                if (!a.scale_tma) load_scales(kb + 2, sc2);
+            for (int kb = kb0; kb < kb1; ++kb, ++it) {
+                if (it % kDeqGroups != grp) continue;
+                float scv[kChunks];
+                if (!a.scale_tma) {                // issued before the wait, which hides their latency
+#pragma unroll
+                    for (int q = 0; q < kChunks; ++q) {
+                        const int idx = dt + q * kGroupThreads;
+                        const int n = n0 + idx / 8, g = kb * 2 + (idx & 7) / 4;
+                        scv[q] = (n < a.N && g < a.G)
+                                     ? __half2float(__ushort_as_half(__ldg(a.scales + (size_t)n * a.G + g)))
+                                     : 0.f;
+                    }
+                }
                 const int s = it % S;
                 if (!mbar_wait_bounded(&full[s], (uint32_t)(it / S) & 1u, kWaitLimit)) { fail(); ok = false; break; }
                 if (*abort_flag) { ok = false; break; }
@@ -715,20 +782,15 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
                 const __half* sst = reinterpret_cast<const __half*>(raw + C::kRawBytes);
 #pragma unroll
                 for (int q = 0; q < kChunks; ++q) {
-                    const int idx = dt + q * kDeqWarps * 32;
+                    const int idx = dt + q * kGroupThreads;
                     const int n = idx >> 3, c = idx & 7;
                     const uint32_t v = *reinterpret_cast<const uint32_t*>(raw + n * 32 + c * 4);
-                    const float sc = a.scale_tma ? __half2float(sst[n * 8 + ((kb * 2 + c / 4) & 7)]) : sc0[q];
+                    const float sc = a.scale_tma ? __half2float(sst[n * 8 + ((kb * 2 + c / 4) & 7)]) : scv[q];
                     *reinterpret_cast<uint4*>(bt + n * 128 + ((c ^ (n & 7)) << 4)) = dequant8(v, sc, dk);
                 }
                 fence_proxy_async_smem();      // generic-proxy writes -> tensor-core reads
                 __syncwarp();
                 if (lane == 0) mbar_arrive_cluster(bready0 + 8u * (uint32_t)s);
-#pragma unroll
-                for (int q = 0; q < kChunks; ++q) {
-                    sc0[q] = sc1[q];
-                    sc1[q] = sc2[q];
-                }
             }
             if (!ok) break;
         }
@@ -737,15 +799,70 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
     tc_fence_before();
     __syncthreads();
     cluster_sync_all();                  // no CTA leaves while the pair's MMAs may read its shared memory
+    if constexpr (SPL > 1) {
+        // Every CTA's partial tile is staged (the cluster barrier orders the writes).  This
+        // CTA stores columns [ks, ks + 1) * BNP / SPL of its 128 rows: the sum of the SPL
+        // pairs' partials of the same half, in pair order.
+        const int t = cluster;
+        if (t < tiles) {
+            constexpr int kCols = BNP / SPL;
+            const int row0 = (t % a.tiles_m) * 256 + (int)rank * 128;
+            const int col0 = (t / a.tiles_m) * BNP + ks * kCols;
+            uint32_t src[SPL];
+#pragma unroll
+            for (int j = 0; j < SPL; ++j) src[j] = peer_addr(stg, 2u * (uint32_t)j + rank);
+            const bool vec_ok = (a.N % 4) == 0 && (reinterpret_cast<uintptr_t>(a.y) & 7) == 0;
+            // kBatch float4 of every partial in flight per thread before the sums
+            constexpr int kQuads = 128 * (kCols / 4), kBatch = 4;
+            for (int e0 = threadIdx.x; e0 < kQuads; e0 += kBatch * (int)blockDim.x) {
+                float4 v[kBatch][SPL];
+#pragma unroll
+                for (int b = 0; b < kBatch; ++b) {
+                    const int e = min(e0 + b * (int)blockDim.x, kQuads - 1);
+                    const int rr = e / (kCols / 4), cc = (e - rr * (kCols / 4)) * 4;
+                    const uint32_t off = (uint32_t)((rr * kStgStride + ks * kCols + cc) * 4);
+#pragma unroll
+                    for (int j = 0; j < SPL; ++j) v[b][j] = ld_cluster_f4(src[j] + off);
+                }
+#pragma unroll
+                for (int b = 0; b < kBatch; ++b) {
+                    const int e = e0 + b * (int)blockDim.x;
+                    if (e >= kQuads) break;
+                    float4 acc = v[b][0];
+#pragma unroll
+                    for (int j = 1; j < SPL; ++j) {
+                        acc.x += v[b][j].x;
+                        acc.y += v[b][j].y;
+                        acc.z += v[b][j].z;
+                        acc.w += v[b][j].w;
+                    }
+                    const int rr = e / (kCols / 4), cc = (e - rr * (kCols / 4)) * 4;
+                    const int row = row0 + rr, col = col0 + cc;
+                    if (row < a.M && col < a.N) {
+                        uint16_t* dst = a.y + (size_t)row * a.N + col;
+                        if (vec_ok && col + 4 <= a.N) {
+                            *reinterpret_cast<uint2*>(dst) =
+                                make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
+                        } else {
+                            const float f[4] = {acc.x, acc.y, acc.z, acc.w};
+                            for (int q = 0; q < 4 && col + q < a.N; ++q)
+                                dst[q] = (uint16_t)(pack_bf16x2(f[q], 0.f) & 0xFFFFu);
+                        }
+                    }
+                }
+            }
+        }
+        cluster_sync_all();              // no CTA leaves while the others read its staged tile
+    }
     tc_fence_after();
     if (warp == kMmaWarp) tmem_dealloc2(tmem_base, C::kTmemCols);
 }
 
-template <int BNP>
+template <int BNP, int SPL>
 bool setup_pair_kernel(size_t* smem)
 {
     *smem = PairCfg<BNP>::kSmem;
-    const void* fn = reinterpret_cast<const void*>(&gemm_pair_kernel<BNP>);
+    const void* fn = reinterpret_cast<const void*>(&gemm_pair_kernel<BNP, SPL>);
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 0) != cudaSuccess) {
         cudaGetLastError();
     }
@@ -763,8 +880,53 @@ bool setup_kernel(size_t* smem)
 
 namespace {
 
-// The CTA-pair kernel with BNP output columns per pair tile.
-template <int BNP>
+std::mutex g_cluster_mutex;
+struct ClusterCap {
+    int device;
+    const void* fn;
+    int capacity;
+};
+ClusterCap g_cluster_cap[16];
+int g_cluster_cap_used = 0;
+
+// How many clusters of the pair kernel <BNP, SPL> (2 * SPL CTAs each) can be resident
+// at once on the current device (0 when none can, or the query fails); cached.
+template <int BNP, int SPL>
+int pair_cluster_capacity(const DeviceInfo& dev)
+{
+    const void* fn = reinterpret_cast<const void*>(&gemm_pair_kernel<BNP, SPL>);
+    {
+        std::lock_guard<std::mutex> lock(g_cluster_mutex);
+        for (int i = 0; i < g_cluster_cap_used; ++i)
+            if (g_cluster_cap[i].device == dev.device && g_cluster_cap[i].fn == fn) return g_cluster_cap[i].capacity;
+    }
+    size_t smem = 0;
+    int capacity = 0;
+    if (setup_pair_kernel<BNP, SPL>(&smem)) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)(2 * SPL));
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = smem;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2 * SPL;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaOccupancyMaxActiveClusters(&capacity, gemm_pair_kernel<BNP, SPL>, &cfg) != cudaSuccess) {
+            cudaGetLastError();
+            capacity = 0;
+        }
+    }
+    std::lock_guard<std::mutex> lock(g_cluster_mutex);
+    if (g_cluster_cap_used < 16) g_cluster_cap[g_cluster_cap_used++] = {dev.device, fn, capacity};
+    return capacity;
+}
+
+// The CTA-pair kernel with BNP output columns per pair tile; SPL pairs per cluster split
+// K (one tile per cluster), SPL == 1 is persistent over the tiles.
+template <int BNP, int SPL>
 q4_status launch_gemm_pair(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed, const uint16_t* scales,
                            int64_t N, uint16_t* y, cudaStream_t stream, const DeviceInfo& dev)
 {
@@ -796,10 +958,10 @@ q4_status launch_gemm_pair(const uint16_t* x, int64_t M, int64_t K, const uint8_
     a.kblocks = (int)((K + kBK - 1) / kBK);
     const long long tiles = (long long)a.tiles_m * a.tiles_n;
     size_t smem = 0;
-    if (!setup_pair_kernel<BNP>(&smem)) return Q4_ERR_CUDA;
-    const long long clusters = std::min<long long>(tiles, dev.sm_count / 2);
+    if (!setup_pair_kernel<BNP, SPL>(&smem)) return Q4_ERR_CUDA;
+    const long long clusters = SPL > 1 ? tiles : std::min<long long>(tiles, dev.sm_count / 2);
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(2 * clusters));
+    cfg.gridDim = dim3((unsigned)(2 * SPL * clusters));
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
@@ -807,12 +969,12 @@ q4_status launch_gemm_pair(const uint16_t* x, int64_t M, int64_t K, const uint8_
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
     attr[1].id = cudaLaunchAttributeClusterDimension;
-    attr[1].val.clusterDim.x = 2;
+    attr[1].val.clusterDim.x = 2 * SPL;
     attr[1].val.clusterDim.y = 1;
     attr[1].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel<BNP>, tm_x, tm_codes, tm_scales, a);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel<BNP, SPL>, tm_x, tm_codes, tm_scales, a);
     return e == cudaSuccess ? Q4_OK : Q4_ERR_CUDA;
 }
 
@@ -821,14 +983,22 @@ q4_status launch_gemm_pair(const uint16_t* x, int64_t M, int64_t K, const uint8_
 q4_status launch_gemm(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed, const uint16_t* scales,
                       int64_t N, uint16_t* y, cudaStream_t stream, const DeviceInfo& dev)
 {
-    // CTA pairs (256-row tiles) from M = 256 on.  A 256 x 128 pair tile is bound by the
-    // latency of its stage ring (measured on B200: about 0.45 us per 64-k block against
-    // 0.55 us for a 256 x 256 tile, which does twice the work), so 256 x 256 tiles are
-    // used whenever they occupy at least half of the SM pairs.
+    // CTA pairs (256-row tiles) from M = 256 on.  A pair's k-block takes about the same
+    // time with 128 output columns as with 256 (measured on B200: 0.45-0.5 us against
+    // 0.55-0.6 us), so 256 x 256 tiles are used throughout; when they leave SM pairs idle,
+    // 4 or 2 pairs share each tile's K range (clusters of 8 or 4 CTAs, each pair at least
+    // 4 k-blocks) as long as every cluster can be resident at once; else 256 x 128 tiles
+    // when 256 x 256 ones would occupy fewer than half of the pairs.
     if (M >= 256 && dev.sm_count >= 2) {
         const long long p256 = ((M + 255) / 256) * ((N + 255) / 256);
-        if (2 * p256 >= dev.sm_count / 2) return launch_gemm_pair<256>(x, M, K, packed, scales, N, y, stream, dev);
-        return launch_gemm_pair<128>(x, M, K, packed, scales, N, y, stream, dev);
+        const long long pairs = dev.sm_count / 2;
+        const long long kblocks = (K + kBK - 1) / kBK;
+        if (p256 * 4 <= pairs && kblocks >= 16 && pair_cluster_capacity<256, 4>(dev) >= p256)
+            return launch_gemm_pair<256, 4>(x, M, K, packed, scales, N, y, stream, dev);
+        if (p256 * 2 <= pairs && kblocks >= 8 && pair_cluster_capacity<256, 2>(dev) >= p256)
+            return launch_gemm_pair<256, 2>(x, M, K, packed, scales, N, y, stream, dev);
+        if (2 * p256 >= pairs) return launch_gemm_pair<256, 1>(x, M, K, packed, scales, N, y, stream, dev);
+        return launch_gemm_pair<128, 1>(x, M, K, packed, scales, N, y, stream, dev);
     }
     // Tile shape: 256 x 128 when that still gives every SM a tile, else 128 x 128, else 128 x 64.
     const long long t256 = ((M + 255) / 256) * ((N + 127) / 128);

@@ -17,22 +17,22 @@
 //    Skinny shapes may also split K across blocks (last-arriver reduction, no
 //    waiting).  The plan picks splits, P and teams per block with a small cost model.
 //  * Arithmetic per mode:
-//      M = 1 (kImma1, f32 or bf16 x): no code becomes a float.  Each group of 32 x values
-//          is scaled by a power of two 2^F_g (max |x| of the group * 2^F_g < 2^30),
+//      M = 1 (kImma1, f32 or bf16 x): no code becomes a float.  Each box of 256 x values
+//          (8 groups) is scaled by a power of two 2^F (max |x| of the box * 2^F < 2^30),
 //          rounded once to integers and cut into four balanced base-256 digit planes;
 //          the codes stay bytes (even k as is, odd k at 16 x code, one AND each) and
 //          mma.sync.m16n8k32 (u8 codes x s8 digits) sums code x digit exactly in int32,
 //          the eight B columns being (plane, even/odd half).  The C operand, a bias
 //          0x4B400000 minus 8 (or 128) x the digit sum, removes the code offset 8 and
 //          makes the int32 result the bit pattern of the exact float 1.5 * 2^23 + sum.
-//          Each group's sum is multiplied by its scale times 2^-F_g and accumulated in
-//          f32 per plane; the planes are combined at the end.
+//          Each group's sum is multiplied by its scale, the box's sums by 2^-F, and
+//          accumulated in f32 per plane; the planes are combined at the end.
 //      M = 2..16 (bf16 x): nibble pair (j, j+4) of a word OR-ed into 0x4300 (one LOP3)
-//          is the bf16 pair (128 + c_j, 128 + c_{j+4}); such pairs, read with ldmatrix,
-//          are the A operand of mma.sync.m16n8k16 (f32 accumulate) and x rows the B
-//          operand, in a permuted k order that matches the pairs.  The MMA's C operand
-//          is -136 * sum(x) of the group (an f64 sum rounded once), so each result is
-//          the exact group dot product up to f32 accumulation.
+//          is the bf16 pair (128 + c_j, 128 + c_{j+4}); one exact bf16x2 subtraction of
+//          136 makes it (c_j - 8, c_{j+4} - 8).  Such pairs, read with ldmatrix, are the
+//          A operand of mma.sync.m16n8k16 and x rows the B operand, in a permuted k order
+//          that matches the pairs; every product is exact and the group's sum is
+//          accumulated in f32 from zero.
 //    In every mode each group's sum is scaled by its binary16 scale and added in f32.
 //  * Every mbarrier wait is bounded.  If one runs out the kernel records
 //    kErrWaitTimeout in the library error word, stops issuing and computing, waits
@@ -149,6 +149,24 @@ __device__ __forceinline__ uint32_t nib_pair(uint32_t v, int j, uint32_t mask, u
     return and_or(v >> (4 * j), mask, magic);
 }
 
+// (128 + c) - 136 = c - 8 for both bf16 halves; exact (small integers).
+__device__ __forceinline__ uint32_t sub_bf16x2(uint32_t a, uint32_t b)
+{
+    uint32_t r;
+    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+// d = A . B for one m16n8k16 tile (bf16 inputs, f32 accumulate from zero).
+__device__ __forceinline__ void mma_bf16_16816_z(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                                 uint32_t b0, uint32_t b1)
+{
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%10,%10,%10,%10};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.0f));
+}
+
 // Four 8x8 b16 matrices from shared memory; lane 8i + r supplies the address of row r of
 // matrix i and lane (g, t) receives the 32-bit word (row g, columns 2t, 2t+1) of each.
 __device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3)
@@ -159,15 +177,6 @@ __device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t& r0, uint32_
 }
 
 // d = A . B + c for one m16n8k16 tile (bf16 inputs, f32 accumulate).
-__device__ __forceinline__ void mma_bf16_16816_c(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                                 uint32_t b0, uint32_t b1, const float4 c)
-{
-    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%10,%11,%12,%13};"
-        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(c.x), "f"(c.y), "f"(c.z), "f"(c.w));
-}
-
 // d += A . B for one m16n8k16 tile (bf16 inputs, f32 accumulate).
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                                uint32_t b0, uint32_t b1)
@@ -218,16 +227,6 @@ __device__ __forceinline__ uint4 pairs_of(const uint4 raw)
     // raw holds x_0..x_7 as (x0,x1)(x2,x3)(x4,x5)(x6,x7); regroup to (x_j, x_{j+4}).
     return make_uint4(__byte_perm(raw.x, raw.z, 0x5410), __byte_perm(raw.x, raw.z, 0x7632),
                       __byte_perm(raw.y, raw.w, 0x5410), __byte_perm(raw.y, raw.w, 0x7632));
-}
-
-__device__ __forceinline__ double sum8_bf16(const uint4 raw)
-{
-    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-    double s = 0.0;
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-        s += (double)__uint_as_float(w[i] << 16) + (double)__uint_as_float(w[i] & 0xFFFF0000u);
-    return s;
 }
 
 // Eight x values (k = 8t .. 8t+7 of a group) as balanced base-256 digit planes of
@@ -302,6 +301,7 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
     constexpr int kTkM = MODE == kImma1 ? 1 : MP;                         // x rows of a top-k list set
     extern __shared__ unsigned char smem_raw[];
     __shared__ int s_last[kMaxWarps];
+    __shared__ unsigned long long s_best[kArgmax ? kMaxWarps : 1];        // argmax, one x row
     __shared__ uint64_t s_xbar;                                            // kMma*: x rows in flight
     const int W = blockDim.x >> 5;
     unsigned char* smem =
@@ -405,9 +405,7 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
     // ---- stage x for this split (zero past the split and past K) ----
     //  kMma* : bf16 pairs [m][group][word][4] for m < M, then one zero row that lanes
     //          of x rows >= M read; each row is padded by one group so that lanes of
-    //          neighbouring x rows fall on different banks.  Beside it, per group, -136 *
-    //          sum(x) of the group for each x row (an f64 sum of the bf16 values, rounded
-    //          once), laid out [group][n-tile][t] as the accumulator fragment of lane (g, t).
+    //          neighbouring x rows fall on different banks.
     //  kImma1: each box of 8 groups (256 x values) is scaled by 2^F (the largest F with
     //          max |x| of the box * 2^F < 2^30, at most 100), rounded to integers X and
     //          cut into four balanced base-256 digits X = d0 2^24 + d1 2^16 + d2 2^8 + d3,
@@ -421,7 +419,6 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
     //          bias - 128 sum(d of odd k) for half 1, which removes the code offset 8.
     //          Then [box] float: 2^-F.  One pass: the 32 lanes that stage a box find its
     //          maximum with five shuffles, so no block-wide reduction is needed.
-    float* xoff = nullptr;
     const int rs = (ngp + 1) * 4;                                         // uint4 per staged x row
     bool x_ok = true;                                                     // kMma*: x rows arrived
     if constexpr (MODE == kImma1) {
@@ -503,7 +500,6 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
         }
     } else {
         uint4* xp = reinterpret_cast<uint4*>(xst);
-        xoff = reinterpret_cast<float*>(xp + (a.M + 1) * rs);
         // The split's part of each x row arrives by one bulk copy, straight where its
         // staged words go (all rows in flight at once), and is then permuted in place.
         if (threadIdx.x == 0) {
@@ -517,40 +513,18 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
         __syncthreads();
         x_ok = mbar_wait_bounded(&s_xbar, 0, kWaitLimit);
         const int total = (a.M + 1) * ngp * 4;
-        for (int i0 = threadIdx.x - lane; i0 < total; i0 += blockDim.x) {    // warp-uniform trips
-            const int i = i0 + lane;
+        for (int i = threadIdx.x; i < total; i += blockDim.x) {
             const int m = i / (ngp * 4);
             const int rem = i - m * ngp * 4;
-            const int lg = rem >> 2;
-            const int wd = rem & 3;
             uint4 raw = make_uint4(0u, 0u, 0u, 0u);
-            if (i < total && m < a.M && lg < ng && x_ok) raw = xp[m * rs + rem];
-            if (i < total) xp[m * rs + rem] = pairs_of(raw);
-            double sum = sum8_bf16(raw);
-            sum += __shfl_xor_sync(0xffffffffu, sum, 1);                    // words (0,1) and (2,3)
-            sum += __shfl_xor_sync(0xffffffffu, sum, 2);                    // all four words
-            if (i < total && wd == 0 && m < a.M) {
-                // the accumulator fragment of lane (g, t) holds columns 2t, 2t+1 in both row halves
-                const float o = (float)(-136.0 * sum);
-                const int n = m >> 3, col = m & 7;
-                float* q = xoff + (((size_t)lg * NT + n) * 4 + (col >> 1)) * 4 + (col & 1);
-                q[0] = o;
-                q[2] = o;
-            }
-        }
-        for (int i = threadIdx.x; i < ngp * MP; i += blockDim.x) {
-            const int lg = i / MP, m = i - lg * MP;
-            if (m >= a.M) {
-                const int n = m >> 3, col = m & 7;
-                float* q = xoff + (((size_t)lg * NT + n) * 4 + (col >> 1)) * 4 + (col & 1);
-                q[0] = 0.f;
-                q[2] = 0.f;
-            }
+            if (m < a.M && (rem >> 2) < ng && x_ok) raw = xp[m * rs + rem];
+            xp[m * rs + rem] = pairs_of(raw);
         }
     }
     __syncthreads();
 
     const uint32_t kmask = pinned_u32(0x000F000Fu), kmagic = pinned_u32(0x43004300u);
+    const uint32_t k136 = pinned_u32(0x43084308u);                        // bf16x2 (136, 136)
     // MMA modes: lane (g, t) supplies the B operand of x row n * 8 + g (the zero row past M).
     const uint4* xrow[NT];
 #pragma unroll
@@ -566,7 +540,11 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
     // so the largest one published so far (tk_floor) is a bar no row below it can pass.
     // A team reads it when it starts a row block and publishes its own when it rises.
     constexpr bool kFloor = kTopk && kTkM == 1;
-    unsigned long long floor_now = 0ull, floor_pub = 0ull;
+    unsigned long long floor_now = 0ull, floor_pub = 0ull, tk_last = 0ull;   // tk_last: the list's k-th key
+    // Argmax with one x row: the best key of the rows this lane has reported so far; the
+    // block reduces them once at the end (a global atomic per row block would queue on
+    // one L2 address).
+    unsigned long long am_best = 0ull;
     int jnext = 0;                                         // this warp's next job
     for (int rbi = 0; rbi < nrb; ++rbi) {
         const int rb = rb_of(rbi);
@@ -703,20 +681,18 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
                                     for (int h = 0; h < 2; ++h) {
                                         const int c = 2 * cp + h;
                                         const uint32_t w0 = h ? r2 : r0, w1 = h ? r3 : r1;
-                                        const uint32_t A0 = nib_pair(w0, 0, kmask, kmagic);
-                                        const uint32_t A1 = nib_pair(w1, 0, kmask, kmagic);
-                                        const uint32_t A2 = nib_pair(w0, 1, kmask, kmagic);
-                                        const uint32_t A3 = nib_pair(w1, 1, kmask, kmagic);
-                                        const uint32_t A4 = nib_pair(w0, 2, kmask, kmagic);
-                                        const uint32_t A5 = nib_pair(w1, 2, kmask, kmagic);
-                                        const uint32_t A6 = nib_pair(w0, 3, kmask, kmagic);
-                                        const uint32_t A7 = nib_pair(w1, 3, kmask, kmagic);
+                                        const uint32_t A0 = sub_bf16x2(nib_pair(w0, 0, kmask, kmagic), k136);
+                                        const uint32_t A1 = sub_bf16x2(nib_pair(w1, 0, kmask, kmagic), k136);
+                                        const uint32_t A2 = sub_bf16x2(nib_pair(w0, 1, kmask, kmagic), k136);
+                                        const uint32_t A3 = sub_bf16x2(nib_pair(w1, 1, kmask, kmagic), k136);
+                                        const uint32_t A4 = sub_bf16x2(nib_pair(w0, 2, kmask, kmagic), k136);
+                                        const uint32_t A5 = sub_bf16x2(nib_pair(w1, 2, kmask, kmagic), k136);
+                                        const uint32_t A6 = sub_bf16x2(nib_pair(w0, 3, kmask, kmagic), k136);
+                                        const uint32_t A7 = sub_bf16x2(nib_pair(w1, 3, kmask, kmagic), k136);
 #pragma unroll
                                         for (int n = 0; n < NT; ++n) {
                                             const uint4 bx = xrow[n][(gb + c) * 4 + t];
-                                            const float4 o4 = reinterpret_cast<const float4*>(
-                                                xoff)[((gb + c) * NT + n) * 4 + t];      // -136 * sum(x)
-                                            mma_bf16_16816_c(d[c - c0][n], A0, A1, A2, A3, bx.x, bx.y, o4);
+                                            mma_bf16_16816_z(d[c - c0][n], A0, A1, A2, A3, bx.x, bx.y);
                                             mma_bf16_16816(d[c - c0][n], A4, A5, A6, A7, bx.z, bx.w);
                                         }
                                     }
@@ -810,26 +786,35 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
                 }
                 return live ? argmax_key(total, a.row_base + (uint32_t)(lrow0 + rr)) : 0ull;
             };
-            if constexpr (kTopk) {                      // lanes 0-15: x row 2h, lanes 16-31: x row 2h + 1
+            if constexpr (kFloor) {
+                // One x row: lanes 0-15 hold the block's 16 rows.  Most blocks have no row
+                // above the list's k-th key (tk_last) or the published floor, and skip the
+                // insert after one vote.
+                const unsigned long long key = rows_out(0);
+                const unsigned long long bar = key_max(tk_last, floor_now);
+                if (__any_sync(0xffffffffu, lane < 16 && key > bar)) {
+                    topk_insert(tk[0], key, lane < 16, a.tk_k, lane, floor_now);
+                    tk_last = __shfl_sync(0xffffffffu, tk[0], a.tk_k - 1);
+                    if (tk_last > floor_pub && tk_last > floor_now) {       // the same on every lane
+                        if (lane == 0) atomicMax(a.tk_floor, tk_last);
+                        floor_pub = tk_last;
+                    }
+                }
+            } else if constexpr (kTopk) {               // lanes 0-15: x row 2h, lanes 16-31: x row 2h + 1
 #pragma unroll
                 for (int h = 0; h < (kTkM + 1) / 2; ++h) {
                     if (h * 32 < kRows * a.M) {
                         const unsigned long long key = rows_out(h * 32);
-                        topk_insert(tk[2 * h], key, lane < 16, a.tk_k, lane, kFloor ? floor_now : 0ull);
-                        if constexpr (kFloor) {
-                            const unsigned long long kth = __shfl_sync(0xffffffffu, tk[0], a.tk_k - 1);
-                            if (kth > floor_pub && kth > floor_now) {       // the same on every lane
-                                if (lane == 0) atomicMax(a.tk_floor, kth);
-                                floor_pub = kth;
-                            }
-                        }
+                        topk_insert(tk[2 * h], key, lane < 16, a.tk_k, lane);
                         if (2 * h + 1 < kTkM) topk_insert(tk[2 * h + 1], key, lane >= 16, a.tk_k, lane);
                     }
                 }
             } else {
                 for (int e0 = 0; e0 < (kFuse ? 0 : kRows * a.M); e0 += 32) {
                     unsigned long long key = rows_out(e0);
-                    if constexpr (kArgmax) {            // the 16 lanes of one x row agree on its best row
+                    if constexpr (kArgmax && MODE == kImma1) {
+                        am_best = key_max(am_best, key);
+                    } else if constexpr (kArgmax) {     // the 16 lanes of one x row agree on its best row
                         const int m = (e0 + lane) / kRows;
 #pragma unroll
                         for (int o = 1; o < kRows; o <<= 1) {
@@ -871,6 +856,18 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
     if (!x_ok && threadIdx.x == 0) mbar_wait_bounded(&s_xbar, 0, kWaitLimit);   // x rows still in flight
 
     if constexpr (kArgmax) {                                // the last block to finish reports and resets
+        if constexpr (MODE == kImma1) {                     // the warps' best keys, then one atomic
+            unsigned long long k = am_best;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) k = key_max(k, __shfl_xor_sync(0xffffffffu, k, o));
+            if (lane == 0) s_best[warp] = k;
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                unsigned long long b = 0ull;
+                for (int w = 0; w < W; ++w) b = key_max(b, s_best[w]);
+                if (b) atomicMax(&a.am_key[0], b);
+            }
+        }
         __syncthreads();
         if (threadIdx.x == 0) {
             __threadfence();
@@ -928,30 +925,26 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
         __syncthreads();
         if (s_last[0]) {
             // The last block: S warps per x row each merge the lists of every S-th block
-            // (k keys each, padded with 0 to 32 lanes), then a tree of warp merges reduces
-            // the S slice lists of each x row to the result.
+            // (k keys each, padded with 0 to 32 lanes), with up to kDepth lists loaded at
+            // once, then a tree of warp merges reduces the S slice lists of each x row to
+            // the result.
             __threadfence();
+            constexpr int kDepth = 12;
             const int S = max(1, W / a.M);
             for (int job = warp; job < a.M * S; job += W) {
                 const int m = job / S, sl = job - m * S;
                 const unsigned long long* src = a.tk_cand + (size_t)m * gridDim.x * kk;
-                // the lists of blocks sl, sl + S, ...: four loads in flight ahead of the merges
-                auto fetch = [&](int b) {
-                    return (b < (int)gridDim.x && lane < kk) ? __ldcg(src + (size_t)b * kk + lane) : 0ull;
-                };
-                unsigned long long nxt[4];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) nxt[q] = fetch(sl + q * S);
                 unsigned long long list = 0ull;
-                for (int b0 = sl; b0 < (int)gridDim.x; b0 += 4 * S) {
-                    unsigned long long cur[4];
+                for (int b0 = sl; b0 < (int)gridDim.x; b0 += kDepth * S) {
+                    unsigned long long cur[kDepth];
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        cur[q] = nxt[q];
-                        nxt[q] = fetch(b0 + (4 + q) * S);
+                    for (int q = 0; q < kDepth; ++q) {
+                        const int b = b0 + q * S;
+                        cur[q] = (b < (int)gridDim.x && lane < kk) ? __ldcg(src + (size_t)b * kk + lane) : 0ull;
                     }
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) list = warp_merge_desc(list, cur[q], lane);
+                    for (int q = 0; q < kDepth; ++q)
+                        if (b0 + q * S < (int)gridDim.x) list = warp_merge_desc(list, cur[q], lane);   // warp-uniform
                 }
                 lists[(size_t)job * 32 + lane] = list;
             }
@@ -988,14 +981,14 @@ size_t per_warp_bytes(int mode)
     return (size_t)kStages * (kStageCodes + kStageScales + sizeof(uint64_t)) + (size_t)kRows * mp * sizeof(float);
 }
 
-// kImma1 per group: B operands 256 B, C operands 32 B, 2^-F_g 4 B, and with INT8
-// matrices in the launch the natural-order B operands, 256 B more.
+// kImma1 per group: B operands 256 B, C operands 32 B, 4 B for the boxes' 2^-F (one
+// float per box of 8 groups), and with INT8 matrices in the launch the natural-order B
+// operands, 256 B more.  kMma*: the M x rows and one zero row, each padded by a group.
 size_t x_stage_bytes(int mode, int nb, int64_t M, bool int8 = false)
 {
-    const int mp = mode == kMma16 ? 16 : mode == kMma8 ? 8 : 1;
     const size_t ngp = (size_t)nb * 8;
     if (mode == kImma1) return ngp * (int8 ? 548 : 292);
-    return (size_t)(M + 1) * (ngp + 1) * 64 + ngp * (mp / 8) * 64;
+    return (size_t)(M + 1) * (ngp + 1) * 64;
 }
 
 size_t smem_bytes(int mode, int warps, int nb, int64_t M, bool int8 = false)

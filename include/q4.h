@@ -148,13 +148,13 @@ Q4_API size_t q4_gemv_workspace_size(int64_t M, int64_t N, int64_t K);
  *              must start at zero (the arrival counters) at zero again, so the
  *              same workspace can be reused by later calls without clearing.
  *              Calls that share a workspace must not overlap on the GPU.
- * Arithmetic.  M = 1 (f32 or bf16 x): each group of 32 x values is scaled by a power of
- * two 2^F_g with max |x| * 2^F_g < 2^30, rounded once to integers and cut into four
+ * Arithmetic.  M = 1 (f32 or bf16 x): each box of 256 x values (8 groups) is scaled by a
+ * power of two 2^F with max |x| * 2^F < 2^30, rounded once to integers and cut into four
  * base-256 digits; the codes times the digits are summed exactly on the integer tensor
- * cores per group, and each group's sum is multiplied by its scale times 2^-F_g and
+ * cores per group, and each group's sum is multiplied by its scale, then by 2^-F, and
  * accumulated in f32 (per digit plane, combined at the end).  M >= 2 with bf16 x: the
- * codes are expanded exactly and multiplied by x on the bf16 tensor cores with f32
- * accumulation, each group's sum scaled and accumulated in f32.  Other shapes (f32 x
+ * codes become the bf16 values code - 8 exactly and multiply x on the bf16 tensor cores
+ * (exact products, f32 sums), each group's sum scaled and accumulated in f32.  Other shapes (f32 x
  * with M >= 2, K % 256 != 0, scales not 16-byte aligned): exact expansion and f32 FMAs.
  */
 Q4_API q4_status q4_gemv(const void* x, q4_dtype x_dtype, int64_t M, int64_t K,
@@ -317,9 +317,9 @@ Q4_API q4_status q4_topk_merge(const float* values, const int64_t* indices, int6
  *   (device, 16-byte aligned, the same contract as q4_gemv, so one x serves both formats),
  *   codes 16-byte aligned, scales 2-byte aligned, y 4-byte aligned.  M == 1 with
  *   K % 256 == 0 and 16-byte aligned scales runs on the Q4 GEMV's TMA kernel: x is cut
- *   into exact digit planes as for q4_gemv (per group of 32, max |x| * 2^F_g < 2^30) and
+ *   into exact digit planes as for q4_gemv (per box of 256, max |x| * 2^F < 2^30) and
  *   the codes multiply them on the integer tensor cores with exact int32 group sums, each
- *   scaled by its binary16 scale times 2^-F_g and accumulated in f32.  Other shapes stage
+ *   scaled by its binary16 scale and by 2^-F and accumulated in f32.  Other shapes stage
  *   x in shared memory as f32 (M*K*4 bytes; a shape whose x does not fit returns
  *   Q4_ERR_SHAPE) and form products in f32 per group of 16 k, scaled and accumulated in
  *   f32.  No workspace.  M == 0 or N == 0 is a no-op.

@@ -59,14 +59,13 @@ def f32_sum_bound(x: np.ndarray, deq: np.ndarray, roundings: int) -> np.ndarray:
     return gamma(roundings, U_CUDA_CORE) * (np.abs(x_f64(x)) @ np.abs(deq).T)
 
 
-def offset_path_bound(x: np.ndarray, scales: np.ndarray, roundings: int) -> np.ndarray:
-    """Bound for the bf16-activation path of M >= 2, which sums x_k * (128 + code_k) on
-    the tensor cores and removes 136 * sum(x) per half group: every partial is at most
-    144 * s_k * |x_k| per term, so |y - y_ref| <= gamma_n * sum_k |x_k| * 144 * s_k,
-    with the tensor-core unit roundoff."""
-    xa = np.abs(x_f64(x))
-    s = np.repeat(scales.view(np.float16).astype(np.float64), 32, axis=1)
-    return gamma(roundings, U_TENSOR_F32) * (xa @ (144.0 * s).T)
+def mma_path_bound(x: np.ndarray, deq: np.ndarray, roundings: int) -> np.ndarray:
+    """Bound for the bf16-activation path of M >= 2: the codes become the bf16 values
+    code - 8 exactly, so each product x_k (code_k - 8) is exact in f32; they are summed
+    inside the tensor-core MMAs (16 per instruction, chained over the group) and the
+    scaled group sums on CUDA cores.  Every rounding is bounded by the tensor-core unit
+    roundoff: |y - y_ref| <= gamma_n(2^-23) * sum_k |x_k w'_k|."""
+    return gamma(roundings, U_TENSOR_F32) * (np.abs(x_f64(x)) @ np.abs(deq).T)
 
 
 def digit_shift(x_group: np.ndarray) -> int:

@@ -68,13 +68,33 @@ def test_tile_128x128():
 
 
 @pytest.mark.parametrize("M,N,K", [
-    (2048, 2432, 128),     # 8 x 19 = 152 tiles of 256 x 128 (>= 148 SMs): the two-accumulator tile
-    (512, 2048, 256),      # the M = 512 prefill tiling (128 x 64 tiles)
-    (2176, 4160, 64),      # ragged in M and N at the 256 x 128 tiling
+    (2048, 2432, 128),     # 8 x 10 CTA-pair tiles of 256 x 256, ragged in N
+    (512, 2048, 256),      # 2 x 16 pair tiles of 256 x 128 (K too short to split)
+    (2176, 4160, 64),      # 9 x 17 = 153 pair tiles: pairs run two or three tiles each, ragged M and N
 ])
 def test_large_tiles_full_output(M, N, K):
     """Every output element of the large-tile paths against the oracle (not a sample)."""
     check(M, N, K, kind="outliers", seed=M + K)
+
+
+@pytest.mark.parametrize("M,N,K", [
+    (300, 200, 2560),      # 2 pair tiles, 4 pairs per tile (40 k-blocks: 10 each)
+    (260, 130, 1088),      # 4 pairs per tile over 17 k-blocks (4, 4, 4, 5), ragged M and N
+    (768, 2048, 512),      # 24 pair tiles, 2 pairs per tile (8 k-blocks: 4 each)
+    (700, 2000, 640),      # 24 pair tiles, 2 pairs per tile, ragged M and N
+])
+def test_split_k_clusters_full_output(M, N, K):
+    """Pair tiles whose K range is split over 2 or 4 CTA pairs of one cluster, the partial
+    tiles summed through distributed shared memory: every output element."""
+    check(M, N, K, kind="outliers", seed=M + N + K)
+
+
+def test_split_k_clusters_repeatable():
+    """The split partials are summed in a fixed order: two runs agree bit for bit."""
+    W = synth_inputs.weights("normal", 512, 2560, seed=5)
+    packed, scales, _ = oracle.quantize(W)
+    x = synth_inputs.activations(512, 2560, "bf16", seed=6)
+    assert np.array_equal(run_gemm(x, packed, scales), run_gemm(x, packed, scales))
 
 
 def test_zero_weights_give_zero():

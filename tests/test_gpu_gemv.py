@@ -7,7 +7,7 @@ import torch
 
 import oracle
 import synth_inputs
-from tests._parity import digit_path_bound, f32_sum_bound, offset_path_bound, rel_inf, to_dev_x
+from tests._parity import digit_path_bound, f32_sum_bound, mma_path_bound, rel_inf, to_dev_x
 
 pytestmark = pytest.mark.gpu
 
@@ -39,14 +39,14 @@ def check(x, W, x_dtype, tight=True):
     if tight:
         # the bound of the path the shape takes: M = 1 with K % 256 == 0 runs on exact
         # integer digit planes of x, M >= 2 with bf16 x and K % 256 == 0 on the bf16
-        # tensor cores with an offset, every other shape on CUDA-core FMAs (the fallback)
+        # tensor cores (exact products, f32 sums), every other shape on CUDA-core FMAs
         n, deq = roundings(W.shape[1]), oracle.dequantize(packed, scales)
         if W.shape[1] % 256 == 0 and x.shape[0] == 1:
             bound = digit_path_bound(x, deq, n)
+        elif W.shape[1] % 256 == 0 and x_dtype == "bf16":
+            bound = mma_path_bound(x, deq, n)
         else:
             bound = f32_sum_bound(x, deq, n)
-            if x_dtype == "bf16":
-                bound = np.maximum(bound, offset_path_bound(x, scales, n))
         assert np.all(np.abs(y - ref) <= bound + 1e-30)
     return y, ref
 
