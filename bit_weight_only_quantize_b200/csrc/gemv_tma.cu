@@ -310,7 +310,8 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
     unsigned char* scl = codes + W * kStages * kStageCodes;               // [warp][stage][16 rows][8 * boxes]
     uint64_t* bars = reinterpret_cast<uint64_t*>(scl + W * kStages * kStageScales);   // [warp][stage]
     float* red = reinterpret_cast<float*>(bars + W * kStages);            // [warp][16 rows][MP]
-    unsigned char* xst = reinterpret_cast<unsigned char*>(red + W * kRows * MP);   // staged x (16-byte aligned)
+    unsigned char* xst = reinterpret_cast<unsigned char*>(                 // staged x, 16-byte aligned
+        (reinterpret_cast<uintptr_t>(red + W * kRows * MP) + 15) & ~uintptr_t(15));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int P = a.P;
@@ -749,7 +750,10 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
             }
         }
         team_sync(team, P);
-        if (wt == 0) {
+        // Plain stores without split-K: every warp of the team stores a share of the
+        // block's (x row, row) outputs; otherwise the team's first warp does the epilogue.
+        const bool share = EPI == kEpiPlain && a.splits == 1;
+        if (wt == 0 || share) {
             const int mi = matrix_of(a, rb);
             const int nrow = a.N[mi];
             const int lrow0 = (rb - a.rb_begin[mi]) * kRows;
@@ -810,7 +814,7 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
                     }
                 }
             } else {
-                for (int e0 = 0; e0 < (kFuse ? 0 : kRows * a.M); e0 += 32) {
+                for (int e0 = share ? wt * 32 : 0; e0 < (kFuse ? 0 : kRows * a.M); e0 += share ? P * 32 : 32) {
                     unsigned long long key = rows_out(e0);
                     if constexpr (kArgmax && MODE == kImma1) {
                         am_best = key_max(am_best, key);
@@ -993,7 +997,7 @@ size_t x_stage_bytes(int mode, int nb, int64_t M, bool int8 = false)
 
 size_t smem_bytes(int mode, int warps, int nb, int64_t M, bool int8 = false)
 {
-    return 1024 + (size_t)warps * per_warp_bytes(mode) + x_stage_bytes(mode, nb, M, int8);
+    return 1024 + 16 + (size_t)warps * per_warp_bytes(mode) + x_stage_bytes(mode, nb, M, int8);
 }
 
 int mode_for(int64_t M, q4_dtype xt)
@@ -1061,7 +1065,7 @@ bool plan_gemv_tma(int64_t M, const int64_t* Ns, int count, int64_t K, q4_dtype 
     };
     // Splits forced by shared memory: the staged x of one split leaves room for 4 warps.
     int splits_min = 1;
-    while (1024 + 4 * pw + x_stage_bytes(mode, split_boxes(splits_min), M, int8) > budget) {
+    while (1040 + 4 * pw + x_stage_bytes(mode, split_boxes(splits_min), M, int8) > budget) {
         if (split_boxes(splits_min) <= kBoxesPerStage) return false;
         ++splits_min;
     }
@@ -1077,8 +1081,8 @@ bool plan_gemv_tma(int64_t M, const int64_t* Ns, int count, int64_t K, q4_dtype 
         const int nbs = split_boxes(sp);
         if ((boxes + nbs - 1) / nbs != sp) continue;                  // same cut as fewer splits
         const size_t xs = x_stage_bytes(mode, nbs, M, int8);
-        if (1024 + pw + xs > budget) continue;
-        const size_t fitw = (budget - 1024 - xs) / pw;
+        if (1040 + pw + xs > budget) continue;
+        const size_t fitw = (budget - 1040 - xs) / pw;
         const int wbs = (int)(fitw < (size_t)kMaxWarps ? fitw : (size_t)kMaxWarps);
         const int nus = (nbs + kBoxesPerStage - 1) / kBoxesPerStage;
         const long long sms = dev.sm_count / sp > 0 ? dev.sm_count / sp : 1;   // blocks of one split
