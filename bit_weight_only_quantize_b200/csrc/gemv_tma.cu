@@ -27,12 +27,12 @@
 //          makes the int32 result the bit pattern of the exact float 1.5 * 2^23 + sum.
 //          Each group's sum is multiplied by its scale, the box's sums by 2^-F, and
 //          accumulated in f32 per plane; the planes are combined at the end.
-//      M = 2..16 (bf16 x): nibble pair (j, j+4) of a word OR-ed into 0x4300 (one LOP3)
-//          is the bf16 pair (128 + c_j, 128 + c_{j+4}); one exact bf16x2 subtraction of
-//          136 makes it (c_j - 8, c_{j+4} - 8).  Such pairs, read with ldmatrix, are the
-//          A operand of mma.sync.m16n8k16 and x rows the B operand, in a permuted k order
-//          that matches the pairs; every product is exact and the group's sum is
-//          accumulated in f32 from zero.
+//      M = 2..16 (bf16 x): byte j of a code word (codes 2j, 2j+1) placed by one PRMT
+//          and OR-ed into 0x4300 (one LOP3) is the bf16 pair (128 + c_2j, 128 + c_2j+1);
+//          one exact bf16x2 subtraction of 136 makes it (c_2j - 8, c_2j+1 - 8).  Such
+//          pairs, read with ldmatrix, are the A operand of mma.sync.m16n8k16 and x rows,
+//          as they arrive, the B operand (both in k order); every product is exact and
+//          the group's sum is accumulated in f32 from zero.
 //    In every mode each group's sum is scaled by its binary16 scale and added in f32.
 //  * Every mbarrier wait is bounded.  If one runs out the kernel records
 //    kErrWaitTimeout in the library error word, stops issuing and computing, waits
@@ -144,9 +144,12 @@ __device__ __forceinline__ uint32_t pinned_u32(uint32_t v)
 
 // Nibble pair (j, j+4) of a word as the bf16 pair (128 + c_j, 128 + c_{j+4}); mask and
 // magic are the registers holding 0x000F000F and 0x43004300.
-__device__ __forceinline__ uint32_t nib_pair(uint32_t v, int j, uint32_t mask, uint32_t magic)
+// Byte j of a code word as the bf16 pair (128 + low nibble, 128 + high nibble): codes
+// 2j and 2j + 1 of the word in k order.  v4 = v >> 4 puts each high nibble where PRMT
+// can take it (byte j of v into the low half, byte j of v4 into the high half).
+__device__ __forceinline__ uint32_t byte_pair(uint32_t v, uint32_t v4, int j, uint32_t mask, uint32_t magic)
 {
-    return and_or(v >> (4 * j), mask, magic);
+    return and_or(__byte_perm(v, v4, (uint32_t)(j | ((4 + j) << 8))), mask, magic);
 }
 
 // (128 + c) - 136 = c - 8 for both bf16 halves; exact (small integers).
@@ -220,13 +223,6 @@ __device__ __forceinline__ float scale_at(const uint4& s8, int c)
 {
     const uint32_t sw = c < 2 ? s8.x : c < 4 ? s8.y : c < 6 ? s8.z : s8.w;
     return __half2float(__ushort_as_half((unsigned short)((c & 1) ? (sw >> 16) : (sw & 0xFFFFu))));
-}
-
-__device__ __forceinline__ uint4 pairs_of(const uint4 raw)
-{
-    // raw holds x_0..x_7 as (x0,x1)(x2,x3)(x4,x5)(x6,x7); regroup to (x_j, x_{j+4}).
-    return make_uint4(__byte_perm(raw.x, raw.z, 0x5410), __byte_perm(raw.x, raw.z, 0x7632),
-                      __byte_perm(raw.y, raw.w, 0x5410), __byte_perm(raw.y, raw.w, 0x7632));
 }
 
 // Eight x values (k = 8t .. 8t+7 of a group) as balanced base-256 digit planes of
@@ -404,9 +400,9 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
         for (int j = 0; j < issued; ++j) issue(j);
 
     // ---- stage x for this split (zero past the split and past K) ----
-    //  kMma* : bf16 pairs [m][group][word][4] for m < M, then one zero row that lanes
-    //          of x rows >= M read; each row is padded by one group so that lanes of
-    //          neighbouring x rows fall on different banks.
+    //  kMma* : x rows [m][group][32 bf16] in k order for m < M, then one zero row that
+    //          lanes of x rows >= M read; each row is padded by one group so that lanes
+    //          of neighbouring x rows fall on different banks.
     //  kImma1: each box of 8 groups (256 x values) is scaled by 2^F (the largest F with
     //          max |x| of the box * 2^F < 2^30, at most 100), rounded to integers X and
     //          cut into four balanced base-256 digits X = d0 2^24 + d1 2^16 + d2 2^8 + d3,
@@ -501,8 +497,9 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
         }
     } else {
         uint4* xp = reinterpret_cast<uint4*>(xst);
-        // The split's part of each x row arrives by one bulk copy, straight where its
-        // staged words go (all rows in flight at once), and is then permuted in place.
+        // The split's part of each x row arrives by one bulk copy, in k order, where the
+        // MMAs read it (all rows in flight at once); the groups past the split's end
+        // and the zero row are cleared meanwhile.
         if (threadIdx.x == 0) {
             mbar_init(&s_xbar, 1);
             fence_mbar_init();
@@ -511,16 +508,14 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
                 bulk_load(xp + m * rs, reinterpret_cast<const uint16_t*>(a.x) + (size_t)m * K + (size_t)g0 * 32,
                           (uint32_t)(ng * 64), &s_xbar);
         }
+        const int tail = (ngp - ng) * 4;                                  // uint4 past the split per row
+        for (int i = threadIdx.x; i < a.M * tail + ngp * 4; i += blockDim.x) {
+            const int m = i < a.M * tail ? i / tail : a.M;
+            const int w = i < a.M * tail ? ng * 4 + (i - m * tail) : i - a.M * tail;
+            xp[m * rs + w] = make_uint4(0u, 0u, 0u, 0u);
+        }
         __syncthreads();
         x_ok = mbar_wait_bounded(&s_xbar, 0, kWaitLimit);
-        const int total = (a.M + 1) * ngp * 4;
-        for (int i = threadIdx.x; i < total; i += blockDim.x) {
-            const int m = i / (ngp * 4);
-            const int rem = i - m * ngp * 4;
-            uint4 raw = make_uint4(0u, 0u, 0u, 0u);
-            if (m < a.M && (rem >> 2) < ng && x_ok) raw = xp[m * rs + rem];
-            xp[m * rs + rem] = pairs_of(raw);
-        }
     }
     __syncthreads();
 
@@ -682,14 +677,17 @@ gemv_tma_kernel(const __grid_constant__ TmaMaps maps, const TmaGemvArgs a)
                                     for (int h = 0; h < 2; ++h) {
                                         const int c = 2 * cp + h;
                                         const uint32_t w0 = h ? r2 : r0, w1 = h ? r3 : r1;
-                                        const uint32_t A0 = sub_bf16x2(nib_pair(w0, 0, kmask, kmagic), k136);
-                                        const uint32_t A1 = sub_bf16x2(nib_pair(w1, 0, kmask, kmagic), k136);
-                                        const uint32_t A2 = sub_bf16x2(nib_pair(w0, 1, kmask, kmagic), k136);
-                                        const uint32_t A3 = sub_bf16x2(nib_pair(w1, 1, kmask, kmagic), k136);
-                                        const uint32_t A4 = sub_bf16x2(nib_pair(w0, 2, kmask, kmagic), k136);
-                                        const uint32_t A5 = sub_bf16x2(nib_pair(w1, 2, kmask, kmagic), k136);
-                                        const uint32_t A6 = sub_bf16x2(nib_pair(w0, 3, kmask, kmagic), k136);
-                                        const uint32_t A7 = sub_bf16x2(nib_pair(w1, 3, kmask, kmagic), k136);
+                                        // codes 8t .. 8t+7 of rows g, g+8 in k order: MMA 1 takes
+                                        // bytes 0, 1 (k 8t .. 8t+3), MMA 2 bytes 2, 3
+                                        const uint32_t v0 = w0 >> 4, v1 = w1 >> 4;
+                                        const uint32_t A0 = sub_bf16x2(byte_pair(w0, v0, 0, kmask, kmagic), k136);
+                                        const uint32_t A1 = sub_bf16x2(byte_pair(w1, v1, 0, kmask, kmagic), k136);
+                                        const uint32_t A2 = sub_bf16x2(byte_pair(w0, v0, 1, kmask, kmagic), k136);
+                                        const uint32_t A3 = sub_bf16x2(byte_pair(w1, v1, 1, kmask, kmagic), k136);
+                                        const uint32_t A4 = sub_bf16x2(byte_pair(w0, v0, 2, kmask, kmagic), k136);
+                                        const uint32_t A5 = sub_bf16x2(byte_pair(w1, v1, 2, kmask, kmagic), k136);
+                                        const uint32_t A6 = sub_bf16x2(byte_pair(w0, v0, 3, kmask, kmagic), k136);
+                                        const uint32_t A7 = sub_bf16x2(byte_pair(w1, v1, 3, kmask, kmagic), k136);
 #pragma unroll
                                         for (int n = 0; n < NT; ++n) {
                                             const uint4 bx = xrow[n][(gb + c) * 4 + t];
