@@ -63,6 +63,7 @@ constexpr int kCounterSlots = 1024;          // same workspace layout as the gen
 constexpr double kMinWarpShare = 12.0;
 constexpr double kEpilogueCost = 0.1;
 constexpr double kSplitCost = 0.9;
+constexpr int kStagingWarps = 8;              // fewest warps per block (extra ones only stage x)
 constexpr size_t kCounterBytes = kCounterSlots * sizeof(unsigned);
 
 // kImma1: one x row on the integer tensor cores; kMma8 / kMma16: 2..8 / 9..16 bf16 x rows.
@@ -1108,7 +1109,13 @@ bool plan_gemv_tma(int64_t M, const int64_t* Ns, int count, int64_t K, q4_dtype 
     if (splits == 0) return false;
     const int ksg = split_boxes(splits) * 8;
     const int nb = ksg / 8;
-    const int warps = P * teams;
+    // A block with few warps stages x slowly (every block stages its split in full), so
+    // small plans get warps that own no rows and only help with the staging.
+    int warps = P * teams;
+    if (warps < kStagingWarps) {
+        const size_t sw = smem_bytes(mode, kStagingWarps, nb, M, int8);
+        if (sw <= budget && blocks_per_sm(kernel_for(mode, epi), kStagingWarps * 32, sw) >= 1) warps = kStagingWarps;
+    }
     const size_t smem = smem_bytes(mode, warps, nb, M, int8);
     if (smem > budget) return false;
     const int per_sm = blocks_per_sm(kernel_for(mode, epi), warps * 32, smem);
@@ -1128,6 +1135,7 @@ bool plan_gemv_tma(int64_t M, const int64_t* Ns, int count, int64_t K, q4_dtype 
     p->workspace_bytes =
         splits > 1 ? kCounterBytes + (size_t)splits * (size_t)M * (size_t)row_blocks * kRows * sizeof(float) : 0;
     p->has_int8 = int8 ? 1 : 0;
+    p->block_warps = warps;
     return true;
 }
 
@@ -1196,7 +1204,7 @@ q4_status launch_gemv_tma(const void* x, q4_dtype xt, int64_t M, int64_t K, cons
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)plan.grid_x, (unsigned)plan.splits);
-    cfg.blockDim = dim3((unsigned)(a.P * a.teams * 32));
+    cfg.blockDim = dim3((unsigned)(plan.block_warps * 32));
     cfg.dynamicSmemBytes = (size_t)plan.smem_bytes;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];

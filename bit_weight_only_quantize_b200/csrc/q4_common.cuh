@@ -39,6 +39,7 @@ struct GemvPlan {
     int smem_bytes;         // dynamic shared memory per block
     size_t workspace_bytes; // partial sums + counters (0 when splits == 1)
     int has_int8;           // TMA kernel: some matrix holds INT8 codes
+    int block_warps;        // TMA kernel: warps per block (>= chunk * xcap; the rest only stage x)
 };
 
 // Chooses the kernels for one or more weight matrices sharing x (all N > 0).
