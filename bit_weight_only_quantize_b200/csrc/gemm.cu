@@ -86,22 +86,15 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar)
 }
 
 // 32 consecutive f32 columns of this warp's 32 accumulator lanes.
-// 32 consecutive f32 columns of this warp's 32 tensor-memory lanes, without waiting
-// (tmem_wait_ld makes them usable).
-__device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, uint32_t (&r)[32])
+// 16 consecutive f32 columns of this warp's 32 tensor-memory lanes.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16])
 {
     asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
         : "r"(taddr)
         : "memory");
-}
-__device__ __forceinline__ void tmem_wait_ld()
-{
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
@@ -516,16 +509,45 @@ __device__ __forceinline__ void mma_commit_pair(uint64_t* bar, uint16_t mask)
         : "memory");
 }
 
-// Four floats from the shared memory of a CTA of this cluster (address from peer_addr).
-// No memory clobber: the loads read data fixed by an earlier cluster barrier, so several
-// may be in flight at once.
-__device__ __forceinline__ float4 ld_cluster_f4(uint32_t cluster_addr)
+// Bulk copy of `bytes` from this CTA's shared memory into another CTA's of this cluster
+// (cluster addresses from peer_addr); completion counts on the destination's mbarrier.
+__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, const void* src, uint32_t bytes,
+                                                  uint32_t bar_cluster)
 {
-    float4 v;
-    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                 : "r"(cluster_addr));
-    return v;
+    asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     dst_cluster),
+                 "r"(smem_addr(src)), "r"(bytes), "r"(bar_cluster)
+                 : "memory");
+}
+
+
+// Arrive on an mbarrier of a CTA of this cluster, releasing this thread's earlier writes
+// (to any CTA's shared memory) at cluster scope.
+__device__ __forceinline__ void mbar_arrive_release_cluster(uint32_t cluster_addr)
+{
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// Bounded wait on one of this CTA's mbarriers that acquires, at cluster scope, the writes
+// the arriving threads of other CTAs released.
+__device__ __forceinline__ bool mbar_wait_acquire_cluster_bounded(uint64_t* bar, uint32_t parity, uint64_t limit_ns)
+{
+    auto try_wait = [&]() {
+        uint32_t ok;
+        asm volatile(
+            "{\n .reg .pred p;\n mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
+            " selp.u32 %0, 1, 0, p;\n}"
+            : "=r"(ok)
+            : "r"(smem_addr(bar)), "r"(parity)
+            : "memory");
+        return ok != 0;
+    };
+    if (try_wait()) return true;
+    const uint64_t t0 = global_ns();
+    while (true) {
+        if (try_wait()) return true;
+        if (global_ns() - t0 > limit_ns) return false;
+    }
 }
 
 template <int BNP>
@@ -544,11 +566,12 @@ struct PairCfg {
     static_assert(kStageBytes % 1024 == 0, "stage alignment");
 };
 
-// SPL > 1: a cluster of SPL pairs computes one pair tile, pair j over the j-th of SPL
-// consecutive k ranges; after its last MMA each CTA stages its f32 partial tile in its
-// own stage ring (idle by then), and each CTA sums the SPL partials of its 128 rows over
-// 1/SPL of the columns through distributed shared memory, in pair order, and stores them
-// as bf16.  One tile per cluster: the launch has one cluster per tile.
+// SPL == 2: a cluster of two pairs computes one pair tile, pair j over the j-th half of the
+// k range, and owns columns [j, j + 1) * BNP / 2 of the tile.  After its last MMA each CTA
+// stages the other pair's column slice of its f32 partial tile in its own (then idle) stage
+// ring and, once the other pair announces that its ring is idle too, sends it there with one
+// bulk copy (same half of the pair); it then sums its own slice over both partials, in pair
+// order, and stores it as bf16.  One tile per cluster: the launch has one cluster per tile.
 template <int BNP, int SPL>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_codes,
@@ -569,7 +592,10 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
     uint64_t* accfull = bars + 3 * S;    // MMA -> epilogues of both CTAs, 2 buffers
     uint64_t* accempty = accfull + 2;    // epilogues of both CTAs -> MMA (CTA 0's copy)
     uint64_t* drain = accempty + 2;      // final commit on abort
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    uint64_t* ring_free = drain + 1;     // SPL == 2: the other pair's ring is idle (4 arrivals)
+    uint64_t* recv_full = ring_free + 1; // SPL == 2: the other pair's slice has arrived (bulk copy bytes)
+    uint64_t* staged = recv_full + 1;    // SPL == 2: the four epilogue warps staged their rows (4)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(staged + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -581,9 +607,15 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
     const int kb0 = ks * a.kblocks / SPL, kb1 = (ks + 1) * a.kblocks / SPL;
     const int cluster = blockIdx.x / (2 * SPL), nclusters = gridDim.x / (2 * SPL);
     const int tiles = a.tiles_m * a.tiles_n;
-    float* stg = reinterpret_cast<float*>(smem);         // SPL > 1: staged partial tile, [128][kStgStride]
-    constexpr int kStgStride = BNP + 4;                  // floats per staged row (spreads the banks)
-    static_assert(SPL == 1 || 128 * kStgStride * 4 <= S * C::kStageBytes, "staging fits the ring");
+    // SPL == 2, in the idle ring: the slice the other pair sends [128 rows][kRS], then the
+    // slice this CTA sends it, staged the same way
+    static_assert(SPL == 1 || SPL == 2, "K splits over one or two pairs");
+    constexpr int kCols = BNP / SPL;                     // columns a pair owns
+    constexpr int kRS = kCols + 4;                       // floats per staged row (spreads the banks)
+    constexpr uint32_t kSliceBytes = 128u * kRS * 4u;
+    float* rcv = reinterpret_cast<float*>(smem);
+    float* snd = rcv + 128 * kRS;
+    static_assert(SPL == 1 || 2 * kSliceBytes <= S * C::kStageBytes, "both slices fit the ring");
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
@@ -596,6 +628,9 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
             mbar_init(&accempty[b], 8);
         }
         mbar_init(drain, 1);
+        mbar_init(ring_free, 4);
+        mbar_init(recv_full, 1);
+        mbar_init(staged, 4);
         *abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tm_x);
@@ -697,22 +732,78 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
             const int row = (t % a.tiles_m) * 256 + (int)rank * 128 + quad * 32 + lane;
             const int n0 = (t / a.tiles_m) * BNP;
             if constexpr (SPL > 1) {
-                // stage the f32 partial tile (64 columns per tensor-memory wait); the
-                // reduction after the role loops stores y
+                // This pair's MMAs are done, so its ring is idle: tell the other pair (same
+                // half), stage its slice here, and send it once its ring is idle too.
+                const int lrow = quad * 32 + lane;             // this thread's row of the CTA's 128
+                const int jd = 1 - ks;                          // the other pair
+                const uint32_t peer = 2u * (uint32_t)jd + rank;
+                if (lane == 0) mbar_arrive_release_cluster(peer_addr(ring_free, peer));
+                if (quad == 0 && lane == 0) mbar_arrive_expect_tx(recv_full, kSliceBytes);
 #pragma unroll 1
-                for (int c0 = 0; c0 < BNP; c0 += 64) {
-                    uint32_t r0[32], r1[32];
-                    const uint32_t ta = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(buf * BNP + c0);
-                    tmem_ld32_nowait(ta, r0);
-                    tmem_ld32_nowait(ta + 32, r1);
-                    tmem_wait_ld();
-                    float4* dst = reinterpret_cast<float4*>(stg + (quad * 32 + lane) * kStgStride + c0);
+                for (int c0 = 0; c0 < kCols; c0 += 32) {
+                    uint32_t r[32];
+                    tmem_ld32(tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(buf * BNP + jd * kCols + c0), r);
+                    float4* d = reinterpret_cast<float4*>(snd + lrow * kRS + c0);
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        dst[q] = make_float4(__uint_as_float(r0[4 * q]), __uint_as_float(r0[4 * q + 1]),
-                                             __uint_as_float(r0[4 * q + 2]), __uint_as_float(r0[4 * q + 3]));
-                        dst[8 + q] = make_float4(__uint_as_float(r1[4 * q]), __uint_as_float(r1[4 * q + 1]),
-                                                 __uint_as_float(r1[4 * q + 2]), __uint_as_float(r1[4 * q + 3]));
+                    for (int q = 0; q < 8; ++q)
+                        d[q] = make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
+                                           __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]));
+                }
+                fence_proxy_async_smem();                       // staged writes -> the bulk copy's reads
+                __syncwarp();
+                if (lane == 0) mbar_arrive(staged);
+                if (quad == 0 && lane == 0) {
+                    bool go = mbar_wait_bounded(staged, 0, kWaitLimit);
+                    go = go && mbar_wait_acquire_cluster_bounded(ring_free, 0, kWaitLimit);
+                    if (go) bulk_copy_to_peer(peer_addr(rcv, peer), snd, kSliceBytes, peer_addr(recv_full, peer));
+                    else fail();
+                }
+                if (!mbar_wait_bounded(recv_full, 0, kWaitLimit)) fail();
+                // own slice: the partials in pair order (this pair's from tensor memory)
+                const int col0 = n0 + ks * kCols;
+                const bool vec_own = (a.N % 8) == 0 && (reinterpret_cast<uintptr_t>(a.y) & 15) == 0;
+#pragma unroll 1
+                for (int c0 = 0; c0 < kCols; c0 += 16) {
+                    uint32_t r[16];
+                    tmem_ld16(tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(buf * BNP + ks * kCols + c0), r);
+                    float v[16];
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) v[q] = 0.f;
+#pragma unroll
+                    for (int js = 0; js < SPL; ++js) {
+                        if (js == ks) {
+#pragma unroll
+                            for (int q = 0; q < 16; ++q) v[q] += __uint_as_float(r[q]);
+                        } else {
+                            const float4* src = reinterpret_cast<const float4*>(rcv + lrow * kRS + c0);
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) {
+                                const float4 w = src[q];
+                                v[4 * q] += w.x;
+                                v[4 * q + 1] += w.y;
+                                v[4 * q + 2] += w.z;
+                                v[4 * q + 3] += w.w;
+                            }
+                        }
+                    }
+                    const int col = col0 + c0;
+                    if (row < a.M) {
+                        uint16_t* dst = a.y + (size_t)row * a.N + col;
+                        if (vec_own && col + 16 <= a.N) {
+#pragma unroll
+                            for (int q = 0; q < 2; ++q) {
+                                uint4 o;
+                                o.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
+                                o.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
+                                o.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
+                                o.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
+                                *reinterpret_cast<uint4*>(dst + 8 * q) = o;
+                            }
+                        } else {
+#pragma unroll
+                            for (int q = 0; q < 16; ++q)
+                                if (col + q < a.N) dst[q] = (uint16_t)(pack_bf16x2(v[q], 0.f) & 0xFFFFu);
+                        }
                     }
                 }
             }
@@ -799,61 +890,6 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
     tc_fence_before();
     __syncthreads();
     cluster_sync_all();                  // no CTA leaves while the pair's MMAs may read its shared memory
-    if constexpr (SPL > 1) {
-        // Every CTA's partial tile is staged (the cluster barrier orders the writes).  This
-        // CTA stores columns [ks, ks + 1) * BNP / SPL of its 128 rows: the sum of the SPL
-        // pairs' partials of the same half, in pair order.
-        const int t = cluster;
-        if (t < tiles) {
-            constexpr int kCols = BNP / SPL;
-            const int row0 = (t % a.tiles_m) * 256 + (int)rank * 128;
-            const int col0 = (t / a.tiles_m) * BNP + ks * kCols;
-            uint32_t src[SPL];
-#pragma unroll
-            for (int j = 0; j < SPL; ++j) src[j] = peer_addr(stg, 2u * (uint32_t)j + rank);
-            const bool vec_ok = (a.N % 4) == 0 && (reinterpret_cast<uintptr_t>(a.y) & 7) == 0;
-            // kBatch float4 of every partial in flight per thread before the sums
-            constexpr int kQuads = 128 * (kCols / 4), kBatch = 4;
-            for (int e0 = threadIdx.x; e0 < kQuads; e0 += kBatch * (int)blockDim.x) {
-                float4 v[kBatch][SPL];
-#pragma unroll
-                for (int b = 0; b < kBatch; ++b) {
-                    const int e = min(e0 + b * (int)blockDim.x, kQuads - 1);
-                    const int rr = e / (kCols / 4), cc = (e - rr * (kCols / 4)) * 4;
-                    const uint32_t off = (uint32_t)((rr * kStgStride + ks * kCols + cc) * 4);
-#pragma unroll
-                    for (int j = 0; j < SPL; ++j) v[b][j] = ld_cluster_f4(src[j] + off);
-                }
-#pragma unroll
-                for (int b = 0; b < kBatch; ++b) {
-                    const int e = e0 + b * (int)blockDim.x;
-                    if (e >= kQuads) break;
-                    float4 acc = v[b][0];
-#pragma unroll
-                    for (int j = 1; j < SPL; ++j) {
-                        acc.x += v[b][j].x;
-                        acc.y += v[b][j].y;
-                        acc.z += v[b][j].z;
-                        acc.w += v[b][j].w;
-                    }
-                    const int rr = e / (kCols / 4), cc = (e - rr * (kCols / 4)) * 4;
-                    const int row = row0 + rr, col = col0 + cc;
-                    if (row < a.M && col < a.N) {
-                        uint16_t* dst = a.y + (size_t)row * a.N + col;
-                        if (vec_ok && col + 4 <= a.N) {
-                            *reinterpret_cast<uint2*>(dst) =
-                                make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
-                        } else {
-                            const float f[4] = {acc.x, acc.y, acc.z, acc.w};
-                            for (int q = 0; q < 4 && col + q < a.N; ++q)
-                                dst[q] = (uint16_t)(pack_bf16x2(f[q], 0.f) & 0xFFFFu);
-                        }
-                    }
-                }
-            }
-        }
-        cluster_sync_all();              // no CTA leaves while the others read its staged tile
-    }
     tc_fence_after();
     if (warp == kMmaWarp) tmem_dealloc2(tmem_base, C::kTmemCols);
 }
@@ -985,16 +1021,14 @@ q4_status launch_gemm(const uint16_t* x, int64_t M, int64_t K, const uint8_t* pa
 {
     // CTA pairs (256-row tiles) from M = 256 on.  A pair's k-block takes about the same
     // time with 128 output columns as with 256 (measured on B200: 0.45-0.5 us against
-    // 0.55-0.6 us), so 256 x 256 tiles are used throughout; when they leave SM pairs idle,
-    // 4 or 2 pairs share each tile's K range (clusters of 8 or 4 CTAs, each pair at least
-    // 4 k-blocks) as long as every cluster can be resident at once; else 256 x 128 tiles
-    // when 256 x 256 ones would occupy fewer than half of the pairs.
+    // 0.55-0.6 us), so 256 x 256 tiles are used throughout; when they leave at least half
+    // of the SM pairs idle, two pairs share each tile's K range (clusters of 4 CTAs, each
+    // pair at least 4 k-blocks) as long as every cluster can be resident at once; else
+    // 256 x 128 tiles when 256 x 256 ones would occupy fewer than half of the pairs.
     if (M >= 256 && dev.sm_count >= 2) {
         const long long p256 = ((M + 255) / 256) * ((N + 255) / 256);
         const long long pairs = dev.sm_count / 2;
         const long long kblocks = (K + kBK - 1) / kBK;
-        if (p256 * 4 <= pairs && kblocks >= 16 && pair_cluster_capacity<256, 4>(dev) >= p256)
-            return launch_gemm_pair<256, 4>(x, M, K, packed, scales, N, y, stream, dev);
         if (p256 * 2 <= pairs && kblocks >= 8 && pair_cluster_capacity<256, 2>(dev) >= p256)
             return launch_gemm_pair<256, 2>(x, M, K, packed, scales, N, y, stream, dev);
         if (2 * p256 >= pairs) return launch_gemm_pair<256, 1>(x, M, K, packed, scales, N, y, stream, dev);

@@ -392,7 +392,7 @@ Q4_API q4_status q4_f16_gemv(const void* x, q4_dtype x_dtype, int64_t M, int64_t
  * Arithmetic: each weight becomes bf16_rn((code - 8) * f32(scale)) (one rounding of an
  * exact product), products run on the tensor cores (tcgen05) with f32 accumulation,
  * and each f32 output is rounded to nearest-even bfloat16.  At small M the K range of a
- * tile may be split over 2 or 4 CTA pairs of one cluster, whose f32 partial tiles are
+ * tile may be split over the 2 CTA pairs of one cluster, whose f32 partial tiles are
  * summed in a fixed order before the rounding (results are repeatable bit for bit).
  * M == 0 or N == 0 is a no-op.  No workspace.
  */

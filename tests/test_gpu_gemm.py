@@ -78,14 +78,14 @@ def test_large_tiles_full_output(M, N, K):
 
 
 @pytest.mark.parametrize("M,N,K", [
-    (300, 200, 2560),      # 2 pair tiles, 4 pairs per tile (40 k-blocks: 10 each)
-    (260, 130, 1088),      # 4 pairs per tile over 17 k-blocks (4, 4, 4, 5), ragged M and N
+    (300, 200, 2560),      # 2 pair tiles, 2 pairs per tile (40 k-blocks: 20 each)
+    (260, 130, 1088),      # 2 pairs per tile over 17 k-blocks (8, 9), ragged M and N
     (768, 2048, 512),      # 24 pair tiles, 2 pairs per tile (8 k-blocks: 4 each)
     (700, 2000, 640),      # 24 pair tiles, 2 pairs per tile, ragged M and N
 ])
 def test_split_k_clusters_full_output(M, N, K):
-    """Pair tiles whose K range is split over 2 or 4 CTA pairs of one cluster, the partial
-    tiles summed through distributed shared memory: every output element."""
+    """Pair tiles whose K range is split over the 2 CTA pairs of one cluster, the partial
+    slices exchanged through distributed shared memory: every output element."""
     check(M, N, K, kind="outliers", seed=M + N + K)
 
 
