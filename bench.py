@@ -194,10 +194,11 @@ def capture(torch, launch, n, stream):
 
 def timed_replays(torch, graph, stream, device, dist=None, clocks=None, min_replays=MIN_REPLAYS,
                   min_ms=MIN_TIMED_MS):
-    """Replay `graph` (untimed first: once, then as many times as it will be timed, so that
-    clocks and power settle), each timed replay bracketed by CUDA events on `stream`, a
-    device synchronisation and, under torchrun, a barrier; returns the list of per-replay
-    milliseconds."""
+    """Replay `graph` (one untimed replay first), each timed replay bracketed by CUDA
+    events on `stream`, a device synchronisation and, under torchrun, a barrier; returns
+    the list of per-replay milliseconds.  The timed replays follow the warm-up directly,
+    so the figure is the burst regime of a kernel timed alone (a load held for longer
+    brings in the power cap and lower SM clocks)."""
     with torch.cuda.stream(stream):
         graph.replay()
     torch.cuda.synchronize(device)
@@ -212,10 +213,6 @@ def timed_replays(torch, graph, stream, device, dist=None, clocks=None, min_repl
         t = torch.tensor([reps], dtype=torch.int64, device=device)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         reps = int(t.item())
-    for _ in range(reps):                             # untimed: clocks and power settle at this load
-        with torch.cuda.stream(stream):
-            graph.replay()
-    torch.cuda.synchronize(device)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
     if clocks is not None:
         clocks.start()
