@@ -758,7 +758,10 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
                     if (go) bulk_copy_to_peer(peer_addr(rcv, peer), snd, kSliceBytes, peer_addr(recv_full, peer));
                     else fail();
                 }
-                if (!mbar_wait_bounded(recv_full, 0, kWaitLimit)) fail();
+                // The other pair issues its copy only after two bounded waits of its own, so
+                // this wait is bounded by three limits: no copy into this CTA can still be
+                // under way when it gives up.
+                if (!mbar_wait_bounded(recv_full, 0, 3 * kWaitLimit)) fail();
                 // own slice: the partials in pair order (this pair's from tensor memory)
                 const int col0 = n0 + ks * kCols;
                 const bool vec_own = (a.N % 8) == 0 && (reinterpret_cast<uintptr_t>(a.y) & 15) == 0;
