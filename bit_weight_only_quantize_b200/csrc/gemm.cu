@@ -436,8 +436,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
 // shared-memory operand traffic and the dequantisation per flop of a single-CTA tile.
 // Both CTAs' dequantise warps arrive on CTA 0's "B ready" barrier and both CTAs'
 // epilogue warps on its "accumulator empty" barrier; MMA completion is committed to the
-// barriers of both CTAs (multicast commit).  No TMA load uses cluster multicast: each
-// CTA loads its own x and code tiles.
+// barriers of both CTAs by one commit addressed to the pair.  Every tensor copy is a plain
+// one: each CTA loads its own x and code tiles.
 
 __device__ __forceinline__ uint32_t cluster_rank()
 {
@@ -588,7 +588,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes);
     uint64_t* full = bars;               // producer -> dequant (own TMA bytes)
     uint64_t* bready = bars + S;         // dequant of both CTAs -> MMA (CTA 0's copy is used)
-    uint64_t* empty = bars + 2 * S;      // MMA -> producers of both CTAs (multicast commit)
+    uint64_t* empty = bars + 2 * S;      // MMA -> producers of both CTAs (one commit to the pair)
     uint64_t* accfull = bars + 3 * S;    // MMA -> epilogues of both CTAs, 2 buffers
     uint64_t* accempty = accfull + 2;    // epilogues of both CTAs -> MMA (CTA 0's copy)
     uint64_t* drain = accempty + 2;      // final commit on abort
