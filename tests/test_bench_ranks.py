@@ -1,6 +1,6 @@
 """Host logic of the multi-process benchmark on CPU: gloo ranks agree on the slowest
 rank's time, the whole-job figure counts every rank's bytes, and the reference arm runs
-on rank 0 only."""
+on rank 0 only and prints a line with the main arm's keys, metric and config."""
 import os
 import socket
 
@@ -51,3 +51,37 @@ def test_reference_arm_prints_on_rank_zero_only(capsys, monkeypatch):
     monkeypatch.setattr(bench, "cpu_baseline", lambda *a, **k: {"value": 1.0})
     bench.run_reference(Args(), 2, 1)
     assert capsys.readouterr().out == ""
+
+
+def test_reference_arm_line_keeps_the_contract(capsys, monkeypatch):
+    """On rank 0 the reference arm prints one JSON line with the keys of the main arm's line,
+    the same metric, unit and config, and an e2e / cpu_baseline that restate its own value
+    (a small head stands in for the LM head so the oracle finishes in well under a second)."""
+    import json
+
+    import synth_inputs
+
+    small = synth_inputs.Workload("gemv_2560x4096_small_head", "gemv", 1, 2560, 4096, "lm_head", "bf16")
+    monkeypatch.setattr(bench, "MAIN", small)
+
+    class Args:
+        steps, warmup, cpu_seconds = 2, 1, 0.01
+    bench.run_reference(Args(), 1, 0)
+    out = capsys.readouterr().out.strip().splitlines()
+    assert len(out) == 1
+    line = json.loads(out[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference"
+    assert (line["metric"], line["unit"], line["higher_is_better"]) == (bench.METRIC, bench.UNIT, True)
+    assert (line["n_gpus"], line["steps"], line["warmup"]) == (1, 2, 1)
+    assert line["config"] == dict(bench.CONFIG, bytes_per_step=bench.STEP_BYTES)   # the main arm's config
+    assert line["value"] > 0
+    # value is the bytes of the sampled rows per step over the time per step
+    assert line["value"] * line["ms_per_step"] * 1e6 == pytest.approx(bench.gemv_bytes(1, small.N, small.K))
+    assert line["e2e"] == {"value": line["value"], "unit": line["unit"], "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == line["value"] and cb["unit"] == line["unit"]
+    assert cb["cores"] >= 1 and str(small.N) in cb["sample"]
