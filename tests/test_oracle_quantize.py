@@ -4,8 +4,9 @@ Checked against: hand-derived encodings (tests/golden/quantize_cases.json),
 exact reconstruction of weights already on the integer grid, the per-element
 round-trip bound |w - w'| <= s/2, an independent binary64 characterisation of
 the code as the nearest integer in [-8, 7] (ties to even), the scale as the
-binary16 cast of f32(amax)/7 through numpy's own conversion, and the structural
-facts every encoded group must satisfy.
+binary16 cast of f32(amax)/7 through numpy's own conversion, the structural
+facts every encoded group must satisfy, and (hypothesis) the same scale and
+nearest-integer rules on arbitrary finite float32 groups spanning every binade.
 """
 import json
 import os
@@ -149,3 +150,64 @@ def test_flags_accumulate_over_groups():
     packed, scales, flags = oracle.quantize(w)
     assert flags == oracle.FLAG_NONFINITE | oracle.FLAG_SCALE_OVERFLOW
     assert scales[0, 0] == 0 and scales[2, 1] == 0 and scales[1, 0] == 0x3092
+
+
+# ---- property test over arbitrary finite float32 groups (hypothesis) ----------------------
+from hypothesis import given, settings, strategies as st  # noqa: E402
+from hypothesis.extra.numpy import arrays  # noqa: E402
+
+
+def _check_groups(w):
+    """Every group of w against definitions that do not use the oracle's float32 quotient:
+    the scale is numpy's binary16 cast of float32(amax) / 7 (a zero group, flagged, when
+    that overflows; a zero group when it is zero), and each code is the binary64 nearest
+    integer to w / s clamped to [-8, 7], except within 2^-19 of a half (where the float32
+    quotient's rounding decides) and within 2^-19 of a clamp end."""
+    packed, scales, flags = oracle.quantize(w)
+    G = w.shape[1] // 32
+    g32 = w.reshape(w.shape[0], G, 32)
+    amax = np.max(np.abs(g32), axis=2)                       # float32
+    with np.errstate(over="ignore"):
+        s16 = (amax / np.float32(7.0)).astype(np.float16)    # numpy's round-to-nearest-even cast
+    overflow = np.isinf(s16)
+    assert flags == (oracle.FLAG_SCALE_OVERFLOW if overflow.any() else 0)
+    codes = (_codes(packed) - 8).reshape(g32.shape)
+    zero = overflow | (s16 == 0)
+    assert np.all(scales[zero] == 0) and np.all(codes[zero] == 0)
+    live = ~zero
+    assert np.array_equal(scales[live], s16[live].view(np.uint16))
+    sf = np.where(live, s16.astype(np.float64), 1.0)
+    t = g32.astype(np.float64) / sf[..., None]
+    near = np.clip(np.rint(t), -8, 7)
+    frac = np.abs(t - np.floor(t) - 0.5)
+    decided = live[..., None] & (frac > 2.0 ** -19) & (np.abs(t - 7.5) > 2.0 ** -19) & (np.abs(t + 8.5) > 2.0 ** -19)
+    assert np.array_equal(codes[decided], near[decided])
+    # codes that the binary64 rule leaves open are one of the neighbours of the clamped quotient
+    open_ = live[..., None] & ~decided
+    assert np.all(np.abs(codes[open_] - np.clip(t[open_], -8, 7)) <= 0.5 + 2.0 ** -18)
+
+
+@st.composite
+def _wide_groups(draw):
+    """4 x 64 float32 weights, each group m_i 2^(e + d_i): mantissas uniform in [-1, 1] from a
+    drawn seed, a drawn group exponent e in [-27, 20] and offsets d_i in [-spread, 0] (spread
+    drawn up to 40), so that groups reach zero, subnormal and overflowing scales and hold
+    values many binades below their maximum."""
+    rng = np.random.default_rng(draw(st.integers(0, 2 ** 32 - 1)))
+    e = np.array(draw(st.lists(st.integers(-27, 20), min_size=8, max_size=8)), dtype=np.float64)
+    spread = draw(st.integers(0, 40))
+    m = rng.uniform(-1.0, 1.0, (4, 64))
+    d = rng.integers(-spread, 1, (4, 64))
+    return (m * np.exp2(np.repeat(e.reshape(4, 2), 32, axis=1) + d)).astype(np.float32)
+
+
+@settings(max_examples=300, deadline=None)
+@given(_wide_groups())
+def test_property_wide_range_groups(w):
+    _check_groups(w)
+
+
+@settings(max_examples=200, deadline=None)
+@given(arrays(np.float32, (2, 64), elements=st.floats(width=32, allow_nan=False, allow_infinity=False)))
+def test_property_any_finite_float32(w):
+    _check_groups(w)
