@@ -6,7 +6,8 @@ Checked against facts that do not go through the oracle's own code: the round-tr
 |w - w'| <= s/2 against the stored scale, exact reconstruction of weights already on the
 grid, zero groups, the clamp reached only through a binary16 scale rounded down, flags for
 non-finite input and scale overflow, and products against numpy's binary16 decoding with a
-torch binary64 matmul and a hand-summed brute force."""
+torch binary64 matmul and a hand-summed brute force; and (hypothesis) the scale and
+nearest-integer rules on arbitrary finite float32 groups spanning every binade."""
 import numpy as np
 import pytest
 import torch
@@ -98,3 +99,51 @@ def test_brute_force_dot_products_k32_k64():
         for n in range(2):
             exact = sum(Fraction(float(x[0, k])) * Fraction(int(c[n, k])) * Fraction(1, 64) for k in range(K))
             assert y[0, n] == float(exact)
+
+
+# ---- property test over arbitrary finite float32 groups (hypothesis) ----------------------
+from hypothesis import given, settings, strategies as st  # noqa: E402
+from hypothesis.extra.numpy import arrays  # noqa: E402
+
+from tests.test_oracle_quantize import _wide_groups  # noqa: E402
+
+
+def _check_groups8(w):
+    """Every group against definitions that do not use the oracle's float32 quotient: the
+    scale is numpy's binary16 cast of float32(amax) / 127 (zero group when it is zero or,
+    flagged, when it overflows) and each code is the binary64 nearest integer to w / s
+    clamped to [-128, 127], except within 2^-15 of a half or of a clamp end (float32
+    quotients near 128 carry ulps of 2^-16)."""
+    codes, scales, flags = oracle.quantize8(w)
+    G = w.shape[1] // 32
+    g32 = w.reshape(w.shape[0], G, 32)
+    amax = np.max(np.abs(g32), axis=2)
+    with np.errstate(over="ignore"):
+        s16 = (amax / np.float32(127.0)).astype(np.float16)
+    overflow = np.isinf(s16)
+    assert flags == (oracle.FLAG_SCALE_OVERFLOW if overflow.any() else 0)
+    c = codes.astype(np.int64).reshape(g32.shape)
+    zero = overflow | (s16 == 0)
+    assert np.all(scales[zero] == 0) and np.all(c[zero] == 0)
+    live = ~zero
+    assert np.array_equal(scales[live], s16[live].view(np.uint16))
+    t = g32.astype(np.float64) / np.where(live, s16.astype(np.float64), 1.0)[..., None]
+    near = np.clip(np.rint(t), -128, 127)
+    eps = 2.0 ** -15
+    decided = (live[..., None] & (np.abs(t - np.floor(t) - 0.5) > eps) & (np.abs(t - 127.5) > eps) &
+               (np.abs(t + 128.5) > eps))
+    assert np.array_equal(c[decided], near[decided])
+    open_ = live[..., None] & ~decided
+    assert np.all(np.abs(c[open_] - np.clip(t[open_], -128, 127)) <= 0.5 + 2 * eps)
+
+
+@settings(max_examples=300, deadline=None)
+@given(_wide_groups())
+def test_property_wide_range_groups(w):
+    _check_groups8(w)
+
+
+@settings(max_examples=200, deadline=None)
+@given(arrays(np.float32, (2, 64), elements=st.floats(width=32, allow_nan=False, allow_infinity=False)))
+def test_property_any_finite_float32(w):
+    _check_groups8(w)
